@@ -1,0 +1,112 @@
+"""Plant plausible mistakes in (a copy of) the oracle and check that a pin catches each.
+
+Each mutation replaces one exact fragment of ``oracle/grape_oracle.py`` and
+executes the result as a fresh module on the CPU; the real oracle is never
+modified.  A mutation passes this test when at least one pin in
+``pins.ALL_PINS`` fails (an assertion or any exception) on the mutated copy.
+"""
+import itertools
+import os
+import sys
+import types
+
+import pytest
+
+import pins
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                   "oracle", "grape_oracle.py")
+
+MUTATIONS = {
+    # Philox
+    "philox_multiplier": ("PHILOX_M0 = 0xD2511F53", "PHILOX_M0 = 0xD2511F55"),
+    "philox_rounds": ("PHILOX_ROUNDS = 10", "PHILOX_ROUNDS = 9"),
+    "philox_weyl": ("k1 = (k1 + np.uint64(PHILOX_W1))", "k1 = (k1 + np.uint64(PHILOX_W0))"),
+    "philox_round_mix": ("c = [hi1 ^ c[1] ^ k0, lo1, hi0 ^ c[3] ^ k1, lo0]",
+                         "c = [hi0 ^ c[1] ^ k0, lo1, hi1 ^ c[3] ^ k1, lo0]"),
+    "counter_layout": ("ctr[:, 1] = np.uint32(layer)\n    ctr[:, 2] = np.uint32(step)",
+                       "ctr[:, 1] = np.uint32(step)\n    ctr[:, 2] = np.uint32(layer)"),
+    # Box-Muller
+    "bm_open_interval": ("u1 = (xa.astype(np.float64) + 1.0)", "u1 = (xa.astype(np.float64) + 0.5)"),
+    "bm_sin_cos_swap": ("return rho * np.cos(2.0 * np.pi * u2), rho * np.sin(2.0 * np.pi * u2)",
+                        "return rho * np.sin(2.0 * np.pi * u2), rho * np.cos(2.0 * np.pi * u2)"),
+    "bm_half_angle": ("return rho * np.cos(2.0 * np.pi * u2), rho * np.sin(2.0 * np.pi * u2)",
+                      "return rho * np.cos(np.pi * u2), rho * np.sin(np.pi * u2)"),
+    "bm_pairing": ("z2, z3 = box_muller(w[:, 2], w[:, 3])", "z2, z3 = box_muller(w[:, 3], w[:, 2])"),
+    # projection matrix
+    "p_unscaled": ("STREAM_PROJECTION, d_in * r).reshape(d_in, r) / np.sqrt(r)",
+                   "STREAM_PROJECTION, d_in * r).reshape(d_in, r)"),
+    "p_scaled_by_r": ("STREAM_PROJECTION, d_in * r).reshape(d_in, r) / np.sqrt(r)",
+                      "STREAM_PROJECTION, d_in * r).reshape(d_in, r) / r"),
+    "p_column_major": ("STREAM_PROJECTION, d_in * r).reshape(d_in, r) / np.sqrt(r)",
+                       "STREAM_PROJECTION, d_in * r).reshape(r, d_in).T / np.sqrt(r)"),
+    "noise_stream": ("STREAM_NOISE, r * d_out)", "STREAM_PROJECTION, r * d_out)"),
+    # gradient and projection
+    "grad_token_misaligned": ("return A_i.T @ Gout_i", "return A_i.T @ Gout_i[::-1]"),
+    "project_transposed": ("return P.T @ G", "return (G.T @ P).T[::-1]"),
+    # clipping
+    "clip_inverted": ("return C / norm if norm > C else 1.0", "return min(1.0, norm / C)"),
+    "clip_always": ("return C / norm if norm > C else 1.0", "return C / norm if norm > 0 else 1.0"),
+    "norm_first_layer_only": ("np.sqrt(sum(np.sum(R[i][l] ** 2) for l in range(L)))",
+                              "np.sqrt(np.sum(R[i][0] ** 2))"),
+    "norm_not_sqrt": ("np.sqrt(sum(np.sum(R[i][l] ** 2) for l in range(L)))",
+                      "sum(np.sum(R[i][l] ** 2) for l in range(L))"),
+    "aggregate_unclipped": ("S_l = sum(c[i] * R[i][l] for i in range(B))",
+                            "S_l = sum(R[i][l] for i in range(B))"),
+    # noise and average
+    "noise_without_C": ("g = (S_l + h.sigma * h.C * xi) / div", "g = (S_l + h.sigma * xi) / div"),
+    "no_batch_average": ("g = (S_l + h.sigma * h.C * xi) / div", "g = (S_l + h.sigma * h.C * xi)"),
+    "noise_averaged_twice": ("g = (S_l + h.sigma * h.C * xi) / div",
+                             "g = S_l / div + h.sigma * h.C * xi / div / div"),
+    # Adam
+    "adam_no_bias_correction_m": ("m_hat = m / (1.0 - beta1 ** t)", "m_hat = m"),
+    "adam_no_bias_correction_v": ("v_hat = v / (1.0 - beta2 ** t)", "v_hat = v"),
+    "adam_eps_inside_sqrt": ("m_hat / (np.sqrt(v_hat) + eps)", "m_hat / np.sqrt(v_hat + eps)"),
+    "adam_v_not_squared": ("v = beta2 * v + (1.0 - beta2) * g * g", "v = beta2 * v + (1.0 - beta2) * g"),
+    "adam_betas_swapped": ("m = beta1 * m + (1.0 - beta1) * g", "m = beta2 * m + (1.0 - beta2) * g"),
+    "adam_t_zero_based": ("t = step_index + 1", "t = step_index + 2"),
+    # back-projection
+    "backproject_other_P": ("state.W[l] = state.W[l] - h.lr * (Ps[l] @ d)",
+                            "state.W[l] = state.W[l] - h.lr * (proj(l, step_index + 1, "
+                            "state.W[l].shape[0], h.r) @ d)"),
+    "backproject_sign": ("state.W[l] = state.W[l] - h.lr * (Ps[l] @ d)",
+                         "state.W[l] = state.W[l] + h.lr * (Ps[l] @ d)"),
+    "backproject_no_lr": ("state.W[l] = state.W[l] - h.lr * (Ps[l] @ d)",
+                          "state.W[l] = state.W[l] - (Ps[l] @ d)"),
+}
+
+# cheap pins first: a mutation stops at the first pin that fails
+ORDER = sorted(pins.ALL_PINS, key=lambda p: {
+    "pin_normal_statistics": 5, "pin_backprojection_unbiased": 6}.get(p.__name__, 0))
+
+
+_COUNT = itertools.count()
+
+
+def _mutant(old: str, new: str) -> types.ModuleType:
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"fragment not found exactly once: {old!r}"
+    name = f"grape_oracle_mutant_{next(_COUNT)}"
+    mod = types.ModuleType(name)
+    mod.__file__ = SRC
+    sys.modules[name] = mod          # dataclasses look their module up here
+    exec(compile(src.replace(old, new), SRC + "[mutant]", "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught(name):
+    mod = _mutant(*MUTATIONS[name])
+    for pin in ORDER:
+        try:
+            pin(mod)
+        except Exception:          # noqa: BLE001  any failure of a pin catches the mutation
+            return
+    pytest.fail(f"mutation {name!r} passed every pin")
+
+
+def test_unmutated_copy_passes_every_pin():
+    """The exec'd copy itself is faithful (guards the harness)."""
+    mod = _mutant("PHILOX_ROUNDS = 10", "PHILOX_ROUNDS = 10")
+    for pin in pins.ALL_PINS:
+        pin(mod)
