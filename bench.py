@@ -1,0 +1,446 @@
+#!/usr/bin/env python
+"""Throughput of the DP-GRAPE step on one node.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (default): four 1024 x 1024 linear layers, r = 128, B = 64 samples of
+T = 128 tokens, bf16 A and Gout, fp32 W and Adam moments (``workloads`` name
+``mlp4x1024``).  A "step" is one full pass of the method over one batch:
+regenerate P, project, per-sample norms, clip, aggregate, noise + projected
+Adam, back-projection onto W.  Inputs are synthetic (seeded, see ``workloads``)
+and rotate over several distinct per-step sets whose total is far larger than
+the 126 MB L2, each set alone already larger than L2.
+
+Prints one JSON line (rank 0).  With N > 1 (launched by torch.distributed.run)
+every rank runs its own B samples (weak scaling); the per-layer S is
+all-reduced over NCCL between aggregation and Adam.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as WL  # noqa: E402
+
+METRIC = "DP-GRAPE step samples/s (tokens/s) on 1 B200; % of tensor-pipe/HBM roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INPUT_SETS = 4
+
+
+def parse(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="mlp4x1024", choices=sorted(WL.WORKLOADS))
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------------------
+# clocks during the timed region (NVML, polled from a thread)
+# ---------------------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001
+            self.nv, self.err = None, str(e)
+
+    def _poll(self):
+        while not self._stop.is_set():
+            self.sample()
+            time.sleep(0.002)
+
+    def sample(self):
+        if not self.nv:
+            return
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for bit, name in self.REASONS.items():
+                if mask & bit:
+                    self.reasons.add(name)
+        except Exception:  # noqa: BLE001
+            pass
+
+    def __enter__(self):
+        self.t = threading.Thread(target=self._poll, daemon=True)
+        self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        self.t.join()
+        self.sample()
+
+    def summary(self):
+        if not self.nv:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "nvml unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------------------
+# roofline bookkeeping
+# ---------------------------------------------------------------------------------------
+
+def peaks():
+    try:
+        p = json.load(open(PEAKS_FILE))
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "sm_max_mhz": float(p.get("sm_max_mhz", 1965.0)), "source": "measured"}
+    except Exception:  # noqa: BLE001
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+def phase_work(w, path: str):
+    """Algorithmic bytes and flops of one launch of each phase (all layers in one call).
+
+    Bytes count each operand once at its storage width: the minimum traffic of that phase.
+    """
+    el = 4 if w.dtype == "f32" else 2
+    ap_el = 4 if path == "simt" else 2
+    dr_el = 4 if path == "simt" else 2
+    p_el = 4 if path == "simt" else 4          # tensor-core path writes P and P^T in bf16
+    rows = w.B * w.T
+    out = {}
+    out["gen_P"] = {"bytes": sum(di * w.r * p_el for di, _ in w.layers), "flops": 0}
+    out["project"] = {"bytes": sum(rows * di * el + rows * w.r * ap_el for di, _ in w.layers),
+                      "flops": sum(2 * rows * di * w.r for di, _ in w.layers)}
+    out["norm"] = {"bytes": sum(rows * do * el + rows * w.r * ap_el for _, do in w.layers),
+                   "flops": sum(2 * rows * w.r * do for _, do in w.layers)}
+    out["clip"] = {"bytes": 8 * w.B, "flops": 0}
+    out["aggregate"] = {"bytes": sum(rows * do * el + rows * w.r * ap_el + 4 * w.r * do
+                                     for _, do in w.layers),
+                        "flops": sum(2 * rows * w.r * do for _, do in w.layers)}
+    out["adam"] = {"bytes": sum(w.r * do * (4 + 16 + dr_el) for _, do in w.layers), "flops": 0}
+    out["backproject"] = {"bytes": sum(8 * di * do + di * w.r * ap_el + w.r * do * dr_el
+                                       for di, do in w.layers),
+                          "flops": sum(2 * di * w.r * do for di, do in w.layers)}
+    return out
+
+
+def step_work(w):
+    """The method's own work per step: FLOPs of the factored projection and back-projection,
+    bytes of A and Gout read once, W read + written, m and v read + written."""
+    el = 4 if w.dtype == "f32" else 2
+    flops = sum(2 * w.B * w.T * w.r * (di + do) + 2 * di * w.r * do for di, do in w.layers)
+    byts = sum(w.B * w.T * (di + do) * el + 8 * di * do + 16 * w.r * do for di, do in w.layers)
+    return flops, byts
+
+
+def kernel_source_sha(path: str) -> str:
+    name = "tc.cu" if path == "tc" else "simt.cu"
+    src = os.path.join(ROOT, "random_gradient_projection_b200", "csrc", name)
+    return hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str, path: str):
+    try:
+        t = json.load(open(TRAFFIC_FILE))
+    except Exception:  # noqa: BLE001
+        return None
+    rec = t.get(f"{path}:{kernel}:{workload}")
+    if not rec or rec.get("source_sha") != kernel_source_sha(path):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------------------
+# the oracle on the host cores (baseline arm and cpu_baseline)
+# ---------------------------------------------------------------------------------------
+
+def oracle_samples_per_s(w, target_s: float, max_steps: int = 1000, sub_batch=None):
+    """Time the fp64 oracle, as it stands, on samples of the workload's batch.
+
+    Each timed call is one oracle step over ``sub_batch`` samples (the whole batch by
+    default); calls repeat until ``target_s`` of CPU work has been timed.  Input drawing
+    is outside the timed calls.  Returns (samples/s, samples timed, seconds, threads)."""
+    import oracle.grape_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # noqa: BLE001
+        threads = os.cpu_count() or 1
+    nb = sub_batch or w.B
+    h = O.Hyper.of(w)
+    st = O.State.init(WL.make_weights(w), w.r)
+    done, spent, s = 0, 0.0, 0
+    while spent < target_s and s < max_steps:
+        x = WL.make_step_inputs(w, s, samples=list(range(nb)), threads=8)
+        A = [x.as_f64(a) for a in x.A]
+        G = [x.as_f64(g) for g in x.Gout]
+        t0 = time.perf_counter()
+        O.step(st, A, G, s, h)
+        spent += time.perf_counter() - t0
+        done += nb
+        s += 1
+    return done / spent, done, spent, threads
+
+
+def run_reference(args, rank: int, world: int):
+    """--impl reference: the fp64 oracle timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    w = WL.get(args.workload)
+    sub = max(1, min(w.B, 4))
+    # warm-up calls (untimed), then K timed calls of a bounded sub-batch each
+    oracle_samples_per_s(w, 0.0, max_steps=max(1, args.warmup), sub_batch=sub)
+    import oracle.grape_oracle as O
+    h = O.Hyper.of(w)
+    st = O.State.init(WL.make_weights(w), w.r)
+    times = []
+    for s in range(args.steps):
+        x = WL.make_step_inputs(w, s, samples=list(range(sub)), threads=8)
+        A = [x.as_f64(a) for a in x.A]
+        G = [x.as_f64(g) for g in x.Gout]
+        t0 = time.perf_counter()
+        O.step(st, A, G, s, h)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = sub * len(times) / total
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count() or 1
+    sample = f"{sub} of {w.B} samples per step, all {w.n_layers} layers, fp64 numpy oracle"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "samples/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "layers": f"{w.n_layers}x{w.layers[0][0]}x{w.layers[0][1]}",
+                   "r": w.r, "B": w.B, "T": w.T, "tokens_per_s": value * w.T},
+        "cpu_baseline": {"value": value, "unit": "samples/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "samples/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------
+
+def main(argv=None):
+    args = parse(argv)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return 0
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    import torch
+    import torch.distributed as dist
+    from random_gradient_projection_b200 import GrapeStep, grape
+    from random_gradient_projection_b200.data_parallel import dp_step
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    w = WL.get(args.workload)
+    path = {"auto": grape.GRAPE_PATH_AUTO, "simt": grape.GRAPE_PATH_SIMT,
+            "tc": grape.GRAPE_PATH_TC}[args.path]
+    g = GrapeStep.for_workload(w, path=path)
+    path_name = {grape.GRAPE_PATH_SIMT: "simt", grape.GRAPE_PATH_TC: "tc"}[g.path]
+    Wd = [torch.from_numpy(x).to(dev) for x in WL.make_weights(w)]
+
+    # distinct per-step input sets; ranks draw different samples (input seed only)
+    win = w.replace(seed=w.seed + 7919 * rank)
+    sets = []
+    for k in range(INPUT_SETS):
+        x = WL.make_step_inputs(win, k, threads=16)
+        conv = (lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)) \
+            if w.dtype == "bf16" else torch.from_numpy
+        sets.append(([conv(a).to(dev) for a in x.A], [conv(a).to(dev) for a in x.Gout]))
+    set_bytes = w.input_bytes()
+
+    def one(s):
+        A, G = sets[s % INPUT_SETS]
+        if world > 1:
+            dp_step(g, A, G, Wd, s)
+        else:
+            g.step(A, G, Wd, s)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    step = 0
+    for _ in range(args.warmup):
+        one(step)
+        step += 1
+    torch.cuda.synchronize()
+
+    # ---- timed region: exactly K steps --------------------------------------------------
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = g.launch_count()
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        e0.record(stream)
+        for _ in range(args.steps):
+            one(step)
+            step += 1
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    launches = g.launch_count() - launches0
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    samples_per_s = world * w.B * args.steps / (ms / 1e3)
+
+    # ---- per-phase device time (same K steps, events between phases) --------------------
+    g.profile(True)
+    for _ in range(args.steps):
+        one(step)
+        step += 1
+    phases = g.profile_read()
+    g.profile(False)
+
+    pk = peaks()
+    work = phase_work(w, path_name)
+    per_phase = {}
+    for name, (pms, calls) in phases.items():
+        if calls == 0:
+            continue
+        avg_s = pms / calls / 1e3
+        per_phase[name] = {"ms_per_launch": pms / calls, "share": None,
+                           "GB/s": work[name]["bytes"] / avg_s / 1e9,
+                           "TFLOP/s": work[name]["flops"] / avg_s / 1e12}
+    tot = sum(v["ms_per_launch"] for v in per_phase.values())
+    for v in per_phase.values():
+        v["share"] = v["ms_per_launch"] / tot if tot > 0 else None
+    dom = max(per_phase, key=lambda k: per_phase[k]["ms_per_launch"])
+    avg_s = per_phase[dom]["ms_per_launch"] / 1e3
+    if path_name == "tc":
+        bound, unit = "hbm", "GB/s"
+        achieved = work[dom]["bytes"] / avg_s / 1e9
+        peak = pk["hbm_gbs"]
+    else:
+        # fp32 FFMA on the CUDA cores: 148 SMs x 128 lanes x 2 flop x max SM clock
+        bound, unit = "alu", "TFLOP/s"
+        achieved = work[dom]["flops"] / avg_s / 1e12
+        peak = 148 * 128 * 2 * pk["sm_max_mhz"] * 1e6 / 1e12
+    traffic = traffic_for(dom, w.name, path_name)
+    flops, byts = step_work(w)
+    t_roof = max(flops / (pk["bf16_tflops"] * 1e12), byts / (pk["hbm_gbs"] * 1e9))
+
+    # ---- end to end through the public API: host buffers, copies in the timed region ----
+    e2e = None
+    if args.e2e_steps > 0:
+        x = WL.make_step_inputs(win, 0, threads=16)
+        hostA = [torch.from_numpy(a.view(np.int16) if w.dtype == "bf16" else a).pin_memory()
+                 for a in x.A]
+        hostG = [torch.from_numpy(a.view(np.int16) if w.dtype == "bf16" else a).pin_memory()
+                 for a in x.Gout]
+        norms = torch.empty(w.B, dtype=torch.float32).pin_memory()
+        g.step_host(hostA, hostG, Wd, step, norms)    # first call allocates the staging
+        step += 1
+        barrier()
+        t0 = time.perf_counter()
+        for _ in range(args.e2e_steps):
+            g.step_host(hostA, hostG, Wd, step, norms)   # synchronises its stream
+            step += 1
+        el = time.perf_counter() - t0
+        if world > 1:
+            t = torch.tensor([el], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            el = float(t.item())
+        e2e = {"value": world * w.B * args.e2e_steps / el, "unit": "samples/s",
+               "h2d_bytes_per_step": set_bytes, "d2h_bytes_per_step": 4 * w.B,
+               "steps": args.e2e_steps, "note": "grape_step_host: pinned host A/Gout copied in, "
+                                                "per-sample norms copied out, every step"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, n, secs, cores = oracle_samples_per_s(w, args.cpu_seconds)
+        cpu = {"value": v, "unit": "samples/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n} samples ({n // w.B} full steps of B={w.B}) of {w.name}, "
+                         f"{secs:.1f} s of fp64 numpy oracle time"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": samples_per_s, "unit": "samples/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "layers": f"{w.n_layers}x{w.layers[0][0]}x{w.layers[0][1]}",
+                       "r": w.r, "B_per_gpu": w.B, "global_batch": w.B * world, "T": w.T,
+                       "path": path_name, "parallelism": f"dp{world}",
+                       "l2": f"inputs rotate over {INPUT_SETS} distinct sets of "
+                             f"{set_bytes / 1e6:.0f} MB each (> 126 MB L2)",
+                       "tokens_per_s": samples_per_s * w.T},
+            "roofline": {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,
+                         "unit": unit, "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": pk["source"] if bound != "alu" else
+                         "derived: 148 SMs x 128 FP32 lanes x 2 x max SM clock"},
+            "step_roofline": {"t_roof_us": t_roof * 1e6, "frac": t_roof / (ms_per_step / 1e3),
+                              "flops": flops, "bytes": byts, "peaks": pk["source"]},
+            "phases": per_phase,
+            "gpu_launches": launches,
+            "clocks": sampler.summary(),
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    g.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,199 @@
+/*
+ * grape.h: C ABI of the B200 (sm_100a) DP-GRAPE projection step.
+ *
+ * The method ("Memory-Efficient Differentially Private Training with Gradient
+ * Random Projection", gist.science/es/paper/2506.15588, Resumen Tecnico,
+ * section "Metodologia: DP-GRAPE"): per linear layer l with weights
+ * W_l (d_in x d_out), every sample's gradient G_i = A_i^T Gout_i is projected
+ * onto a Gaussian matrix P_l (d_in x r) regenerated from a seed (design
+ * choice 1), the projection comes before clipping and noise (design choice 2),
+ * and Adam's moments live in the projected r x d_out space (design choice 3).
+ * One step, as the closing paragraph of that section orders it:
+ *
+ *   P_l[k,j]  = z(seed, l, s, stream 0, e = k*r + j) / sqrt(r)
+ *   R_{i,l}   = (A_{i,l} P_l)^T Gout_{i,l}              (G_i never formed)
+ *   n_i       = sqrt(sum_l ||R_{i,l}||_F^2),  c_i = C/n_i if n_i > C else 1
+ *   S_l       = sum_i c_i R_{i,l}
+ *   g_l       = (S_l + sigma*C*xi_l) / B,  xi_l[j,n] = z(seed, l, s, stream 1, e = j*d_out + n)
+ *   m, v      = Adam moments of g_l (r x d_out),  t = s + 1
+ *   dR_l      = (m/(1-beta1^t)) / (sqrt(v/(1-beta2^t)) + eps)
+ *   W_l      -= lr * P_l dR_l
+ *
+ * z(...) is a standard normal from Philox4x32-10 (Salmon et al., "Parallel
+ * Random Numbers: As Easy as 1, 2, 3", SC'11) with key (seed lo, seed hi) and
+ * counter (e/4, layer, step, stream), and Box-Muller: words (x0, x1) give
+ * elements 4q, 4q+1 (cosine, sine), words (x2, x3) give 4q+2, 4q+3, with
+ * u1 = (x_a + 1)/2^32 and u2 = x_b/2^32.
+ *
+ * Conventions
+ *  - Every device pointer is a CUDA device address on the context's device;
+ *    host pointers are ordinary (preferably pinned) host memory.
+ *  - Matrices are row-major.  A_l is B x T x d_in, Gout_l is B x T x d_out
+ *    (samples contiguous, each sample's T token rows contiguous), in the
+ *    context's input dtype (fp32, or bf16 as raw 16-bit patterns).  W_l is
+ *    fp32 d_in x d_out.  Every device pointer must be 16-byte aligned.
+ *  - The caller owns A, Gout, W and the stream; W is updated in place.  The
+ *    library owns the Adam moments, the per-step projection scratch, the
+ *    norms and the workspace, all allocated by grape_create and freed by
+ *    grape_destroy.
+ *  - All work is enqueued on the caller's stream; no call synchronises the
+ *    device unless its comment says so.  Asynchronous faults surface as
+ *    GRAPE_ECUDA from a later call.
+ *  - Every function returns GRAPE_OK (0) or an error code; the reason is kept
+ *    for grape_last_error(ctx).  A failed call leaves W, m and v unchanged
+ *    unless it returns GRAPE_ECUDA.
+ */
+#ifndef GRAPE_H_
+#define GRAPE_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GRAPE_API __attribute__((visibility("default")))
+#else
+#define GRAPE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GRAPE_OK 0
+#define GRAPE_EINVAL 1        /* bad argument: null/misaligned pointer, bad size */
+#define GRAPE_ENOMEM 2        /* device or host allocation failed */
+#define GRAPE_ECUDA 3         /* a CUDA call failed (message in grape_last_error) */
+#define GRAPE_ETIMEOUT 4      /* a bounded device-side wait gave up */
+#define GRAPE_EUNSUPPORTED 5  /* the configuration has no kernel on this device */
+
+#define GRAPE_MAX_LAYERS 64
+
+enum grape_dtype { GRAPE_F32 = 0, GRAPE_BF16 = 1 };
+
+/* Kernel family.  AUTO picks the tensor-core (tcgen05) path for bf16 inputs
+ * and the fp32 CUDA-core path for fp32 inputs.  SIMT forces the fp32
+ * CUDA-core kernels (exact fp32 arithmetic, any shape).  TC forces the
+ * tcgen05 path and fails with GRAPE_EUNSUPPORTED where it does not apply. */
+enum grape_path { GRAPE_PATH_AUTO = 0, GRAPE_PATH_SIMT = 1, GRAPE_PATH_TC = 2 };
+
+typedef struct grape_ctx grape_ctx;                 /* opaque, library-owned */
+typedef struct { int32_t d_in, d_out; } grape_layer;
+typedef struct { double lr, beta1, beta2, eps; } grape_adam;
+
+/* Create a context for a fixed stack of linear layers and a fixed batch shape.
+ *  layers[n_layers]  layer shapes (1 <= n_layers <= GRAPE_MAX_LAYERS)
+ *  r                 projection dimension, 1 <= r <= d_in of every layer
+ *                    (reading: the pages only say r << d)
+ *  C, sigma          clipping threshold (> 0) and noise multiplier (>= 0)
+ *  seed              64-bit seed of the projection and noise streams
+ *  adam              lr, beta1, beta2 in [0, 1), eps > 0
+ *                    (scalars are taken in double; derived constants such as
+ *                    1 - beta are formed in double before the kernels round
+ *                    them to fp32)
+ *  B, T              samples per batch and tokens per sample (>= 1)
+ *  in_dtype          GRAPE_F32 or GRAPE_BF16 (A and Gout)
+ *  path              enum grape_path
+ * Allocates the Adam moments (zeroed) and the workspace on the current CUDA
+ * device; synchronises that device once.  *out receives the handle. */
+GRAPE_API int grape_create(const grape_layer* layers, int32_t n_layers, int32_t r, double C, double sigma,
+                 uint64_t seed, const grape_adam* adam, int32_t B, int32_t T, int32_t in_dtype,
+                 int32_t path, grape_ctx** out);
+
+/* One full step s = step (>= 0; Adam uses t = s + 1) on `stream`
+ * (a cudaStream_t, NULL = default stream).
+ *  A[l], Gout[l]  device pointers of layer l's inputs (read only)
+ *  W[l]           device pointer of layer l's fp32 weights (updated in place) */
+GRAPE_API int grape_step(grape_ctx* ctx, const void* const* A, const void* const* Gout, float* const* W,
+               int64_t step, void* stream);
+
+/* The same step from HOST buffers: A and Gout are copied to library-owned
+ * device staging on `stream` (allocated on first use), the step runs, and
+ * the B per-sample norms n_i are copied to norms_host (may be NULL).  W
+ * stays on the device.  Synchronises `stream` before returning, so the host
+ * buffers may be reused and norms_host is valid on return. */
+GRAPE_API int grape_step_host(grape_ctx* ctx, const void* const* A_host, const void* const* Gout_host,
+                    float* const* W, int64_t step, float* norms_host, void* stream);
+
+/* The data-parallel split of grape_step.  grape_accumulate runs the
+ * projection, the per-sample norms, clipping and the aggregation, leaving
+ * S_l = sum_i c_i R_{i,l} (fp32, r x d_out, row-major) in library memory,
+ * whose device address grape_S_ptr returns.  A caller may all-reduce (sum)
+ * every S_l across ranks, then grape_apply adds the noise, divides by
+ * batch_total (the global batch; 0 means B), runs Adam and back-projects
+ * onto W.  grape_step(ctx, ...) equals accumulate + apply(batch_total = B). */
+GRAPE_API int grape_accumulate(grape_ctx* ctx, const void* const* A, const void* const* Gout, int64_t step,
+                     void* stream);
+GRAPE_API int grape_S_ptr(grape_ctx* ctx, int32_t layer, float** S_dev);
+GRAPE_API int grape_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_total, void* stream);
+
+/* Checkpoint / resume of the projected Adam moments of one layer (r x d_out
+ * fp32 each, device pointers), enqueued on `stream`.  P is not state: it is
+ * regenerated from (seed, layer, step). */
+GRAPE_API int grape_get_state(grape_ctx* ctx, int32_t layer, float* m_dev, float* v_dev, void* stream);
+GRAPE_API int grape_set_state(grape_ctx* ctx, int32_t layer, const float* m_dev, const float* v_dev,
+                    void* stream);
+
+/* Intermediates of the last step, copied to host memory (synchronises the
+ * context's device).  what: */
+enum grape_debug_what {
+  GRAPE_DBG_NORMS = 0,   /* B floats: n_i */
+  GRAPE_DBG_CLIP = 1,    /* B floats: c_i */
+  GRAPE_DBG_S = 2,       /* r x d_out floats of `layer` */
+  GRAPE_DBG_P = 3,       /* d_in x r floats of `layer`, as used by the last step */
+  GRAPE_DBG_DR = 4,      /* r x d_out floats of `layer`: the Adam direction */
+  GRAPE_DBG_M = 5,       /* r x d_out floats of `layer` */
+  GRAPE_DBG_V = 6        /* r x d_out floats of `layer` */
+};
+GRAPE_API int grape_debug(grape_ctx* ctx, int32_t what, int32_t layer, void* host_out);
+
+/* Measurement.  While profiling is on, every phase of every step is bracketed
+ * by two CUDA events recorded on the step's stream; grape_profile_read
+ * synchronises the device and returns, per phase, the summed milliseconds and
+ * the number of bracketed calls since profiling was switched on (then starts
+ * the sums again).  ms_out and count_out hold GRAPE_N_PHASES entries each
+ * (either may be NULL).  grape_launch_count returns how many kernels the
+ * context has launched since it was created. */
+enum grape_phase {
+  GRAPE_PHASE_GEN_P = 0,        /* regenerate P from (seed, layer, step) */
+  GRAPE_PHASE_PROJECT = 1,      /* AP = A P over the stacked rows */
+  GRAPE_PHASE_NORM = 2,         /* R_i = (A_i P)^T Gout_i and its squared norm */
+  GRAPE_PHASE_CLIP = 3,         /* n_i and c_i */
+  GRAPE_PHASE_AGGREGATE = 4,    /* S = sum_i c_i R_i */
+  GRAPE_PHASE_ADAM = 5,         /* noise + projected Adam */
+  GRAPE_PHASE_BACKPROJECT = 6,  /* W -= lr P dR */
+  GRAPE_N_PHASES = 7
+};
+GRAPE_API int grape_profile(grape_ctx* ctx, int32_t enable);
+GRAPE_API int grape_profile_read(grape_ctx* ctx, double* ms_out, int64_t* count_out);
+GRAPE_API int grape_launch_count(const grape_ctx* ctx, uint64_t* launches);
+
+/* Bytes of device memory the context holds (moments + workspace). */
+GRAPE_API int grape_device_bytes(const grape_ctx* ctx, uint64_t* bytes);
+
+/* Which kernel family the context runs (enum grape_path, never AUTO). */
+GRAPE_API int grape_path_of(const grape_ctx* ctx, int32_t* path);
+
+/* Reason of the last failure on this context ("" if none).  Valid until the
+ * next call on ctx. */
+GRAPE_API const char* grape_last_error(const grape_ctx* ctx);
+
+/* Reason of the last failure of a call without a context (grape_create,
+ * the generator entry points).  Thread-local. */
+GRAPE_API const char* grape_global_error(void);
+
+GRAPE_API void grape_destroy(grape_ctx* ctx);
+
+/* The method's generator on its own (Salmon et al. SC'11 Philox4x32-10 and
+ * Box-Muller as above), for checking it against other implementations.
+ *  grape_philox_words: out_dev[4q + w] = word w of counter (q, layer, step,
+ *      stream) for q = 0 .. n_blocks-1 (uint32 device buffer, 4*n_blocks words).
+ *  grape_gaussian: out_dev[e] = z(seed, layer, step, stream, e), e < n (fp32). */
+GRAPE_API int grape_philox_words(uint64_t seed, uint32_t layer, uint32_t step, uint32_t stream_id,
+                       int64_t n_blocks, uint32_t* out_dev, void* stream);
+GRAPE_API int grape_gaussian(uint64_t seed, uint32_t layer, uint32_t step, uint32_t stream_id, int64_t n,
+                   float* out_dev, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GRAPE_H_ */

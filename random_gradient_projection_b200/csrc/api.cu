@@ -1,0 +1,644 @@
+// C ABI of the DP-GRAPE step: context, validation, workspace and the order of the
+// phases (see include/grape.h for the contract of every entry point).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/grape.h"
+#include "kernels.h"
+#include "tc.h"
+
+namespace {
+
+thread_local std::string g_global_error;
+
+int set_global(int code, const std::string& msg) {
+  g_global_error = msg;
+  return code;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Test hook: GRAPE_FAULT_ALLOC=n makes the n-th device allocation of a context fail.
+int fault_alloc_index() {
+  const char* s = std::getenv("GRAPE_FAULT_ALLOC");
+  return s ? std::atoi(s) : 0;
+}
+
+}  // namespace
+
+struct grape_ctx {
+  grape::StepShape sh{};
+  int path = GRAPE_PATH_SIMT;  // resolved (never AUTO)
+  int device = 0;
+  std::vector<grape_layer> layers;
+  std::vector<grape::LayerWs> ws;
+  void* arena = nullptr;
+  size_t arena_bytes = 0;
+  float* partials = nullptr;
+  float* norms = nullptr;
+  float* clip = nullptr;
+  grape::TcWorkspace tc{};
+  // staging for grape_step_host (allocated on first use)
+  std::vector<void*> stage_A, stage_G;
+  int64_t last_step = -1;
+  double beta1 = 0.9, beta2 = 0.999;   // as given (bias corrections are formed in double)
+  std::string err;
+  // measurement
+  bool prof_on = false;
+  std::vector<cudaEvent_t> ev_pool;
+  size_t ev_used = 0;
+  struct Mark { int phase; cudaEvent_t a, b; };
+  std::vector<Mark> marks;
+  uint64_t launches = 0;
+
+  cudaEvent_t next_event() {
+    if (ev_used == ev_pool.size()) {
+      cudaEvent_t e = nullptr;
+      if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+      ev_pool.push_back(e);
+    }
+    return ev_pool[ev_used++];
+  }
+
+  int fail(int code, const std::string& msg) {
+    err = msg;
+    return code;
+  }
+  int cuda_fail(cudaError_t e, const char* where) {
+    err = std::string(where) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
+    return GRAPE_ECUDA;
+  }
+};
+
+namespace {
+
+struct Arena {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) & ~static_cast<size_t>(255);
+    return o;
+  }
+};
+
+size_t in_elsize(int dtype) { return dtype == GRAPE_BF16 ? 2 : 4; }
+
+int validate_io(grape_ctx* ctx, const void* const* A, const void* const* G, float* const* W,
+                bool need_ag, bool need_w) {
+  if (need_ag && (!A || !G)) return ctx->fail(GRAPE_EINVAL, "A and Gout arrays must not be null");
+  if (need_w && !W) return ctx->fail(GRAPE_EINVAL, "W array must not be null");
+  for (int l = 0; l < ctx->sh.L; ++l) {
+    if (need_ag) {
+      if (!A[l] || !G[l])
+        return ctx->fail(GRAPE_EINVAL, "A[" + std::to_string(l) + "] or Gout[" + std::to_string(l) +
+                                           "] is null");
+      if (!aligned16(A[l]) || !aligned16(G[l]))
+        return ctx->fail(GRAPE_EINVAL, "A/Gout of layer " + std::to_string(l) +
+                                           " not 16-byte aligned");
+    }
+    if (need_w) {
+      if (!W[l]) return ctx->fail(GRAPE_EINVAL, "W[" + std::to_string(l) + "] is null");
+      if (!aligned16(W[l]))
+        return ctx->fail(GRAPE_EINVAL, "W of layer " + std::to_string(l) + " not 16-byte aligned");
+    }
+  }
+  return GRAPE_OK;
+}
+
+int check_step_index(grape_ctx* ctx, int64_t step) {
+  if (step < 0 || step > 0xFFFFFFFFll)
+    return ctx->fail(GRAPE_EINVAL, "step must be in [0, 2^32)");
+  return GRAPE_OK;
+}
+
+// Run one phase: launch it, count its kernels and, when profiling, bracket it
+// with two events on the step's stream.
+template <class F>
+int phase(grape_ctx* ctx, int id, const char* what, cudaStream_t st, F&& launch) {
+  cudaEvent_t a = nullptr;
+  if (ctx->prof_on) {
+    a = ctx->next_event();
+    if (!a) return ctx->fail(GRAPE_ECUDA, "cudaEventCreate failed");
+    cudaEventRecord(a, st);
+  }
+  int n = 0;
+  const cudaError_t e = launch(&n);
+  if (e != cudaSuccess) return ctx->cuda_fail(e, what);
+  ctx->launches += static_cast<uint64_t>(n);
+  if (ctx->prof_on) {
+    cudaEvent_t b = ctx->next_event();
+    if (!b) return ctx->fail(GRAPE_ECUDA, "cudaEventCreate failed");
+    cudaEventRecord(b, st);
+    ctx->marks.push_back({id, a, b});
+  }
+  return GRAPE_OK;
+}
+
+int run_accumulate(grape_ctx* ctx, const void* const* A, const void* const* G, int64_t step,
+                   cudaStream_t st) {
+  std::vector<grape::LayerIo> io(ctx->sh.L);
+  for (int l = 0; l < ctx->sh.L; ++l) io[l] = grape::LayerIo{A[l], G[l], nullptr};
+  const grape::StepShape& sh = ctx->sh;
+  const grape::LayerWs* ws = ctx->ws.data();
+  const uint32_t s = static_cast<uint32_t>(step);
+  int rc;
+  if (ctx->path == GRAPE_PATH_TC) {
+    const grape::TcWorkspace& tc = ctx->tc;
+    rc = phase(ctx, GRAPE_PHASE_GEN_P, "generate P", st,
+               [&](int* n) { return grape::tc_generate_P(sh, ws, tc, s, st, n); });
+    if (rc) return rc;
+    rc = phase(ctx, GRAPE_PHASE_PROJECT, "project", st,
+               [&](int* n) { return grape::tc_project(sh, ws, io.data(), tc, st, n); });
+    if (rc) return rc;
+    rc = phase(ctx, GRAPE_PHASE_NORM, "per-sample norms", st, [&](int* n) {
+      return grape::tc_project_norm(sh, ws, io.data(), tc, ctx->partials, st, n);
+    });
+    if (rc) return rc;
+  } else {
+    rc = phase(ctx, GRAPE_PHASE_GEN_P, "generate P", st, [&](int* n) {
+      *n = 1;
+      return grape::simt_generate_P(sh, ws, s, st);
+    });
+    if (rc) return rc;
+    rc = phase(ctx, GRAPE_PHASE_PROJECT, "project", st, [&](int* n) {
+      *n = 1;
+      return grape::simt_project_ap(sh, ws, io.data(), st);
+    });
+    if (rc) return rc;
+    rc = phase(ctx, GRAPE_PHASE_NORM, "per-sample norms", st, [&](int* n) {
+      *n = 1;
+      return grape::simt_project_norm(sh, ws, io.data(), ctx->partials, st);
+    });
+    if (rc) return rc;
+  }
+  rc = phase(ctx, GRAPE_PHASE_CLIP, "clip", st, [&](int* n) {
+    if (ctx->path == GRAPE_PATH_TC)
+      return grape::tc_clip_scale(sh, ws, ctx->tc, ctx->partials, ctx->norms, ctx->clip, st, n);
+    *n = 1;
+    return grape::finalize_clip(sh, ctx->partials, ctx->norms, ctx->clip, st);
+  });
+  if (rc) return rc;
+  if (ctx->path == GRAPE_PATH_TC) {
+    rc = phase(ctx, GRAPE_PHASE_AGGREGATE, "aggregate", st, [&](int* n) {
+      return grape::tc_aggregate(sh, ws, io.data(), ctx->tc, ctx->clip, st, n);
+    });
+  } else {
+    rc = phase(ctx, GRAPE_PHASE_AGGREGATE, "aggregate", st, [&](int* n) {
+      *n = 1;
+      return grape::simt_aggregate(sh, ws, io.data(), ctx->clip, st);
+    });
+  }
+  if (rc) return rc;
+  ctx->last_step = step;
+  return GRAPE_OK;
+}
+
+int run_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_total, cudaStream_t st) {
+  const int64_t bt = batch_total > 0 ? batch_total : ctx->sh.B;
+  const double t = static_cast<double>(step) + 1.0;
+  grape::UpdateScalars u{};
+  u.step = static_cast<uint32_t>(step);
+  u.inv_batch = static_cast<float>(1.0 / static_cast<double>(bt));
+  u.inv_bc1 = static_cast<float>(1.0 / (1.0 - std::pow(ctx->beta1, t)));
+  u.inv_bc2 = static_cast<float>(1.0 / (1.0 - std::pow(ctx->beta2, t)));
+  std::vector<grape::LayerIo> io(ctx->sh.L);
+  for (int l = 0; l < ctx->sh.L; ++l) io[l] = grape::LayerIo{nullptr, nullptr, W[l]};
+  const bool tc = ctx->path == GRAPE_PATH_TC;
+  const grape::StepShape& sh = ctx->sh;
+  const grape::LayerWs* ws = ctx->ws.data();
+  int rc = phase(ctx, GRAPE_PHASE_ADAM, "noise + adam", st, [&](int* n) {
+    *n = 1;
+    return grape::noise_adam(sh, ws, u, tc, st);
+  });
+  if (rc) return rc;
+  return phase(ctx, GRAPE_PHASE_BACKPROJECT, "back-project", st, [&](int* n) {
+    if (tc) return grape::tc_backproject(sh, ws, io.data(), ctx->tc, sh.lr, st, n);
+    *n = 1;
+    return grape::simt_backproject(sh, ws, io.data(), sh.lr, st);
+  });
+}
+
+// After a device synchronisation: a tensor-core wait that gave up leaves a nonzero word.
+int check_device_error(grape_ctx* ctx) {
+  if (ctx->path != GRAPE_PATH_TC) return GRAPE_OK;
+  int* word = grape::tc_error_word(ctx->tc);
+  if (!word) return GRAPE_OK;
+  int v = 0;
+  cudaError_t e = cudaMemcpy(&v, word, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return ctx->cuda_fail(e, "read error word");
+  if (v != 0) {
+    cudaMemset(word, 0, sizeof(int));
+    return ctx->fail(GRAPE_ETIMEOUT, "a tensor-core kernel gave up waiting (code " +
+                                         std::to_string(v) + ")");
+  }
+  return GRAPE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int grape_create(const grape_layer* layers, int32_t n_layers, int32_t r, double C, double sigma,
+                 uint64_t seed, const grape_adam* adam, int32_t B, int32_t T, int32_t in_dtype,
+                 int32_t path, grape_ctx** out) {
+  if (!out) return set_global(GRAPE_EINVAL, "out must not be null");
+  *out = nullptr;
+  if (!layers) return set_global(GRAPE_EINVAL, "layers must not be null");
+  if (!adam) return set_global(GRAPE_EINVAL, "adam must not be null");
+  if (n_layers < 1 || n_layers > GRAPE_MAX_LAYERS)
+    return set_global(GRAPE_EINVAL, "n_layers must be in [1, " + std::to_string(GRAPE_MAX_LAYERS) + "]");
+  if (B < 1 || T < 1) return set_global(GRAPE_EINVAL, "B and T must be >= 1");
+  if (r < 1) return set_global(GRAPE_EINVAL, "r must be >= 1");
+  if (!(C > 0.0) || !std::isfinite(C)) return set_global(GRAPE_EINVAL, "C must be finite and > 0");
+  if (!(sigma >= 0.0) || !std::isfinite(sigma)) return set_global(GRAPE_EINVAL, "sigma must be finite and >= 0");
+  if (!(adam->lr >= 0.0) || !(adam->beta1 >= 0.0 && adam->beta1 < 1.0) ||
+      !(adam->beta2 >= 0.0 && adam->beta2 < 1.0) || !(adam->eps > 0.0))
+    return set_global(GRAPE_EINVAL, "adam: need lr >= 0, beta1 and beta2 in [0, 1), eps > 0");
+  if (in_dtype != GRAPE_F32 && in_dtype != GRAPE_BF16)
+    return set_global(GRAPE_EINVAL, "in_dtype must be GRAPE_F32 or GRAPE_BF16");
+  if (path < GRAPE_PATH_AUTO || path > GRAPE_PATH_TC)
+    return set_global(GRAPE_EINVAL, "path must be a grape_path value");
+  for (int l = 0; l < n_layers; ++l) {
+    if (layers[l].d_in < 1 || layers[l].d_out < 1)
+      return set_global(GRAPE_EINVAL, "layer " + std::to_string(l) + ": d_in and d_out must be >= 1");
+    if (r > layers[l].d_in)
+      return set_global(GRAPE_EINVAL, "layer " + std::to_string(l) + ": r must be <= d_in");
+  }
+  if (static_cast<int64_t>(B) * T > (int64_t{1} << 31) / 4)
+    return set_global(GRAPE_EINVAL, "B*T too large");
+
+  int resolved = path;
+  if (resolved == GRAPE_PATH_AUTO) resolved = (in_dtype == GRAPE_BF16) ? GRAPE_PATH_TC : GRAPE_PATH_SIMT;
+  if (resolved == GRAPE_PATH_TC && in_dtype != GRAPE_BF16)
+    return set_global(GRAPE_EUNSUPPORTED, "the tensor-core path takes bf16 inputs");
+
+  int dev = 0;
+  cudaError_t ce = cudaGetDevice(&dev);
+  if (ce != cudaSuccess) return set_global(GRAPE_ECUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(ce));
+  if (resolved == GRAPE_PATH_TC) {
+    std::string why;
+    if (!grape::tc_supported(dev, layers, n_layers, r, B, T, &why)) {
+      if (path == GRAPE_PATH_TC) return set_global(GRAPE_EUNSUPPORTED, why);
+      return set_global(GRAPE_EUNSUPPORTED, "bf16 inputs need the tensor-core path: " + why);
+    }
+  }
+
+  grape_ctx* ctx = new grape_ctx();
+  ctx->device = dev;
+  ctx->path = resolved;
+  ctx->layers.assign(layers, layers + n_layers);
+  grape::StepShape& sh = ctx->sh;
+  sh.L = n_layers;
+  sh.r = r;
+  sh.B = B;
+  sh.T = T;
+  sh.dtype = in_dtype;
+  sh.seed = seed;
+  sh.C = static_cast<float>(C);
+  sh.sigma_C = static_cast<float>(sigma * C);
+  sh.lr = static_cast<float>(adam->lr);
+  sh.beta1 = static_cast<float>(adam->beta1);
+  sh.beta2 = static_cast<float>(adam->beta2);
+  sh.one_minus_beta1 = static_cast<float>(1.0 - adam->beta1);
+  sh.one_minus_beta2 = static_cast<float>(1.0 - adam->beta2);
+  sh.eps = static_cast<float>(adam->eps);
+  ctx->beta1 = adam->beta1;
+  ctx->beta2 = adam->beta2;
+
+  const bool tc = resolved == GRAPE_PATH_TC;
+  const size_t ap_el = tc ? 2 : 4;
+  Arena ar;
+  struct Offs { size_t P32, Pt16, P16, AP, S, m, v, dR; };
+  std::vector<Offs> offs(n_layers);
+  int part = 0;
+  ctx->ws.resize(n_layers);
+  for (int l = 0; l < n_layers; ++l) {
+    const size_t di = layers[l].d_in, dout = layers[l].d_out;
+    Offs& o = offs[l];
+    o.P32 = tc ? SIZE_MAX : ar.take(di * r * 4);
+    o.Pt16 = tc ? ar.take(di * r * 2) : SIZE_MAX;
+    o.P16 = tc ? ar.take(di * r * 2) : SIZE_MAX;
+    o.AP = ar.take(static_cast<size_t>(B) * T * r * ap_el);
+    o.S = ar.take(r * dout * 4);
+    o.m = ar.take(r * dout * 4);
+    o.v = ar.take(r * dout * 4);
+    o.dR = ar.take(r * dout * (tc ? 2 : 4));
+    grape::LayerWs& w = ctx->ws[l];
+    w.d_in = layers[l].d_in;
+    w.d_out = layers[l].d_out;
+    w.part_base = part;
+    w.part_count = tc ? grape::tc_partials_per_sample(r, layers[l].d_out)
+                      : grape::simt_partials_per_sample(r, layers[l].d_out);
+    part += w.part_count;
+  }
+  sh.part_stride = part;
+  const size_t off_part = ar.take(static_cast<size_t>(B) * part * 4);
+  const size_t off_norms = ar.take(static_cast<size_t>(B) * 4);
+  const size_t off_clip = ar.take(static_cast<size_t>(B) * 4);
+  size_t off_tc = 0;
+  size_t tc_bytes = tc ? grape::tc_workspace_bytes(sh, ctx->ws.data()) : 0;
+  if (tc) off_tc = ar.take(tc_bytes);
+  ctx->arena_bytes = ar.off;
+
+  const int fault = fault_alloc_index();
+  if (fault == 1) {
+    delete ctx;
+    return set_global(GRAPE_ENOMEM, "device allocation failed (GRAPE_FAULT_ALLOC)");
+  }
+  ce = cudaMalloc(&ctx->arena, ctx->arena_bytes);
+  if (ce != cudaSuccess) {
+    delete ctx;
+    cudaGetLastError();
+    return set_global(GRAPE_ENOMEM, "cudaMalloc of " + std::to_string(ar.off) + " bytes: " + cudaGetErrorString(ce));
+  }
+  char* base = static_cast<char*>(ctx->arena);
+  auto at = [&](size_t o) -> char* { return o == SIZE_MAX ? nullptr : base + o; };
+  for (int l = 0; l < n_layers; ++l) {
+    grape::LayerWs& w = ctx->ws[l];
+    const Offs& o = offs[l];
+    w.P32 = reinterpret_cast<float*>(at(o.P32));
+    w.Pt16 = reinterpret_cast<__nv_bfloat16*>(at(o.Pt16));
+    w.P16 = reinterpret_cast<__nv_bfloat16*>(at(o.P16));
+    w.AP = at(o.AP);
+    w.S = reinterpret_cast<float*>(at(o.S));
+    w.m = reinterpret_cast<float*>(at(o.m));
+    w.v = reinterpret_cast<float*>(at(o.v));
+    w.dR = at(o.dR);
+  }
+  ctx->partials = reinterpret_cast<float*>(at(off_part));
+  ctx->norms = reinterpret_cast<float*>(at(off_norms));
+  ctx->clip = reinterpret_cast<float*>(at(off_clip));
+  // Everything starts at zero: moments, S, norms, partial slots.
+  ce = cudaMemset(ctx->arena, 0, ctx->arena_bytes);
+  if (ce == cudaSuccess) ce = cudaDeviceSynchronize();
+  if (ce != cudaSuccess) {
+    cudaFree(ctx->arena);
+    delete ctx;
+    return set_global(GRAPE_ECUDA, std::string("cudaMemset: ") + cudaGetErrorString(ce));
+  }
+  if (tc) {
+    ce = grape::tc_init(sh, ctx->ws.data(), at(off_tc), tc_bytes, &ctx->tc);
+    if (ce == cudaSuccess) ce = cudaDeviceSynchronize();
+    if (ce != cudaSuccess) {
+      grape::tc_release(&ctx->tc);
+      cudaFree(ctx->arena);
+      delete ctx;
+      return set_global(GRAPE_ECUDA, std::string("tensor-core set-up: ") + cudaGetErrorString(ce));
+    }
+  }
+  *out = ctx;
+  return GRAPE_OK;
+}
+
+int grape_step(grape_ctx* ctx, const void* const* A, const void* const* Gout, float* const* W,
+               int64_t step, void* stream) {
+  if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  int rc = check_step_index(ctx, step);
+  if (rc) return rc;
+  rc = validate_io(ctx, A, Gout, W, true, true);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = run_accumulate(ctx, A, Gout, step, st);
+  if (rc) return rc;
+  return run_apply(ctx, W, step, 0, st);
+}
+
+int grape_step_host(grape_ctx* ctx, const void* const* A_host, const void* const* Gout_host,
+                    float* const* W, int64_t step, float* norms_host, void* stream) {
+  if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  int rc = check_step_index(ctx, step);
+  if (rc) return rc;
+  if (!A_host || !Gout_host) return ctx->fail(GRAPE_EINVAL, "A_host and Gout_host must not be null");
+  for (int l = 0; l < ctx->sh.L; ++l)
+    if (!A_host[l] || !Gout_host[l]) return ctx->fail(GRAPE_EINVAL, "null host input pointer");
+  rc = validate_io(ctx, nullptr, nullptr, W, false, true);
+  if (rc) return rc;
+  const size_t el = in_elsize(ctx->sh.dtype);
+  const size_t rows = static_cast<size_t>(ctx->sh.B) * ctx->sh.T;
+  if (ctx->stage_A.empty()) {
+    ctx->stage_A.assign(ctx->sh.L, nullptr);
+    ctx->stage_G.assign(ctx->sh.L, nullptr);
+    for (int l = 0; l < ctx->sh.L; ++l) {
+      if (cudaMalloc(&ctx->stage_A[l], rows * ctx->layers[l].d_in * el) != cudaSuccess ||
+          cudaMalloc(&ctx->stage_G[l], rows * ctx->layers[l].d_out * el) != cudaSuccess) {
+        cudaGetLastError();
+        return ctx->fail(GRAPE_ENOMEM, "staging allocation for grape_step_host failed");
+      }
+    }
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int l = 0; l < ctx->sh.L; ++l) {
+    cudaError_t e = cudaMemcpyAsync(ctx->stage_A[l], A_host[l], rows * ctx->layers[l].d_in * el,
+                                    cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(ctx->stage_G[l], Gout_host[l], rows * ctx->layers[l].d_out * el,
+                          cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return ctx->cuda_fail(e, "host-to-device copy");
+  }
+  rc = run_accumulate(ctx, ctx->stage_A.data(), ctx->stage_G.data(), step, st);
+  if (rc) return rc;
+  rc = run_apply(ctx, W, step, 0, st);
+  if (rc) return rc;
+  if (norms_host) {
+    cudaError_t e = cudaMemcpyAsync(norms_host, ctx->norms, ctx->sh.B * sizeof(float),
+                                    cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return ctx->cuda_fail(e, "device-to-host copy");
+  }
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return ctx->cuda_fail(e, "stream synchronize");
+  return check_device_error(ctx);
+}
+
+int grape_accumulate(grape_ctx* ctx, const void* const* A, const void* const* Gout, int64_t step,
+                     void* stream) {
+  if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  int rc = check_step_index(ctx, step);
+  if (rc) return rc;
+  rc = validate_io(ctx, A, Gout, nullptr, true, false);
+  if (rc) return rc;
+  return run_accumulate(ctx, A, Gout, step, static_cast<cudaStream_t>(stream));
+}
+
+int grape_S_ptr(grape_ctx* ctx, int32_t layer, float** S_dev) {
+  if (!ctx || !S_dev) return set_global(GRAPE_EINVAL, "ctx and S_dev must not be null");
+  if (layer < 0 || layer >= ctx->sh.L) return ctx->fail(GRAPE_EINVAL, "layer out of range");
+  *S_dev = ctx->ws[layer].S;
+  return GRAPE_OK;
+}
+
+int grape_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_total, void* stream) {
+  if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  int rc = check_step_index(ctx, step);
+  if (rc) return rc;
+  if (batch_total < 0) return ctx->fail(GRAPE_EINVAL, "batch_total must be >= 0");
+  rc = validate_io(ctx, nullptr, nullptr, W, false, true);
+  if (rc) return rc;
+  return run_apply(ctx, W, step, batch_total, static_cast<cudaStream_t>(stream));
+}
+
+int grape_get_state(grape_ctx* ctx, int32_t layer, float* m_dev, float* v_dev, void* stream) {
+  if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  if (layer < 0 || layer >= ctx->sh.L) return ctx->fail(GRAPE_EINVAL, "layer out of range");
+  if (!m_dev || !v_dev) return ctx->fail(GRAPE_EINVAL, "m_dev and v_dev must not be null");
+  const size_t bytes = static_cast<size_t>(ctx->sh.r) * ctx->layers[layer].d_out * 4;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(m_dev, ctx->ws[layer].m, bytes, cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(v_dev, ctx->ws[layer].v, bytes, cudaMemcpyDeviceToDevice, st);
+  return e == cudaSuccess ? GRAPE_OK : ctx->cuda_fail(e, "get_state copy");
+}
+
+int grape_set_state(grape_ctx* ctx, int32_t layer, const float* m_dev, const float* v_dev,
+                    void* stream) {
+  if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  if (layer < 0 || layer >= ctx->sh.L) return ctx->fail(GRAPE_EINVAL, "layer out of range");
+  if (!m_dev || !v_dev) return ctx->fail(GRAPE_EINVAL, "m_dev and v_dev must not be null");
+  const size_t bytes = static_cast<size_t>(ctx->sh.r) * ctx->layers[layer].d_out * 4;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(ctx->ws[layer].m, m_dev, bytes, cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(ctx->ws[layer].v, v_dev, bytes, cudaMemcpyDeviceToDevice, st);
+  return e == cudaSuccess ? GRAPE_OK : ctx->cuda_fail(e, "set_state copy");
+}
+
+int grape_debug(grape_ctx* ctx, int32_t what, int32_t layer, void* host_out) {
+  if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  if (!host_out) return ctx->fail(GRAPE_EINVAL, "host_out must not be null");
+  const bool per_layer = what >= GRAPE_DBG_S;
+  if (what < GRAPE_DBG_NORMS || what > GRAPE_DBG_V) return ctx->fail(GRAPE_EINVAL, "unknown debug item");
+  if (per_layer && (layer < 0 || layer >= ctx->sh.L)) return ctx->fail(GRAPE_EINVAL, "layer out of range");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return ctx->cuda_fail(e, "synchronize");
+  if (int rc = check_device_error(ctx)) return rc;
+  const int r = ctx->sh.r;
+  const bool tc = ctx->path == GRAPE_PATH_TC;
+  const grape::LayerWs* w = per_layer ? &ctx->ws[layer] : nullptr;
+  auto copy_bf16_as_f32 = [&](const void* src, size_t n) -> cudaError_t {
+    std::vector<uint16_t> tmp(n);
+    cudaError_t ce = cudaMemcpy(tmp.data(), src, n * 2, cudaMemcpyDeviceToHost);
+    float* o = static_cast<float*>(host_out);
+    for (size_t k = 0; k < n; ++k) {
+      uint32_t u = static_cast<uint32_t>(tmp[k]) << 16;
+      std::memcpy(&o[k], &u, 4);
+    }
+    return ce;
+  };
+  switch (what) {
+    case GRAPE_DBG_NORMS:
+      e = cudaMemcpy(host_out, ctx->norms, ctx->sh.B * 4, cudaMemcpyDeviceToHost);
+      break;
+    case GRAPE_DBG_CLIP:
+      e = cudaMemcpy(host_out, ctx->clip, ctx->sh.B * 4, cudaMemcpyDeviceToHost);
+      break;
+    case GRAPE_DBG_S:
+      e = cudaMemcpy(host_out, w->S, static_cast<size_t>(r) * w->d_out * 4, cudaMemcpyDeviceToHost);
+      break;
+    case GRAPE_DBG_M:
+      e = cudaMemcpy(host_out, w->m, static_cast<size_t>(r) * w->d_out * 4, cudaMemcpyDeviceToHost);
+      break;
+    case GRAPE_DBG_V:
+      e = cudaMemcpy(host_out, w->v, static_cast<size_t>(r) * w->d_out * 4, cudaMemcpyDeviceToHost);
+      break;
+    case GRAPE_DBG_P:
+      e = tc ? copy_bf16_as_f32(w->P16, static_cast<size_t>(w->d_in) * r)
+             : cudaMemcpy(host_out, w->P32, static_cast<size_t>(w->d_in) * r * 4, cudaMemcpyDeviceToHost);
+      break;
+    case GRAPE_DBG_DR:
+      e = tc ? copy_bf16_as_f32(w->dR, static_cast<size_t>(r) * w->d_out)
+             : cudaMemcpy(host_out, w->dR, static_cast<size_t>(r) * w->d_out * 4, cudaMemcpyDeviceToHost);
+      break;
+  }
+  return e == cudaSuccess ? GRAPE_OK : ctx->cuda_fail(e, "debug copy");
+}
+
+int grape_profile(grape_ctx* ctx, int32_t enable) {
+  if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return ctx->cuda_fail(e, "synchronize");
+  ctx->marks.clear();
+  ctx->ev_used = 0;
+  ctx->prof_on = enable != 0;
+  return GRAPE_OK;
+}
+
+int grape_profile_read(grape_ctx* ctx, double* ms_out, int64_t* count_out) {
+  if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return ctx->cuda_fail(e, "synchronize");
+  double ms[GRAPE_N_PHASES] = {};
+  int64_t cnt[GRAPE_N_PHASES] = {};
+  for (const auto& mk : ctx->marks) {
+    float t = 0.0f;
+    e = cudaEventElapsedTime(&t, mk.a, mk.b);
+    if (e != cudaSuccess) return ctx->cuda_fail(e, "cudaEventElapsedTime");
+    ms[mk.phase] += t;
+    cnt[mk.phase] += 1;
+  }
+  ctx->marks.clear();
+  ctx->ev_used = 0;
+  if (int rc = check_device_error(ctx)) return rc;
+  for (int k = 0; k < GRAPE_N_PHASES; ++k) {
+    if (ms_out) ms_out[k] = ms[k];
+    if (count_out) count_out[k] = cnt[k];
+  }
+  return GRAPE_OK;
+}
+
+int grape_launch_count(const grape_ctx* ctx, uint64_t* launches) {
+  if (!ctx || !launches) return set_global(GRAPE_EINVAL, "ctx and launches must not be null");
+  *launches = ctx->launches;
+  return GRAPE_OK;
+}
+
+int grape_device_bytes(const grape_ctx* ctx, uint64_t* bytes) {
+  if (!ctx || !bytes) return set_global(GRAPE_EINVAL, "ctx and bytes must not be null");
+  *bytes = ctx->arena_bytes;
+  return GRAPE_OK;
+}
+
+int grape_path_of(const grape_ctx* ctx, int32_t* path) {
+  if (!ctx || !path) return set_global(GRAPE_EINVAL, "ctx and path must not be null");
+  *path = ctx->path;
+  return GRAPE_OK;
+}
+
+const char* grape_last_error(const grape_ctx* ctx) { return ctx ? ctx->err.c_str() : ""; }
+
+const char* grape_global_error(void) { return g_global_error.c_str(); }
+
+void grape_destroy(grape_ctx* ctx) {
+  if (!ctx) return;
+  grape::tc_release(&ctx->tc);
+  for (cudaEvent_t e : ctx->ev_pool) cudaEventDestroy(e);
+  for (void* p : ctx->stage_A) cudaFree(p);
+  for (void* p : ctx->stage_G) cudaFree(p);
+  if (ctx->arena) cudaFree(ctx->arena);
+  delete ctx;
+}
+
+int grape_philox_words(uint64_t seed, uint32_t layer, uint32_t step, uint32_t stream_id,
+                       int64_t n_blocks, uint32_t* out_dev, void* stream) {
+  if (n_blocks < 0 || n_blocks > 0xFFFFFFFFll) return set_global(GRAPE_EINVAL, "n_blocks out of range");
+  if (n_blocks == 0) return GRAPE_OK;
+  if (!out_dev || !aligned16(out_dev)) return set_global(GRAPE_EINVAL, "out_dev null or not 16-byte aligned");
+  cudaError_t e = grape::launch_philox_words(seed, layer, step, stream_id, n_blocks, out_dev,
+                                             static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GRAPE_OK : set_global(GRAPE_ECUDA, cudaGetErrorString(e));
+}
+
+int grape_gaussian(uint64_t seed, uint32_t layer, uint32_t step, uint32_t stream_id, int64_t n,
+                   float* out_dev, void* stream) {
+  if (n < 0 || n > 4 * 0xFFFFFFFFll) return set_global(GRAPE_EINVAL, "n out of range");
+  if (n == 0) return GRAPE_OK;
+  if (!out_dev) return set_global(GRAPE_EINVAL, "out_dev must not be null");
+  cudaError_t e = grape::launch_gaussian(seed, layer, step, stream_id, n, out_dev,
+                                         static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GRAPE_OK : set_global(GRAPE_ECUDA, cudaGetErrorString(e));
+}
+
+}  // extern "C"

@@ -1,0 +1,825 @@
+// Tensor-core (tcgen05 / TMEM / TMA) path of the DP-GRAPE step for bf16 inputs.
+//
+// The step's dense contractions run as one warp-specialised UMMA kernel
+// template, instantiated four times:
+//
+//   PROJECT    AP   = A P            M = B*T rows, N = r,     K = d_in
+//   NORM       ||R_i||^2, R_i = (A_i P)^T Gout_i
+//                                    M = r,        N = d_out, K = T  (per sample)
+//   AGGREGATE  S    = sum_i c_i R_i  M = r,        N = d_out, K = B*T (split-K)
+//   BACKPROJ   W   -= lr P dR        M = d_in,     N = d_out, K = r
+//
+// (the four contractions of the closing paragraph of "Metodologia: DP-GRAPE" in
+// the technical summary of "Memory-Efficient Differentially Private Training
+// with Gradient Random Projection": per-sample projection, norms for clipping,
+// aggregation, and the projected update of the parameters).
+//
+// CTA layout (192 threads): warp 0 issues TMA loads into a ring of shared-memory
+// stages (128-byte swizzle), warp 1 owns the TMEM allocation and one of its
+// threads issues tcgen05.mma (M = 128, N = BN, K = 16 per instruction) into a
+// 128 x BN fp32 TMEM accumulator, warps 2-5 read the accumulator back with
+// tcgen05.ld (each warp its 32 TMEM lanes) and run the epilogue.  Stage reuse
+// is tracked with mbarriers (TMA completion -> full, tcgen05.commit -> empty);
+// every wait is bounded and reports a timeout through an error word.
+//
+// Operands: A, P (as the A operand of BACKPROJ) are K-major tiles of 128 rows x
+// 64 bf16; AP^T (NORM / AGGREGATE) and every B operand (P, Gout, dR) are
+// M/N-major: 64-element chunks of 64 K-rows x 128 bytes, one TMA box each.
+// Samples with T not a multiple of 64 load through 3-D tensor maps
+// (B x T x cols): rows past T are zero-filled by the TMA unit, so no sample
+// mixes with the next.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <array>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "philox.cuh"
+#include "tc.h"
+#include "tc_ptx.cuh"
+
+namespace grape {
+namespace {
+
+constexpr int kBM = 128;           // UMMA M (one CTA, TMEM lanes)
+constexpr int kBK = 64;            // K per stage: one 128-byte swizzle row of bf16
+constexpr int kThreads = 192;      // 6 warps
+constexpr int kMaxGroup = 16;      // layers per launch
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+
+enum Mode : int { PROJECT = 0, NORM = 1, AGGREGATE = 2, BACKPROJ = 3 };
+
+// error word bits
+constexpr int kErrTimeoutProducer = 1;
+constexpr int kErrTimeoutMma = 2;
+constexpr int kErrTimeoutEpilogue = 4;
+
+struct GroupLayer {
+  int tiles_begin;   // first tile of this layer in the launch
+  int mt, nt, ns;    // m tiles, n tiles, splits (AGGREGATE) / samples (NORM)
+  int kblocks;       // k-blocks of the whole K extent
+  int M, N;          // output extent
+  int ldo;           // leading dimension of the output
+  void* out;         // PROJECT: AP (bf16); AGGREGATE: S; BACKPROJ: W
+  float* split_ws;   // AGGREGATE with ns > 1: ns partial copies of S
+  int* counters;     // AGGREGATE with ns > 1: arrivals per output tile
+  int part_base;     // NORM: first partial slot of this layer
+};
+
+struct GroupParams {
+  CUtensorMap mapA[kMaxGroup];
+  CUtensorMap mapB[kMaxGroup];
+  GroupLayer lay[kMaxGroup];
+  int n_layers;
+  int part_stride;   // NORM
+  float* partials;   // NORM
+  float lr;          // BACKPROJ
+  int* err;
+};
+
+template <int MODE>
+struct ModeTraits {
+  static constexpr bool kAMn = (MODE == NORM || MODE == AGGREGATE);
+  static constexpr bool kA3d = (MODE == NORM);
+  static constexpr bool kB3d = (MODE == NORM);
+};
+
+template <int BN, int STAGES>
+struct Smem {
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStage = kABytes + kBBytes;
+  static constexpr int kBarOff = STAGES * kStage;
+  static constexpr int kBytes = kBarOff + 256 + 1024;   // + barriers + alignment slack
+};
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+template <int MODE, int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ GroupParams p) {
+  using T = ModeTraits<MODE>;
+  using S = Smem<BN, STAGES>;
+  constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+  constexpr uint32_t kIdesc = ptx::idesc_bf16(kBM, BN, T::kAMn, true);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accfull = empty + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 1);
+  float* red = reinterpret_cast<float*>(tmem_slot + 2);   // 4 floats
+  int* flag = reinterpret_cast<int*>(red + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- which tile ----
+  int g = 0;
+  while (g + 1 < p.n_layers && static_cast<int>(blockIdx.x) >= p.lay[g + 1].tiles_begin) ++g;
+  const GroupLayer& L = p.lay[g];
+  int t = static_cast<int>(blockIdx.x) - L.tiles_begin;
+  const int n_t = t % L.nt;
+  t /= L.nt;
+  const int m_t = t % L.mt;
+  const int s_t = t / L.mt;
+  int kb0 = 0, kb1 = L.kblocks;
+  if (MODE == AGGREGATE) {
+    kb0 = static_cast<int>(static_cast<int64_t>(s_t) * L.kblocks / L.ns);
+    kb1 = static_cast<int>(static_cast<int64_t>(s_t + 1) * L.kblocks / L.ns);
+  }
+  const int nkb = kb1 - kb0;
+  const CUtensorMap* mapA = &p.mapA[g];
+  const CUtensorMap* mapB = &p.mapB[g];
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    ptx::mbar_init(accfull, 1);
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(mapA);
+    ptx::prefetch_tmap(mapB);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      for (int k = 0; k < nkb; ++k) {
+        const int s = k % STAGES;
+        if (k >= STAGES && !ptx::mbar_wait(&empty[s], ((k / STAGES) & 1) ^ 1, kWaitLimitNs)) {
+          atomicOr(p.err, kErrTimeoutProducer);
+          break;
+        }
+        uint8_t* sa = smem + s * S::kStage;
+        uint8_t* sb = sa + S::kABytes;
+        ptx::mbar_arrive_expect_tx(&full[s], S::kStage);
+        const int kk = (kb0 + k) * kBK;
+        if (MODE == PROJECT || MODE == BACKPROJ) {
+          ptx::tma_load_2d(sa, mapA, &full[s], kk, m_t * kBM);
+        } else if (MODE == NORM) {
+#pragma unroll
+          for (int c = 0; c < kBM / 64; ++c)
+            ptx::tma_load_3d(sa + c * 8192, mapA, &full[s], m_t * kBM + 64 * c, kk, s_t);
+        } else {
+#pragma unroll
+          for (int c = 0; c < kBM / 64; ++c)
+            ptx::tma_load_2d(sa + c * 8192, mapA, &full[s], m_t * kBM + 64 * c, kk);
+        }
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c) {
+          if (T::kB3d)
+            ptx::tma_load_3d(sb + c * 8192, mapB, &full[s], n_t * BN + 64 * c, kk, s_t);
+          else
+            ptx::tma_load_2d(sb + c * 8192, mapB, &full[s], n_t * BN + 64 * c, kk);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- UMMA issuer ----------------
+    if (lane == 0) {
+      for (int k = 0; k < nkb; ++k) {
+        const int s = k % STAGES;
+        if (!ptx::mbar_wait(&full[s], (k / STAGES) & 1, kWaitLimitNs)) {
+          atomicOr(p.err, kErrTimeoutMma);
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t a_base = ptx::smem_u32(smem + s * S::kStage);
+        const uint32_t b_base = a_base + S::kABytes;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          // K-major: next 16 elements are 32 bytes further along the swizzled row;
+          // M/N-major: next 16 K-rows are 16 x 128 bytes further.
+          const uint64_t ad = T::kAMn ? ptx::desc_sw128(a_base + kk * 2048, 8192, 1024)
+                                      : ptx::desc_sw128(a_base + kk * 32, 16, 1024);
+          const uint64_t bd = ptx::desc_sw128(b_base + kk * 2048, 8192, 1024);
+          ptx::umma_bf16(tmem, ad, bd, kIdesc, (k > 0 || kk > 0) ? 1u : 0u);
+        }
+        ptx::umma_commit(&empty[s]);
+      }
+      ptx::umma_commit(accfull);
+    }
+  } else {
+    // ---------------- epilogue: warps 2..5 ----------------
+    const int q = warp & 3;                 // TMEM lanes 32q .. 32q+31
+    const int row = q * 32 + lane;          // accumulator row of this thread
+    const bool got = ptx::mbar_wait(accfull, 0, kWaitLimitNs);
+    if (!got) atomicOr(p.err, kErrTimeoutEpilogue);
+    ptx::tc_fence_after();
+    const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const bool have = got && nkb > 0;
+
+    if (MODE == PROJECT) {
+      const int m = m_t * kBM + row;
+      __nv_bfloat16* AP = static_cast<__nv_bfloat16*>(L.out);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        ptx::tmem_ld32(tbase + c * 32, v);
+        if (have && m < L.M) {
+          uint4* dst = reinterpret_cast<uint4*>(AP + static_cast<size_t>(m) * L.ldo + n_t * BN + c * 32);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            dst[u] = make_uint4(pack_bf16(v[8 * u + 0], v[8 * u + 1]), pack_bf16(v[8 * u + 2], v[8 * u + 3]),
+                                pack_bf16(v[8 * u + 4], v[8 * u + 5]), pack_bf16(v[8 * u + 6], v[8 * u + 7]));
+        }
+      }
+    } else if (MODE == NORM) {
+      float ss = 0.0f;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        ptx::tmem_ld32(tbase + c * 32, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
+      }
+      if (!have) ss = 0.0f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (lane == 0) red[q] = ss;
+      epi_bar();
+      if (warp == 2 && lane == 0) {
+        const float tot = ((red[0] + red[1]) + red[2]) + red[3];
+        p.partials[static_cast<size_t>(s_t) * p.part_stride + L.part_base + m_t * L.nt + n_t] = tot;
+      }
+    } else if (MODE == AGGREGATE) {
+      const int m = m_t * kBM + row;
+      float* dst = (L.ns > 1) ? L.split_ws + static_cast<size_t>(s_t) * L.M * L.ldo
+                              : static_cast<float*>(L.out);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        ptx::tmem_ld32(tbase + c * 32, v);
+        const int n0 = n_t * BN + c * 32;
+        if (m < L.M) {
+          float* o = dst + static_cast<size_t>(m) * L.ldo + n0;
+          if (n0 + 32 <= L.N) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              reinterpret_cast<float4*>(o)[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+          } else {
+            for (int j = 0; j < 32 && n0 + j < L.N; ++j) o[j] = v[j];
+          }
+        }
+      }
+      if (L.ns > 1) {
+        // Serial split-K fix-up: the last CTA of this output tile to arrive sums the
+        // partial copies in split order (0, 1, ...), so the result does not depend
+        // on which CTA arrives last.
+        __threadfence();
+        epi_bar();
+        if (warp == 2 && lane == 0) {
+          const int old = atomicAdd(&L.counters[m_t * L.nt + n_t], 1);
+          *flag = (old == L.ns - 1);
+        }
+        epi_bar();
+        if (*flag) {
+          __threadfence();
+          if (m < L.M) {
+            float* Sout = static_cast<float*>(L.out);
+            for (int c = 0; c < BN / 32; ++c) {
+              const int n0 = n_t * BN + c * 32;
+              for (int j = 0; j < 32; j += 4) {
+                if (n0 + j >= L.N) break;
+                const size_t o = static_cast<size_t>(m) * L.ldo + n0 + j;
+                float4 acc = *reinterpret_cast<const float4*>(L.split_ws + o);
+                for (int s = 1; s < L.ns; ++s) {
+                  const float4 x = *reinterpret_cast<const float4*>(
+                      L.split_ws + static_cast<size_t>(s) * L.M * L.ldo + o);
+                  acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+                }
+                *reinterpret_cast<float4*>(Sout + o) = acc;
+              }
+            }
+          }
+          if (warp == 2 && lane == 0) L.counters[m_t * L.nt + n_t] = 0;
+        }
+      }
+    } else {  // BACKPROJ: W -= lr * P dR
+      const int m = m_t * kBM + row;
+      float* Wm = static_cast<float*>(L.out) + static_cast<size_t>(m) * L.ldo;
+      const float lr = p.lr;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        ptx::tmem_ld32(tbase + c * 32, v);
+        const int n0 = n_t * BN + c * 32;
+        if (have && m < L.M) {
+          if (n0 + 32 <= L.N) {
+            float4* w4 = reinterpret_cast<float4*>(Wm + n0);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              float4 x = w4[u];
+              x.x = fmaf(-lr, v[4 * u + 0], x.x);
+              x.y = fmaf(-lr, v[4 * u + 1], x.y);
+              x.z = fmaf(-lr, v[4 * u + 2], x.z);
+              x.w = fmaf(-lr, v[4 * u + 3], x.w);
+              w4[u] = x;
+            }
+          } else {
+            for (int j = 0; j < 32 && n0 + j < L.N; ++j) Wm[n0 + j] = fmaf(-lr, v[j], Wm[n0 + j]);
+          }
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---- P_l in bf16, row-major d_in x r: element e = k*r + j ----------------------------
+struct PTable {
+  __nv_bfloat16* P16[GRAPE_MAX_LAYERS];
+  int d_in[GRAPE_MAX_LAYERS];
+};
+
+__global__ void __launch_bounds__(256) gen_P_bf16_kernel(PTable t, uint64_t seed, uint32_t step, int r) {
+  const int l = blockIdx.y;
+  const int64_t nq = static_cast<int64_t>(t.d_in[l]) * r / 4;   // r is a multiple of 64
+  const float scale = rsqrtf(static_cast<float>(r));
+  uint2* out = reinterpret_cast<uint2*>(t.P16[l]);
+  for (int64_t q = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; q < nq;
+       q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 z = gaussian4(seed, static_cast<uint32_t>(l), step, kStreamProjection,
+                               static_cast<uint32_t>(q));
+    out[q] = make_uint2(pack_bf16(z.x * scale, z.y * scale), pack_bf16(z.z * scale, z.w * scale));
+  }
+}
+
+// ---- n_i, c_i, and AP rows of sample i scaled by c_i (all layers) -------------------
+struct ApTable {
+  __nv_bfloat16* AP[GRAPE_MAX_LAYERS];
+};
+
+__global__ void __launch_bounds__(256) clip_scale_kernel(ApTable t, int L, int r, int T, int part_stride,
+                                                         float C, const float* partials, float* norms,
+                                                         float* clip) {
+  __shared__ float red[8];
+  __shared__ float c_sh;
+  const int i = blockIdx.x;
+  const float* pp = partials + static_cast<size_t>(i) * part_stride;
+  float ss = 0.0f;
+  for (int k = threadIdx.x; k < part_stride; k += 256) ss += pp[k];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float tot = 0.0f;
+    for (int w = 0; w < 8; ++w) tot += red[w];
+    const float n = sqrtf(tot);
+    const float c = (n > C) ? C / n : 1.0f;
+    norms[i] = n;
+    clip[i] = c;
+    c_sh = c;
+  }
+  __syncthreads();
+  const float c = c_sh;
+  if (c == 1.0f) return;
+  const size_t n8 = static_cast<size_t>(T) * r / 8;   // 8 bf16 per 16-byte vector
+  for (int l = 0; l < L; ++l) {
+    uint4* rows = reinterpret_cast<uint4*>(t.AP[l] + static_cast<size_t>(i) * T * r);
+    for (size_t k = threadIdx.x; k < n8; k += 256) {
+      uint4 x = rows[k];
+      __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&x);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 f = __bfloat1622float2(h[u]);
+        h[u] = __floats2bfloat162_rn(f.x * c, f.y * c);
+      }
+      rows[k] = x;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// bf16 row-major [rows][cols] as a 2-D map with a (box_cols x box_rows) box, 128-byte swizzle.
+bool map_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_cols,
+            uint32_t box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 [B][T][cols] as a 3-D map with a (64 x 64 x 1) box: rows past T read as zero.
+bool map_3d(CUtensorMap* m, const void* ptr, uint64_t B, uint64_t T, uint64_t cols) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cols, T, B};
+  cuuint64_t strides[2] = {cols * 2, T * cols * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Small cache of encoded maps keyed by base pointer (callers often reuse buffers).
+struct MapCache {
+  struct Entry { const void* ptr; CUtensorMap map; uint64_t used; };
+  std::vector<Entry> e;
+  uint64_t tick = 0;
+  template <class F>
+  bool get(const void* ptr, CUtensorMap* out, F&& make) {
+    ++tick;
+    for (auto& x : e)
+      if (x.ptr == ptr) {
+        x.used = tick;
+        *out = x.map;
+        return true;
+      }
+    Entry n{ptr, {}, tick};
+    if (!make(&n.map)) return false;
+    if (e.size() < 8) {
+      e.push_back(n);
+    } else {
+      size_t lru = 0;
+      for (size_t k = 1; k < e.size(); ++k)
+        if (e[k].used < e[lru].used) lru = k;
+      e[lru] = n;
+    }
+    *out = n.map;
+    return true;
+  }
+};
+
+constexpr int kBnProject = 128;    // r = 128: one N tile; larger r uses 256-wide tiles
+constexpr int kBnWide = 256;
+constexpr int kStagesProject = 4;
+constexpr int kStagesNorm = 4;
+constexpr int kStagesAgg = 4;
+constexpr int kStagesBack = 2;
+
+struct HostState {
+  int L = 0, r = 0, B = 0, T = 0;
+  std::vector<int> d_in, d_out;
+  // fixed maps (library buffers)
+  std::vector<CUtensorMap> mapP_mn;     // P16 as the MN-major B operand of PROJECT
+  std::vector<CUtensorMap> mapP_k;      // P16 as the K-major A operand of BACKPROJ
+  std::vector<CUtensorMap> mapAP3;      // AP as [B][T][r] (NORM A operand)
+  std::vector<CUtensorMap> mapAP2;      // AP as [B*T][r] (AGGREGATE A operand)
+  std::vector<CUtensorMap> mapDR;       // dR as [r][d_out] (BACKPROJ B operand)
+  // per-step maps, cached by pointer
+  std::vector<MapCache> cacheA, cacheG3, cacheG2;
+  // aggregation split-K
+  std::vector<int> agg_ns;
+  std::vector<float*> agg_ws;
+  std::vector<int*> agg_cnt;
+  int* err = nullptr;
+  int bn_project = 128;
+  GroupParams gp;   // host staging of one launch's kernel parameters
+};
+
+int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+
+template <int MODE, int BN, int STAGES>
+cudaError_t launch_group(const GroupParams& gp, int tiles, cudaStream_t st) {
+  using S = Smem<BN, STAGES>;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<MODE, BN, STAGES>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  tc_gemm_kernel<MODE, BN, STAGES><<<tiles, kThreads, S::kBytes, st>>>(gp);
+  return cudaGetLastError();
+}
+
+// Build and launch the groups of one mode.  fill(g, l, gp) sets maps and the layer record
+// (except tiles_begin) and returns the tile count of layer l.
+template <int MODE, int BN, int STAGES, class Fill>
+cudaError_t run_mode(const HostState& hs, int L, cudaStream_t st, int* launches, const Fill& fill,
+                     GroupParams& gp) {
+  for (int l0 = 0; l0 < L; l0 += kMaxGroup) {
+    const int n = (L - l0) < kMaxGroup ? (L - l0) : kMaxGroup;
+    gp.n_layers = n;
+    int tiles = 0;
+    for (int g = 0; g < n; ++g) {
+      int t = 0;
+      if (!fill(g, l0 + g, &t)) return cudaErrorInvalidValue;
+      gp.lay[g].tiles_begin = tiles;
+      tiles += t;
+    }
+    cudaError_t e = launch_group<MODE, BN, STAGES>(gp, tiles, st);
+    if (e != cudaSuccess) return e;
+    ++*launches;
+  }
+  (void)hs;
+  return cudaSuccess;
+}
+
+}  // namespace
+
+bool tc_supported(int device, const grape_layer* layers, int n_layers, int r, int B, int T,
+                  std::string* why) {
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device);
+  if (major != 10 || minor != 0) {
+    if (why) *why = "the tensor-core kernels are built for sm_100a (B200)";
+    return false;
+  }
+  if (!encode_fn()) {
+    if (why) *why = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  // Every TMA box starts inside its tensor (no box lies wholly out of bounds): the
+  // projection width r tiles by 128 (and by 256 above 256), d_out by 256.
+  if (r % 128 != 0 || (r > 256 && r % 256 != 0)) {
+    if (why) *why = "the tensor-core path needs r to be a multiple of 128 (and of 256 above 256)";
+    return false;
+  }
+  for (int l = 0; l < n_layers; ++l)
+    if (layers[l].d_in % 8 != 0 || layers[l].d_out % 256 != 0) {
+      if (why) *why = "the tensor-core path needs d_in % 8 == 0 and d_out % 256 == 0";
+      return false;
+    }
+  (void)B;
+  (void)T;
+  return true;
+}
+
+int tc_partials_per_sample(int r, int d_out) { return cdiv(r, kBM) * cdiv(d_out, kBnWide); }
+
+namespace {
+int agg_splits(int r, int d_out, int B, int T, int L) {
+  // aim for about two CTAs per SM over the whole launch group
+  const int tiles = cdiv(r, kBM) * cdiv(d_out, kBnWide) * (L < kMaxGroup ? L : kMaxGroup);
+  const int kblocks = cdiv(static_cast<int64_t>(B) * T, kBK);
+  int ns = cdiv(296, tiles);
+  if (ns > kblocks) ns = kblocks;
+  if (ns > 16) ns = 16;
+  return ns < 1 ? 1 : ns;
+}
+}  // namespace
+
+size_t tc_workspace_bytes(const StepShape& sh, const LayerWs* ws) {
+  size_t b = 256;  // error word
+  for (int l = 0; l < sh.L; ++l) {
+    const int ns = agg_splits(sh.r, ws[l].d_out, sh.B, sh.T, sh.L);
+    if (ns > 1) {
+      b += (static_cast<size_t>(ns) * sh.r * ws[l].d_out * 4 + 255) & ~size_t(255);
+      b += (static_cast<size_t>(cdiv(sh.r, kBM)) * cdiv(ws[l].d_out, kBnWide) * 4 + 255) & ~size_t(255);
+    }
+  }
+  return b;
+}
+
+cudaError_t tc_init(const StepShape& sh, const LayerWs* ws, void* scratch, size_t bytes,
+                    TcWorkspace* out) {
+  HostState* hs = new HostState();
+  hs->L = sh.L;
+  hs->r = sh.r;
+  hs->B = sh.B;
+  hs->T = sh.T;
+  hs->bn_project = sh.r == 128 ? 128 : 256;
+  char* base = static_cast<char*>(scratch);
+  size_t off = 0;
+  hs->err = reinterpret_cast<int*>(base + off);
+  off += 256;
+  hs->mapP_mn.resize(sh.L);
+  hs->mapP_k.resize(sh.L);
+  hs->mapAP3.resize(sh.L);
+  hs->mapAP2.resize(sh.L);
+  hs->mapDR.resize(sh.L);
+  hs->cacheA.resize(sh.L);
+  hs->cacheG3.resize(sh.L);
+  hs->cacheG2.resize(sh.L);
+  hs->agg_ns.resize(sh.L);
+  hs->agg_ws.assign(sh.L, nullptr);
+  hs->agg_cnt.assign(sh.L, nullptr);
+  const uint64_t rows = static_cast<uint64_t>(sh.B) * sh.T;
+  for (int l = 0; l < sh.L; ++l) {
+    hs->d_in.push_back(ws[l].d_in);
+    hs->d_out.push_back(ws[l].d_out);
+    bool ok = map_2d(&hs->mapP_mn[l], ws[l].P16, ws[l].d_in, sh.r, 64, 64) &&
+              map_2d(&hs->mapP_k[l], ws[l].P16, ws[l].d_in, sh.r, 64, kBM) &&
+              map_3d(&hs->mapAP3[l], ws[l].AP, sh.B, sh.T, sh.r) &&
+              map_2d(&hs->mapAP2[l], ws[l].AP, rows, sh.r, 64, 64) &&
+              map_2d(&hs->mapDR[l], ws[l].dR, sh.r, ws[l].d_out, 64, 64);
+    if (!ok) {
+      delete hs;
+      return cudaErrorInvalidValue;
+    }
+    const int ns = agg_splits(sh.r, ws[l].d_out, sh.B, sh.T, sh.L);
+    hs->agg_ns[l] = ns;
+    if (ns > 1) {
+      hs->agg_ws[l] = reinterpret_cast<float*>(base + off);
+      off += (static_cast<size_t>(ns) * sh.r * ws[l].d_out * 4 + 255) & ~size_t(255);
+      hs->agg_cnt[l] = reinterpret_cast<int*>(base + off);
+      off += (static_cast<size_t>(cdiv(sh.r, kBM)) * cdiv(ws[l].d_out, kBnWide) * 4 + 255) & ~size_t(255);
+    }
+  }
+  if (off > bytes) {
+    delete hs;
+    return cudaErrorInvalidValue;
+  }
+  out->base = scratch;
+  out->bytes = bytes;
+  out->host_state = hs;
+  return cudaSuccess;
+}
+
+void tc_release(TcWorkspace* tc) {
+  if (tc && tc->host_state) {
+    delete static_cast<HostState*>(tc->host_state);
+    tc->host_state = nullptr;
+  }
+}
+
+int* tc_error_word(const TcWorkspace& tc) {
+  return tc.host_state ? static_cast<HostState*>(tc.host_state)->err : nullptr;
+}
+
+cudaError_t tc_generate_P(const StepShape& sh, const LayerWs* ws, const TcWorkspace&, uint32_t step,
+                          cudaStream_t st, int* launches) {
+  PTable t{};
+  int64_t most = 0;
+  for (int l = 0; l < sh.L; ++l) {
+    t.P16[l] = ws[l].P16;
+    t.d_in[l] = ws[l].d_in;
+    const int64_t q = static_cast<int64_t>(ws[l].d_in) * sh.r / 4;
+    most = q > most ? q : most;
+  }
+  int gx = cdiv(most, 256);
+  gx = gx < 1184 ? gx : 1184;
+  gen_P_bf16_kernel<<<dim3(gx, sh.L), 256, 0, st>>>(t, sh.seed, step, sh.r);
+  ++*launches;
+  return cudaGetLastError();
+}
+
+cudaError_t tc_project(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
+                       const TcWorkspace& tc, cudaStream_t st, int* launches) {
+  HostState& hs = *static_cast<HostState*>(tc.host_state);
+  GroupParams& gp = hs.gp;
+  std::memset(&gp, 0, sizeof(gp));
+  gp.err = hs.err;
+  const int64_t rows = static_cast<int64_t>(sh.B) * sh.T;
+  auto fill = [&](int g, int l, int* tiles) {
+    if (!hs.cacheA[l].get(io[l].A, &gp.mapA[g], [&](CUtensorMap* m) {
+          return map_2d(m, io[l].A, rows, ws[l].d_in, 64, kBM);
+        }))
+      return false;
+    gp.mapB[g] = hs.mapP_mn[l];
+    GroupLayer& L = gp.lay[g];
+    L.mt = cdiv(rows, kBM);
+    L.nt = sh.r / hs.bn_project;
+    L.ns = 1;
+    L.kblocks = cdiv(ws[l].d_in, kBK);
+    L.M = static_cast<int>(rows);
+    L.N = sh.r;
+    L.ldo = sh.r;
+    L.out = ws[l].AP;
+    *tiles = L.mt * L.nt;
+    return true;
+  };
+  if (hs.bn_project == 128)
+    return run_mode<PROJECT, 128, kStagesProject>(hs, sh.L, st, launches, fill, gp);
+  return run_mode<PROJECT, 256, kStagesProject>(hs, sh.L, st, launches, fill, gp);
+}
+
+cudaError_t tc_project_norm(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
+                            const TcWorkspace& tc, float* partials, cudaStream_t st, int* launches) {
+  HostState& hs = *static_cast<HostState*>(tc.host_state);
+  GroupParams& gp = hs.gp;
+  std::memset(&gp, 0, sizeof(gp));
+  gp.err = hs.err;
+  gp.partials = partials;
+  gp.part_stride = sh.part_stride;
+  auto fill = [&](int g, int l, int* tiles) {
+    gp.mapA[g] = hs.mapAP3[l];
+    if (!hs.cacheG3[l].get(io[l].G, &gp.mapB[g], [&](CUtensorMap* m) {
+          return map_3d(m, io[l].G, sh.B, sh.T, ws[l].d_out);
+        }))
+      return false;
+    GroupLayer& L = gp.lay[g];
+    L.mt = cdiv(sh.r, kBM);
+    L.nt = cdiv(ws[l].d_out, kBnWide);
+    L.ns = sh.B;
+    L.kblocks = cdiv(sh.T, kBK);
+    L.M = sh.r;
+    L.N = ws[l].d_out;
+    L.part_base = ws[l].part_base;
+    *tiles = L.mt * L.nt * sh.B;
+    return true;
+  };
+  return run_mode<NORM, kBnWide, kStagesNorm>(hs, sh.L, st, launches, fill, gp);
+}
+
+cudaError_t tc_clip_scale(const StepShape& sh, const LayerWs* ws, const TcWorkspace&,
+                          const float* partials, float* norms, float* clip, cudaStream_t st,
+                          int* launches) {
+  ApTable t{};
+  for (int l = 0; l < sh.L; ++l) t.AP[l] = static_cast<__nv_bfloat16*>(ws[l].AP);
+  clip_scale_kernel<<<sh.B, 256, 0, st>>>(t, sh.L, sh.r, sh.T, sh.part_stride, sh.C, partials, norms,
+                                          clip);
+  ++*launches;
+  return cudaGetLastError();
+}
+
+cudaError_t tc_aggregate(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
+                         const TcWorkspace& tc, const float* clip, cudaStream_t st, int* launches) {
+  (void)clip;   // the clip factors were folded into AP by tc_clip_scale
+  HostState& hs = *static_cast<HostState*>(tc.host_state);
+  GroupParams& gp = hs.gp;
+  std::memset(&gp, 0, sizeof(gp));
+  gp.err = hs.err;
+  const int64_t rows = static_cast<int64_t>(sh.B) * sh.T;
+  auto fill = [&](int g, int l, int* tiles) {
+    gp.mapA[g] = hs.mapAP2[l];
+    if (!hs.cacheG2[l].get(io[l].G, &gp.mapB[g], [&](CUtensorMap* m) {
+          return map_2d(m, io[l].G, rows, ws[l].d_out, 64, 64);
+        }))
+      return false;
+    GroupLayer& L = gp.lay[g];
+    L.mt = cdiv(sh.r, kBM);
+    L.nt = cdiv(ws[l].d_out, kBnWide);
+    L.ns = hs.agg_ns[l];
+    L.kblocks = cdiv(rows, kBK);
+    L.M = sh.r;
+    L.N = ws[l].d_out;
+    L.ldo = ws[l].d_out;
+    L.out = ws[l].S;
+    L.split_ws = hs.agg_ws[l];
+    L.counters = hs.agg_cnt[l];
+    *tiles = L.mt * L.nt * L.ns;
+    return true;
+  };
+  return run_mode<AGGREGATE, kBnWide, kStagesAgg>(hs, sh.L, st, launches, fill, gp);
+}
+
+cudaError_t tc_backproject(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
+                           const TcWorkspace& tc, float lr, cudaStream_t st, int* launches) {
+  HostState& hs = *static_cast<HostState*>(tc.host_state);
+  GroupParams& gp = hs.gp;
+  std::memset(&gp, 0, sizeof(gp));
+  gp.err = hs.err;
+  gp.lr = lr;
+  auto fill = [&](int g, int l, int* tiles) {
+    gp.mapA[g] = hs.mapP_k[l];
+    gp.mapB[g] = hs.mapDR[l];
+    GroupLayer& L = gp.lay[g];
+    L.mt = cdiv(ws[l].d_in, kBM);
+    L.nt = cdiv(ws[l].d_out, kBnWide);
+    L.ns = 1;
+    L.kblocks = cdiv(sh.r, kBK);
+    L.M = ws[l].d_in;
+    L.N = ws[l].d_out;
+    L.ldo = ws[l].d_out;
+    L.out = io[l].W;
+    *tiles = L.mt * L.nt;
+    return true;
+  };
+  return run_mode<BACKPROJ, kBnWide, kStagesBack>(hs, sh.L, st, launches, fill, gp);
+}
+
+}  // namespace grape

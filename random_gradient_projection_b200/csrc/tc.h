@@ -1,0 +1,42 @@
+// Tensor-core (tcgen05 / TMEM / TMA) path of the DP-GRAPE step for bf16 inputs.
+#pragma once
+#include <cuda_runtime.h>
+
+#include <string>
+
+#include "kernels.h"
+
+namespace grape {
+
+struct TcWorkspace {
+  void* base = nullptr;       // library scratch inside the context arena
+  size_t bytes = 0;
+  void* host_state = nullptr; // tensor maps and launch plans (host memory)
+};
+
+bool tc_supported(int device, const grape_layer* layers, int n_layers, int r, int B, int T,
+                  std::string* why);
+int tc_partials_per_sample(int r, int d_out);
+size_t tc_workspace_bytes(const StepShape& sh, const LayerWs* ws);
+cudaError_t tc_init(const StepShape& sh, const LayerWs* ws, void* scratch, size_t bytes,
+                    TcWorkspace* out);
+void tc_release(TcWorkspace* tc);
+// Device word where the tensor-core kernels record bounded waits that gave up (0 = none).
+int* tc_error_word(const TcWorkspace& tc);
+// The phases of the tensor-core path; each enqueues on `st`, adds the number of
+// kernels it launched to *launches and returns the first CUDA error.
+cudaError_t tc_generate_P(const StepShape& sh, const LayerWs* ws, const TcWorkspace& tc,
+                          uint32_t step, cudaStream_t st, int* launches);
+cudaError_t tc_project(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
+                       const TcWorkspace& tc, cudaStream_t st, int* launches);
+cudaError_t tc_project_norm(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
+                            const TcWorkspace& tc, float* partials, cudaStream_t st, int* launches);
+cudaError_t tc_clip_scale(const StepShape& sh, const LayerWs* ws, const TcWorkspace& tc,
+                          const float* partials, float* norms, float* clip, cudaStream_t st,
+                          int* launches);
+cudaError_t tc_aggregate(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
+                         const TcWorkspace& tc, const float* clip, cudaStream_t st, int* launches);
+cudaError_t tc_backproject(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
+                           const TcWorkspace& tc, float lr, cudaStream_t st, int* launches);
+
+}  // namespace grape

@@ -1,0 +1,22 @@
+"""Data-parallel DP-GRAPE step: one process per GPU, samples sharded across ranks.
+
+Per-sample work (projection, norms, clipping) needs no exchange: every rank
+clips its own samples.  The one exchange is the sum of the clipped projected
+gradients S_l = sum_i c_i R_{i,l} over all ranks (an all-reduce of r x d_out
+fp32 per layer).  Every rank then adds the same noise (the same Philox key),
+divides by the global batch, runs Adam and back-projects, so the replicas
+stay identical.
+"""
+from __future__ import annotations
+
+
+def dp_step(g, A, Gout, W, step: int, group=None, stream=None):
+    """One step of context ``g`` (a GrapeStep or an object with the same methods)
+    inside ``torch.distributed`` process group ``group``."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    g.accumulate(A, Gout, step, stream)
+    if world > 1:
+        for l in range(len(g.layers)):
+            dist.all_reduce(g.S_tensor(l), op=dist.ReduceOp.SUM, group=group)
+    g.apply(W, step, g.B * world, stream)

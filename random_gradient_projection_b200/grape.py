@@ -1,0 +1,328 @@
+"""ctypes binding of libgrape.so (the C ABI in include/grape.h).
+
+Argument marshalling only: every step of the method runs in the library's
+CUDA kernels.  The functions keep the C names; ``GrapeStep`` is a small
+owner of a context that accepts torch tensors.  Importing this module fails
+loudly when the library has not been built: there is no other code path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libgrape.so")
+
+GRAPE_OK, GRAPE_EINVAL, GRAPE_ENOMEM, GRAPE_ECUDA, GRAPE_ETIMEOUT, GRAPE_EUNSUPPORTED = range(6)
+GRAPE_MAX_LAYERS = 64
+GRAPE_F32, GRAPE_BF16 = 0, 1
+GRAPE_PATH_AUTO, GRAPE_PATH_SIMT, GRAPE_PATH_TC = 0, 1, 2
+(GRAPE_DBG_NORMS, GRAPE_DBG_CLIP, GRAPE_DBG_S, GRAPE_DBG_P, GRAPE_DBG_DR, GRAPE_DBG_M,
+ GRAPE_DBG_V) = range(7)
+
+# the entry points include/grape.h declares
+EXPORTS = (
+    "grape_create", "grape_step", "grape_step_host", "grape_accumulate", "grape_S_ptr",
+    "grape_apply", "grape_get_state", "grape_set_state", "grape_debug", "grape_device_bytes",
+    "grape_path_of", "grape_last_error", "grape_global_error", "grape_destroy",
+    "grape_philox_words", "grape_gaussian", "grape_profile", "grape_profile_read",
+    "grape_launch_count",
+)
+PHASES = ("gen_P", "project", "norm", "clip", "aggregate", "adam", "backproject")
+
+
+class grape_layer(ctypes.Structure):
+    _fields_ = [("d_in", ctypes.c_int32), ("d_out", ctypes.c_int32)]
+
+
+class grape_adam(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_double), ("beta1", ctypes.c_double), ("beta2", ctypes.c_double),
+                ("eps", ctypes.c_double)]
+
+
+class GrapeError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"grape error {code}: {msg}")
+        self.code = code
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m random_gradient_projection_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i32, i64, u32, u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_uint64
+    pp = ctypes.POINTER(ctypes.c_void_p)
+    sig = {
+        "grape_create": ([ctypes.POINTER(grape_layer), i32, i32, ctypes.c_double, ctypes.c_double, u64,
+                          ctypes.POINTER(grape_adam), i32, i32, i32, i32, ctypes.POINTER(vp)], i32),
+        "grape_step": ([vp, pp, pp, pp, i64, vp], i32),
+        "grape_step_host": ([vp, pp, pp, pp, i64, vp, vp], i32),
+        "grape_accumulate": ([vp, pp, pp, i64, vp], i32),
+        "grape_S_ptr": ([vp, i32, ctypes.POINTER(vp)], i32),
+        "grape_apply": ([vp, pp, i64, i64, vp], i32),
+        "grape_get_state": ([vp, i32, vp, vp, vp], i32),
+        "grape_set_state": ([vp, i32, vp, vp, vp], i32),
+        "grape_debug": ([vp, i32, i32, vp], i32),
+        "grape_device_bytes": ([vp, ctypes.POINTER(u64)], i32),
+        "grape_path_of": ([vp, ctypes.POINTER(i32)], i32),
+        "grape_last_error": ([vp], ctypes.c_char_p),
+        "grape_global_error": ([], ctypes.c_char_p),
+        "grape_destroy": ([vp], None),
+        "grape_philox_words": ([u64, u32, u32, u32, i64, vp, vp], i32),
+        "grape_gaussian": ([u64, u32, u32, u32, i64, vp, vp], i32),
+        "grape_profile": ([vp, i32], i32),
+        "grape_profile_read": ([vp, vp, vp], i32),
+        "grape_launch_count": ([vp, ctypes.POINTER(u64)], i32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = load()
+    return _lib
+
+
+def _ptr(x) -> int:
+    """Address of a torch tensor, an int, or None (0)."""
+    if x is None:
+        return 0
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr()
+    if isinstance(x, np.ndarray):
+        return x.ctypes.data
+    raise TypeError(f"cannot take the address of {type(x)}")
+
+
+def _array(ptrs) -> ctypes.Array:
+    return (ctypes.c_void_p * len(ptrs))(*[_ptr(p) for p in ptrs])
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int, ctx=None):
+    if rc != GRAPE_OK:
+        L = lib()
+        msg = (L.grape_last_error(ctx) if ctx else L.grape_global_error()) or b""
+        raise GrapeError(rc, msg.decode())
+
+
+# ---- the C names, marshalled ------------------------------------------------
+
+def grape_create(layers: Sequence[Sequence[int]], r: int, C: float, sigma: float, seed: int,
+                 lr: float, beta1: float, beta2: float, eps: float, B: int, T: int,
+                 dtype: int, path: int = GRAPE_PATH_AUTO) -> int:
+    arr = (grape_layer * len(layers))(*[grape_layer(int(a), int(b)) for a, b in layers])
+    adam = grape_adam(lr, beta1, beta2, eps)
+    out = ctypes.c_void_p()
+    _check(lib().grape_create(arr, len(layers), r, C, sigma, seed & (2**64 - 1), ctypes.byref(adam),
+                              B, T, dtype, path, ctypes.byref(out)))
+    return out.value
+
+
+def grape_step(ctx: int, A, Gout, W, step: int, stream=None):
+    _check(lib().grape_step(ctx, _array(A), _array(Gout), _array(W), step, _stream(stream)), ctx)
+
+
+def grape_step_host(ctx: int, A_host, Gout_host, W, step: int, norms_host=None, stream=None):
+    _check(lib().grape_step_host(ctx, _array(A_host), _array(Gout_host), _array(W), step,
+                                 _ptr(norms_host), _stream(stream)), ctx)
+
+
+def grape_accumulate(ctx: int, A, Gout, step: int, stream=None):
+    _check(lib().grape_accumulate(ctx, _array(A), _array(Gout), step, _stream(stream)), ctx)
+
+
+def grape_S_ptr(ctx: int, layer: int) -> int:
+    out = ctypes.c_void_p()
+    _check(lib().grape_S_ptr(ctx, layer, ctypes.byref(out)), ctx)
+    return out.value
+
+
+def grape_apply(ctx: int, W, step: int, batch_total: int = 0, stream=None):
+    _check(lib().grape_apply(ctx, _array(W), step, batch_total, _stream(stream)), ctx)
+
+
+def grape_get_state(ctx: int, layer: int, m, v, stream=None):
+    _check(lib().grape_get_state(ctx, layer, _ptr(m), _ptr(v), _stream(stream)), ctx)
+
+
+def grape_set_state(ctx: int, layer: int, m, v, stream=None):
+    _check(lib().grape_set_state(ctx, layer, _ptr(m), _ptr(v), _stream(stream)), ctx)
+
+
+def grape_debug(ctx: int, what: int, layer: int, shape) -> np.ndarray:
+    out = np.empty(shape, dtype=np.float32)
+    _check(lib().grape_debug(ctx, what, layer, out.ctypes.data), ctx)
+    return out
+
+
+def grape_device_bytes(ctx: int) -> int:
+    out = ctypes.c_uint64()
+    _check(lib().grape_device_bytes(ctx, ctypes.byref(out)), ctx)
+    return out.value
+
+
+def grape_path_of(ctx: int) -> int:
+    out = ctypes.c_int32()
+    _check(lib().grape_path_of(ctx, ctypes.byref(out)), ctx)
+    return out.value
+
+
+def grape_profile(ctx: int, enable: bool):
+    _check(lib().grape_profile(ctx, 1 if enable else 0), ctx)
+
+
+def grape_profile_read(ctx: int):
+    """{phase name: (milliseconds, calls)} since profiling was switched on."""
+    ms = np.zeros(len(PHASES), dtype=np.float64)
+    cnt = np.zeros(len(PHASES), dtype=np.int64)
+    _check(lib().grape_profile_read(ctx, ms.ctypes.data, cnt.ctypes.data), ctx)
+    return {name: (float(ms[k]), int(cnt[k])) for k, name in enumerate(PHASES)}
+
+
+def grape_launch_count(ctx: int) -> int:
+    out = ctypes.c_uint64()
+    _check(lib().grape_launch_count(ctx, ctypes.byref(out)), ctx)
+    return out.value
+
+
+def grape_destroy(ctx: int):
+    lib().grape_destroy(ctx)
+
+
+def grape_philox_words(seed: int, layer: int, step: int, stream_id: int, n_blocks: int, out,
+                       stream=None):
+    _check(lib().grape_philox_words(seed & (2**64 - 1), layer, step, stream_id, n_blocks, _ptr(out),
+                                    _stream(stream)))
+
+
+def grape_gaussian(seed: int, layer: int, step: int, stream_id: int, n: int, out, stream=None):
+    _check(lib().grape_gaussian(seed & (2**64 - 1), layer, step, stream_id, n, _ptr(out),
+                                _stream(stream)))
+
+
+# ---- a context owner for torch tensors ---------------------------------------
+
+class _DeviceArray:
+    """Wraps a library-owned device buffer for torch.as_tensor (no copy)."""
+
+    def __init__(self, ptr: int, shape, typestr: str = "<f4"):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr,
+                                         "data": (ptr, False), "version": 3, "strides": None}
+
+
+class GrapeStep:
+    """One DP-GRAPE context: a fixed layer stack, batch shape and hyper-parameters."""
+
+    def __init__(self, layers, r, C, sigma, seed, B, T, dtype="bf16", lr=1e-3, beta1=0.9,
+                 beta2=0.999, eps=1e-8, path=GRAPE_PATH_AUTO):
+        self.layers = [tuple(int(x) for x in l) for l in layers]
+        self.r, self.B, self.T = int(r), int(B), int(T)
+        self.dtype = GRAPE_BF16 if dtype in ("bf16", GRAPE_BF16) else GRAPE_F32
+        self.ctx = grape_create(self.layers, self.r, C, sigma, seed, lr, beta1, beta2, eps, B, T,
+                                self.dtype, path)
+
+    @classmethod
+    def for_workload(cls, w, path=GRAPE_PATH_AUTO, B=None):
+        return cls(w.layers, w.r, w.C, w.sigma, w.seed, B or w.B, w.T, w.dtype, w.lr, w.beta1,
+                   w.beta2, w.eps, path)
+
+    def close(self):
+        if self.ctx:
+            grape_destroy(self.ctx)
+            self.ctx = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # noqa: BLE001  interpreter shutdown
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    @property
+    def path(self) -> int:
+        return grape_path_of(self.ctx)
+
+    def device_bytes(self) -> int:
+        return grape_device_bytes(self.ctx)
+
+    def profile(self, enable: bool = True):
+        grape_profile(self.ctx, enable)
+
+    def profile_read(self):
+        return grape_profile_read(self.ctx)
+
+    def launch_count(self) -> int:
+        return grape_launch_count(self.ctx)
+
+    def step(self, A, Gout, W, step: int, stream=None):
+        grape_step(self.ctx, A, Gout, W, step, stream)
+
+    def step_host(self, A_host, Gout_host, W, step: int, norms_host=None, stream=None):
+        grape_step_host(self.ctx, A_host, Gout_host, W, step, norms_host, stream)
+
+    def accumulate(self, A, Gout, step: int, stream=None):
+        grape_accumulate(self.ctx, A, Gout, step, stream)
+
+    def apply(self, W, step: int, batch_total: int = 0, stream=None):
+        grape_apply(self.ctx, W, step, batch_total, stream)
+
+    def S_tensor(self, layer: int):
+        """S_l as a torch tensor sharing the library's memory (for all-reduce)."""
+        import torch
+        ptr = grape_S_ptr(self.ctx, layer)
+        return torch.as_tensor(_DeviceArray(ptr, (self.r, self.layers[layer][1])), device="cuda")
+
+    def get_state(self, layer: int, m, v, stream=None):
+        grape_get_state(self.ctx, layer, m, v, stream)
+
+    def set_state(self, layer: int, m, v, stream=None):
+        grape_set_state(self.ctx, layer, m, v, stream)
+
+    # intermediates of the last step (host copies)
+    def norms(self):
+        return grape_debug(self.ctx, GRAPE_DBG_NORMS, 0, (self.B,))
+
+    def clip(self):
+        return grape_debug(self.ctx, GRAPE_DBG_CLIP, 0, (self.B,))
+
+    def S(self, l):
+        return grape_debug(self.ctx, GRAPE_DBG_S, l, (self.r, self.layers[l][1]))
+
+    def P(self, l):
+        return grape_debug(self.ctx, GRAPE_DBG_P, l, (self.layers[l][0], self.r))
+
+    def dR(self, l):
+        return grape_debug(self.ctx, GRAPE_DBG_DR, l, (self.r, self.layers[l][1]))
+
+    def m(self, l):
+        return grape_debug(self.ctx, GRAPE_DBG_M, l, (self.r, self.layers[l][1]))
+
+    def v(self, l):
+        return grape_debug(self.ctx, GRAPE_DBG_V, l, (self.r, self.layers[l][1]))

@@ -1,0 +1,70 @@
+"""The C-ABI library loads and exports what include/grape.h declares (no GPU needed)."""
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "grape.h")
+
+
+def declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"GRAPE_API\s+[\w\s\*]*?\b(grape_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from random_gradient_projection_b200 import build, grape
+    build.build()
+    return grape.load()
+
+
+def test_header_declares_the_boundary():
+    names = declared()
+    for must in ("grape_create", "grape_step", "grape_destroy", "grape_step_host",
+                 "grape_accumulate", "grape_apply", "grape_get_state", "grape_set_state"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from random_gradient_projection_b200 import grape
+    out = subprocess.run(["nm", "-D", "--defined-only", grape.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(grape_\w+)$", out, flags=re.M))
+    missing = [n for n in declared() if n not in exported]
+    assert not missing, missing
+    for n in declared():
+        assert hasattr(lib, n)
+    # the binding wraps exactly the declared set
+    assert sorted(grape.EXPORTS) == declared()
+
+
+@pytest.mark.parametrize("kw,msg", [
+    (dict(layers=[(64, 32)], r=80), "r must be <= d_in"),
+    (dict(layers=[], r=8), "n_layers"),
+    (dict(layers=[(64, 32)], r=8, C=0.0), "C must be"),
+    (dict(layers=[(64, 32)], r=8, sigma=-1.0), "sigma"),
+    (dict(layers=[(64, 32)], r=8, B=0), "B and T"),
+    (dict(layers=[(64, 32)], r=8, beta1=1.0), "adam"),
+    (dict(layers=[(64, 32)], r=8, dtype=7), "in_dtype"),
+    (dict(layers=[(64, 32)] * 65, r=8), "n_layers"),
+])
+def test_create_validates_before_touching_the_device(lib, kw, msg):
+    from random_gradient_projection_b200 import grape
+    args = dict(layers=[(64, 32)], r=8, C=1.0, sigma=1.0, seed=0, lr=1e-3, beta1=0.9,
+                beta2=0.999, eps=1e-8, B=4, T=16, dtype=grape.GRAPE_F32, path=0)
+    args.update(kw)
+    with pytest.raises(grape.GrapeError) as e:
+        grape.grape_create(**args)
+    assert e.value.code == grape.GRAPE_EINVAL
+    assert msg in str(e.value)
+
+
+def test_generator_entry_points_validate(lib):
+    from random_gradient_projection_b200 import grape
+    with pytest.raises(grape.GrapeError) as e:
+        grape.grape_philox_words(0, 0, 0, 0, 16, 8, stream=0)   # misaligned output
+    assert e.value.code == grape.GRAPE_EINVAL
+    grape.grape_gaussian(0, 0, 0, 0, 0, 0, stream=0)              # empty request is a no-op

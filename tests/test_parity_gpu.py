@@ -1,0 +1,270 @@
+"""Parity of the CUDA library with the fp64 oracle, through the C ABI (needs a B200)."""
+import numpy as np
+import pytest
+
+import oracle.grape_oracle as O
+import workloads as W
+from harness import compare, rel_fro, run_library, run_oracle, to_device
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+from random_gradient_projection_b200 import GrapeError, GrapeStep, grape  # noqa: E402
+
+SIMT, TC = grape.GRAPE_PATH_SIMT, grape.GRAPE_PATH_TC
+
+# ---------------------------------------------------------------------------------
+# the generator
+# ---------------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("seed,layer,step,stream", [(0, 0, 0, 0), (1, 3, 7, 1),
+                                                     (0x0123456789ABCDEF, 27, 12345, 0),
+                                                     (2**64 - 1, 2**32 - 1, 2**31, 1)])
+def test_philox_words_bit_exact(seed, layer, step, stream):
+    n = 100_003
+    out = torch.empty(4 * n, dtype=torch.int32, device="cuda")
+    grape.grape_philox_words(seed, layer, step, stream, n, out)
+    got = out.cpu().numpy().view(np.uint32).reshape(n, 4)
+    ref = O.philox_words(seed, layer, step, stream, n)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("n", [1, 3, 4, 4097, 1 << 20])
+def test_gaussian_matches_oracle(n):
+    out = torch.empty(n, dtype=torch.float32, device="cuda")
+    grape.grape_gaussian(42, 5, 9, 1, n, out)
+    got = out.cpu().numpy().astype(np.float64)
+    ref = O.gaussian_stream(42, 5, 9, 1, n)
+    # fp32 log / sqrt / sincospi of the same words: a few fp32 ulps of |z| <= 6.7
+    assert np.max(np.abs(got - ref)) < 2e-5
+    assert rel_fro(got, ref) < 1e-6
+
+
+# ---------------------------------------------------------------------------------
+# full steps against the oracle
+# ---------------------------------------------------------------------------------
+
+CASES = {
+    # name: (workload, steps)
+    "tiny_f32": (W.get("tiny_f32"), 3),
+    # MLP layers at reduced batch: several 64/128 tiles
+    "mlp_2x1024_B4": (W.scaled(W.get("mlp4x1024"), n_layers=2, B=4), 3),
+    # ViT shapes with the ragged T = 197 and d_out = 2304, 768
+    "vit_qkv_down_B3": (W.scaled(W.get("vit_b"), layers=((768, 2304), (3072, 768)), B=3), 2),
+    # sparse loss tokens, C = 0.5, T = 1000 (ragged)
+    "longctx_1layer_T1000": (W.scaled(W.get("longctx"), layers=((2048, 2048),), B=2, T=1000), 2),
+    # r = 512 (two 256-wide N tiles, four 128-row M tiles), ragged T
+    "r512_T130": (W.Workload("r512", ((1024, 2816), (2816, 1024)), r=512, B=2, T=130,
+                             dtype="bf16", C=1.0, sigma=0.6, steps=2), 2),
+    # more layers than one launch group holds (16)
+    "20_layers": (W.Workload("twenty", tuple([(256, 256), (512, 256)] * 10), r=128, B=3, T=64,
+                             dtype="bf16", C=1.0, sigma=1.0, steps=2), 2),
+    # degenerate shapes (CUDA-core path only: r not a multiple of 128)
+    "T1_B1": (W.Workload("T1_B1", ((96, 40),), r=16, B=1, T=1, dtype="bf16", C=1.0,
+                         sigma=0.5, steps=2), 2),
+    "r_equals_d_in": (W.Workload("r_eq_din", ((64, 32), (64, 48)), r=64, B=3, T=9,
+                                 dtype="f32", C=1.0, sigma=1.0, steps=2), 2),
+    "odd_sizes": (W.Workload("odd", ((37, 19), (53, 7)), r=5, B=5, T=13, dtype="f32",
+                             C=0.7, sigma=0.3, steps=2), 2),
+    "no_noise": (W.scaled(W.get("tiny_f32"), sigma=0.0), 3),
+    "no_noise_bf16": (W.scaled(W.get("mlp4x1024"), n_layers=2, B=4, T=64, sigma=0.0), 2),
+    "T1_bf16_tc": (W.Workload("T1_tc", ((256, 256),), r=128, B=5, T=1, dtype="bf16", C=1.0,
+                              sigma=0.5, steps=2), 2),
+}
+
+
+def _tc_ok(w):
+    return (w.dtype == "bf16" and w.r % 128 == 0 and (w.r <= 256 or w.r % 256 == 0)
+            and all(di % 8 == 0 and do % 256 == 0 for di, do in w.layers))
+
+
+def _tol(w, path):
+    if w.dtype == "f32":
+        return 1e-5
+    return 1e-4 if path == SIMT else 2e-2
+
+
+PAIRS = [(c, SIMT) for c in sorted(CASES)] + [(c, TC) for c in sorted(CASES) if _tc_ok(CASES[c][0])]
+
+
+@pytest.mark.parametrize("case,path", PAIRS, ids=[f"{c}-{'tc' if p == TC else 'simt'}" for c, p in PAIRS])
+def test_step_matches_oracle(case, path):
+    w, steps = CASES[case]
+    lib = run_library(w, steps, path)
+    assert lib["path"] == path
+    orc = run_oracle(w, steps)
+    worst = compare(w, lib, orc, _tol(w, path), steps)
+    print(case, "tc" if path == TC else "simt", {k: f"{v:.2e}" for k, v in worst.items()})
+
+
+def test_bench_workload_full_size_tc():
+    """The benchmarked workload (4 x 1024^2, r = 128, B = 64, T = 128) at full size on the
+    tensor-core path, two steps, against the oracle on the whole batch."""
+    w = W.get("mlp4x1024")
+    lib = run_library(w, 2, TC)
+    orc = run_oracle(w, 2)
+    worst = compare(w, lib, orc, 2e-2, 2)
+    print("mlp4x1024 full", {k: f"{v:.2e}" for k, v in worst.items()})
+
+
+def test_auto_path_picks_tensor_cores_for_bf16():
+    g = GrapeStep.for_workload(W.scaled(W.get("mlp4x1024"), n_layers=1, B=2, T=16))
+    assert g.path == TC
+    g.close()
+
+
+def test_tiny_f32_matches_golden():
+    """The fp32 workload against the stored oracle values (tests/golden)."""
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "tiny_f32_oracle.json")))
+    w = W.get("tiny_f32")
+    lib = run_library(w, w.steps, grape.GRAPE_PATH_AUTO)
+    assert lib["path"] == SIMT
+    assert rel_fro(lib["W"][0], g["W"][0]) < 1e-5
+    assert rel_fro(lib["trace"][-1]["m"][0], g["m"][0]) < 1e-5
+    assert rel_fro(lib["trace"][-1]["v"][0], g["v"][0]) < 1e-5
+    for s in range(w.steps):
+        assert rel_fro(lib["trace"][s]["S"][0], g["steps"][s]["S"][0]) < 1e-5
+        assert rel_fro(lib["trace"][s]["norms"], g["steps"][s]["norms"]) < 1e-5
+
+
+# ---------------------------------------------------------------------------------
+# properties of the library itself
+# ---------------------------------------------------------------------------------
+
+def _inputs(w, s):
+    x = W.make_step_inputs(w, s)
+    return [to_device(a, w.dtype) for a in x.A], [to_device(a, w.dtype) for a in x.Gout]
+
+
+@pytest.mark.parametrize("path", [SIMT, TC], ids=["simt", "tc"])
+def test_bitwise_reproducible(path):
+    """Fixed-order reductions: two runs of the same steps give identical bits."""
+    w = W.scaled(W.get("mlp4x1024"), n_layers=2, B=3, T=64)
+    a = run_library(w, 2, path)
+    b = run_library(w, 2, path)
+    for l in range(w.n_layers):
+        assert np.array_equal(a["W"][l], b["W"][l])
+        assert np.array_equal(a["trace"][-1]["m"][l], b["trace"][-1]["m"][l])
+
+
+@pytest.mark.parametrize("path", [SIMT, TC], ids=["simt", "tc"])
+def test_clipped_norm_bound(path):
+    """Every clip factor brings the sample to norm <= C; unclipped samples keep 1."""
+    w = W.scaled(W.get("mlp4x1024"), n_layers=2, B=16, T=32)
+    lib = run_library(w, 1, path)
+    n, c = lib["trace"][0]["norms"], lib["trace"][0]["clip"]
+    assert np.all(c * n <= w.C * (1 + 1e-6))
+    assert np.all(c[n <= w.C] == 1.0)
+    assert (c < 1).any() and (c == 1).any()
+
+
+@pytest.mark.parametrize("path", [SIMT, TC], ids=["simt", "tc"])
+def test_accumulate_apply_equals_step(path):
+    w = W.scaled(W.get("mlp4x1024"), n_layers=2, B=3, T=32)
+    W0 = W.make_weights(w)
+    g1, g2 = GrapeStep.for_workload(w, path=path), GrapeStep.for_workload(w, path=path)
+    W1 = [torch.from_numpy(x).cuda() for x in W0]
+    W2 = [torch.from_numpy(x).cuda() for x in W0]
+    for s in range(2):
+        A, G = _inputs(w, s)
+        g1.step(A, G, W1, s)
+        g2.accumulate(A, G, s)
+        g2.apply(W2, s)
+    torch.cuda.synchronize()
+    for l in range(w.n_layers):
+        assert torch.equal(W1[l], W2[l])
+
+
+@pytest.mark.parametrize("path", [SIMT, TC], ids=["simt", "tc"])
+def test_step_host_equals_step(path):
+    w = W.scaled(W.get("mlp4x1024"), n_layers=2, B=3, T=32)
+    W0 = W.make_weights(w)
+    g1, g2 = GrapeStep.for_workload(w, path=path), GrapeStep.for_workload(w, path=path)
+    W1 = [torch.from_numpy(x).cuda() for x in W0]
+    W2 = [torch.from_numpy(x).cuda() for x in W0]
+    for s in range(2):
+        x = W.make_step_inputs(w, s)
+        A = [to_device(a, w.dtype) for a in x.A]
+        G = [to_device(a, w.dtype) for a in x.Gout]
+        g1.step(A, G, W1, s)
+        hostA = [torch.from_numpy(a.view(np.int16)).pin_memory() for a in x.A]
+        hostG = [torch.from_numpy(a.view(np.int16)).pin_memory() for a in x.Gout]
+        norms = np.zeros(w.B, dtype=np.float32)
+        g2.step_host(hostA, hostG, W2, s, norms)
+        assert np.array_equal(norms, g1.norms())
+    torch.cuda.synchronize()
+    for l in range(w.n_layers):
+        assert torch.equal(W1[l], W2[l])
+
+
+@pytest.mark.parametrize("path", [SIMT, TC], ids=["simt", "tc"])
+def test_checkpoint_resume_bitwise(path):
+    """Stop after step 1, move m and v to a fresh context, continue: identical W.
+    P is not state (it is regenerated from seed, layer and step)."""
+    w = W.scaled(W.get("mlp4x1024"), n_layers=2, B=3, T=32)
+    W0 = W.make_weights(w)
+    ref = GrapeStep.for_workload(w, path=path)
+    Wr = [torch.from_numpy(x).cuda() for x in W0]
+    for s in range(3):
+        A, G = _inputs(w, s)
+        ref.step(A, G, Wr, s)
+    first = GrapeStep.for_workload(w, path=path)
+    Wc = [torch.from_numpy(x).cuda() for x in W0]
+    for s in range(2):
+        A, G = _inputs(w, s)
+        first.step(A, G, Wc, s)
+    saved = []
+    for l, (di, do) in enumerate(w.layers):
+        m = torch.empty(w.r, do, device="cuda")
+        v = torch.empty(w.r, do, device="cuda")
+        first.get_state(l, m, v)
+        saved.append((m, v))
+    first.close()
+    second = GrapeStep.for_workload(w, path=path)
+    for l, (m, v) in enumerate(saved):
+        second.set_state(l, m, v)
+    A, G = _inputs(w, 2)
+    second.step(A, G, Wc, 2)
+    torch.cuda.synchronize()
+    for l in range(w.n_layers):
+        assert torch.equal(Wr[l], Wc[l])
+
+
+def test_moment_memory_is_projected():
+    """Optimizer state is O(r x layers): the context holds far less than 2 x 4 bytes x W."""
+    w = W.get("mlp4x1024")
+    g = GrapeStep.for_workload(w, path=SIMT)
+    full_adam = sum(2 * 4 * di * do for di, do in w.layers)
+    moments = sum(2 * 4 * w.r * do for _, do in w.layers)
+    assert moments * 8 == full_adam         # r = d/8 here
+    assert g.device_bytes() < full_adam     # moments plus the whole workspace
+    g.close()
+
+
+def test_errors_are_reported():
+    w = W.get("tiny_f32")
+    g = GrapeStep.for_workload(w)
+    x = W.make_step_inputs(w, 0)
+    A = [to_device(a, "f32") for a in x.A]
+    G = [to_device(a, "f32") for a in x.Gout]
+    Wt = [torch.zeros(64, 32, device="cuda")]
+    with pytest.raises(GrapeError) as e:
+        g.step([A[0].data_ptr() + 4], G, Wt, 0)      # misaligned
+    assert e.value.code == grape.GRAPE_EINVAL
+    with pytest.raises(GrapeError) as e:
+        g.step(A, G, Wt, -1)
+    assert e.value.code == grape.GRAPE_EINVAL
+    g.step(A, G, Wt, 0)                              # still usable afterwards
+    torch.cuda.synchronize()
+    g.close()
+
+
+def test_allocation_failure_is_reported(monkeypatch):
+    monkeypatch.setenv("GRAPE_FAULT_ALLOC", "1")
+    with pytest.raises(GrapeError) as e:
+        GrapeStep.for_workload(W.get("tiny_f32"))
+    assert e.value.code == grape.GRAPE_ENOMEM
