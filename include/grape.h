@@ -192,6 +192,34 @@ GRAPE_API int grape_philox_words(uint64_t seed, uint32_t layer, uint32_t step, u
 GRAPE_API int grape_gaussian(uint64_t seed, uint32_t layer, uint32_t step, uint32_t stream_id, int64_t n,
                    float* out_dev, void* stream);
 
+/* Per-sample squared projected norms ||(A_i P)^T Gout_i||_F^2 of ONE bf16 layer
+ * (the quantity grape_step sums over layers before clipping), computed without
+ * allocating anything.  The paper has no counterpart of this call: it exists
+ * for callers that must not allocate device memory, e.g. code running under a
+ * framework whose caching allocator has reserved the GPU's memory (a side
+ * cudaMalloc can fail or fragment its pool) and latency-critical code that
+ * cannot afford cudaMalloc/cudaFree, which may synchronise the device.
+ *
+ *  A, Gout        device pointers, bf16, B x T x d_in and B x T x d_out
+ *  r              projection width; P = z(seed, layer, step, stream 0, .)/sqrt(r)
+ *  sqnorms_out    device pointer, B floats (written; NaN if a device-side wait
+ *                 gave up)
+ *  stream         cudaStream_t (NULL = default stream); nothing is synchronised
+ * Limits: r % 128 == 0 (and % 256 above 256), d_in % 8 == 0, d_out % 256 == 0,
+ * and d_in*r*2 + B*T*r*2 + B*ceil(r/128)*ceil(d_out/256)*4 + 256 bytes of
+ * scratch within the library's static device array of 8 MiB; larger problems
+ * are rejected with GRAPE_EINVAL before anything is launched.
+ * All calls share that one array (every GPU that loads the library holds its
+ * 8 MiB until the process exits), so calls whose work overlaps on the GPU, on
+ * different streams or host threads, race on it; serialise them.  The first
+ * call on a device looks the array's address up on that device (it must be the
+ * current device); make that first call before any stream capture.  Errors are
+ * reported through grape_global_error(). */
+GRAPE_API int grape_layer_sqnorms_static(const void* A, const void* Gout, int32_t d_in, int32_t d_out,
+                                         int32_t r, int32_t B, int32_t T, uint64_t seed,
+                                         uint32_t layer, uint32_t step, float* sqnorms_out,
+                                         void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -641,4 +641,31 @@ int grape_gaussian(uint64_t seed, uint32_t layer, uint32_t step, uint32_t stream
   return e == cudaSuccess ? GRAPE_OK : set_global(GRAPE_ECUDA, cudaGetErrorString(e));
 }
 
+int grape_layer_sqnorms_static(const void* A, const void* Gout, int32_t d_in, int32_t d_out,
+                               int32_t r, int32_t B, int32_t T, uint64_t seed, uint32_t layer,
+                               uint32_t step, float* sqnorms_out, void* stream) {
+  if (!A || !Gout || !sqnorms_out) return set_global(GRAPE_EINVAL, "A, Gout and sqnorms_out must not be null");
+  if (!aligned16(A) || !aligned16(Gout)) return set_global(GRAPE_EINVAL, "A and Gout must be 16-byte aligned");
+  if (B < 1 || T < 1 || d_in < 1 || d_out < 1 || r < 1 || r > d_in)
+    return set_global(GRAPE_EINVAL, "need B, T, d_in, d_out >= 1 and 1 <= r <= d_in");
+  if (r % 128 != 0 || (r > 256 && r % 256 != 0) || d_in % 8 != 0 || d_out % 256 != 0)
+    return set_global(GRAPE_EINVAL, "need r % 128 == 0 (and % 256 above 256), d_in % 8 == 0, d_out % 256 == 0");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return set_global(GRAPE_ECUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0) return set_global(GRAPE_EUNSUPPORTED, "needs an sm_100a device (B200)");
+  const size_t need = grape::tc_static_scratch_needed(d_in, d_out, r, B, T);
+  if (need > grape::tc_static_scratch_bytes())
+    return set_global(GRAPE_EINVAL, "problem needs " + std::to_string(need) + " bytes of scratch; the static scratch holds " +
+                                        std::to_string(grape::tc_static_scratch_bytes()) +
+                                        " (d_in*r*2 + B*T*r*2 + B*slots*4 + 256 bytes)");
+  e = grape::tc_layer_sqnorms_static(A, Gout, d_in, d_out, r, B, T, seed, layer, step, sqnorms_out,
+                                     static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return set_global(GRAPE_ECUDA, std::string("layer sqnorms: ") + cudaGetErrorString(e));
+  return GRAPE_OK;
+}
+
 }  // extern "C"

@@ -822,4 +822,138 @@ cudaError_t tc_backproject(const StepShape& sh, const LayerWs* ws, const LayerIo
   return run_mode<BACKPROJ, kBnWide, kStagesBack>(hs, sh.L, st, launches, fill, gp);
 }
 
+// ---------------------------------------------------------------------------------
+// Per-sample squared norms of one layer with no allocation (grape_layer_sqnorms_static).
+// ---------------------------------------------------------------------------------
+namespace {
+
+// The scratch of that entry point: a file-scope device array, present on every GPU
+// that loads the library until the process exits.  Layout per call: error word |
+// P (d_in x r bf16) | AP (B*T x r bf16) | norm partials (B x slots fp32).
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_ptr[kMaxDevices] = {};
+
+size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
+
+// P of one layer with an explicit Philox layer index.
+__global__ void __launch_bounds__(256) gen_P_layer_static_kernel(__nv_bfloat16* P16, int d_in, int r,
+                                                                 uint64_t seed, uint32_t layer,
+                                                                 uint32_t step) {
+  const int64_t nq = static_cast<int64_t>(d_in) * r / 4;
+  const float scale = rsqrtf(static_cast<float>(r));
+  uint2* out = reinterpret_cast<uint2*>(P16);
+  for (int64_t q = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; q < nq;
+       q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 z = gaussian4(seed, layer, step, kStreamProjection, static_cast<uint32_t>(q));
+    out[q] = make_uint2(pack_bf16(z.x * scale, z.y * scale), pack_bf16(z.z * scale, z.w * scale));
+  }
+}
+
+// out[i] = sum of sample i's partial slots in slot order; NaN if a bounded wait gave up.
+__global__ void sum_slots_static_kernel(const float* partials, int slots, int B, const int* err,
+                                        float* out) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= B) return;
+  float s = 0.0f;
+  for (int k = 0; k < slots; ++k) s += partials[static_cast<size_t>(i) * slots + k];
+  out[i] = (*err == 0) ? s : __int_as_float(0x7fc00000);
+}
+
+}  // namespace
+
+size_t tc_static_scratch_bytes() { return kStaticScratchBytes; }
+
+size_t tc_static_scratch_needed(int d_in, int d_out, int r, int B, int T) {
+  const size_t slots = static_cast<size_t>(cdiv(r, kBM)) * cdiv(d_out, kBnWide);
+  return 256 + round256(static_cast<size_t>(d_in) * r * 2) +
+         round256(static_cast<size_t>(B) * T * r * 2) + round256(static_cast<size_t>(B) * slots * 4);
+}
+
+cudaError_t tc_layer_sqnorms_static(const void* A, const void* G, int d_in, int d_out, int r, int B,
+                                    int T, uint64_t seed, uint32_t layer, uint32_t step, float* out,
+                                    cudaStream_t st) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  void* base_v = nullptr;
+  {
+    // First call on this device (which is current): take the array's device address.
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ptr[dev]) {
+      e = cudaGetSymbolAddress(&g_static_ptr[dev], g_static_scratch);
+      if (e != cudaSuccess) {
+        g_static_ptr[dev] = nullptr;
+        return e;
+      }
+    }
+    base_v = g_static_ptr[dev];
+  }
+  char* base = static_cast<char*>(base_v);
+  int* err = reinterpret_cast<int*>(base);
+  __nv_bfloat16* P16 = reinterpret_cast<__nv_bfloat16*>(base + 256);
+  __nv_bfloat16* AP = reinterpret_cast<__nv_bfloat16*>(base + 256 + round256(static_cast<size_t>(d_in) * r * 2));
+  float* partials = reinterpret_cast<float*>(reinterpret_cast<char*>(AP) +
+                                             round256(static_cast<size_t>(B) * T * r * 2));
+  const int slots = cdiv(r, kBM) * cdiv(d_out, kBnWide);
+  const int64_t rows = static_cast<int64_t>(B) * T;
+
+  // The error word is the only state that must start at zero; P, AP and every
+  // partial slot are fully rewritten below.
+  e = cudaMemsetAsync(err, 0, sizeof(int), st);
+  if (e != cudaSuccess) return e;
+
+  int gx = cdiv(static_cast<int64_t>(d_in) * r / 4, 256);
+  gx = gx < 1184 ? gx : 1184;
+  gen_P_layer_static_kernel<<<gx, 256, 0, st>>>(P16, d_in, r, seed, layer, step);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  GroupParams gp;   // kernel parameters, staged on the host stack
+  std::memset(&gp, 0, sizeof(gp));
+  gp.err = err;
+  gp.n_layers = 1;
+  const int bnp = (r == 128) ? 128 : 256;
+  // AP = A P
+  if (!map_2d(&gp.mapA[0], A, rows, d_in, 64, kBM) || !map_2d(&gp.mapB[0], P16, d_in, r, 64, 64))
+    return cudaErrorInvalidValue;
+  GroupLayer& L = gp.lay[0];
+  L.tiles_begin = 0;
+  L.mt = cdiv(rows, kBM);
+  L.nt = r / bnp;
+  L.ns = 1;
+  L.kblocks = cdiv(d_in, kBK);
+  L.M = static_cast<int>(rows);
+  L.N = r;
+  L.ldo = r;
+  L.out = AP;
+  e = (bnp == 128) ? launch_group<PROJECT, 128, kStagesProject>(gp, L.mt * L.nt, st)
+                   : launch_group<PROJECT, 256, kStagesProject>(gp, L.mt * L.nt, st);
+  if (e != cudaSuccess) return e;
+  // ||(A_i P)^T Gout_i||^2 per sample, as partial slots
+  std::memset(&gp, 0, sizeof(gp));
+  gp.err = err;
+  gp.n_layers = 1;
+  gp.partials = partials;
+  gp.part_stride = slots;
+  if (!map_3d(&gp.mapA[0], AP, B, T, r) || !map_3d(&gp.mapB[0], G, B, T, d_out))
+    return cudaErrorInvalidValue;
+  L = GroupLayer{};
+  L.mt = cdiv(r, kBM);
+  L.nt = cdiv(d_out, kBnWide);
+  L.ns = B;
+  L.kblocks = cdiv(T, kBK);
+  L.M = r;
+  L.N = d_out;
+  L.part_base = 0;
+  e = launch_group<NORM, kBnWide, kStagesNorm>(gp, L.mt * L.nt * B, st);
+  if (e != cudaSuccess) return e;
+  sum_slots_static_kernel<<<cdiv(B, 128), 128, 0, st>>>(partials, slots, B, err, out);
+  return cudaGetLastError();
+}
+
 }  // namespace grape

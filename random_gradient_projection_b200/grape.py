@@ -29,7 +29,7 @@ EXPORTS = (
     "grape_apply", "grape_get_state", "grape_set_state", "grape_debug", "grape_device_bytes",
     "grape_path_of", "grape_last_error", "grape_global_error", "grape_destroy",
     "grape_philox_words", "grape_gaussian", "grape_profile", "grape_profile_read",
-    "grape_launch_count",
+    "grape_launch_count", "grape_layer_sqnorms_static",
 )
 PHASES = ("gen_P", "project", "norm", "clip", "aggregate", "adam", "backproject")
 
@@ -76,6 +76,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "grape_profile": ([vp, i32], i32),
         "grape_profile_read": ([vp, vp, vp], i32),
         "grape_launch_count": ([vp, ctypes.POINTER(u64)], i32),
+        "grape_layer_sqnorms_static": ([vp, vp, i32, i32, i32, i32, i32, u64, u32, u32, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -205,6 +206,15 @@ def grape_launch_count(ctx: int) -> int:
     out = ctypes.c_uint64()
     _check(lib().grape_launch_count(ctx, ctypes.byref(out)), ctx)
     return out.value
+
+
+def grape_layer_sqnorms_static(A, Gout, d_in: int, d_out: int, r: int, B: int, T: int, seed: int,
+                               layer: int, step: int, sqnorms_out, stream=None):
+    """Per-sample squared projected norms of one bf16 layer; uses only the library's
+    static device scratch (no allocation).  See include/grape.h."""
+    _check(lib().grape_layer_sqnorms_static(_ptr(A), _ptr(Gout), d_in, d_out, r, B, T,
+                                            seed & (2**64 - 1), layer, step, _ptr(sqnorms_out),
+                                            _stream(stream)))
 
 
 def grape_destroy(ctx: int):
