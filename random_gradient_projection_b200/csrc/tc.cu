@@ -35,6 +35,8 @@
 
 #include <array>
 #include <cstdint>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -61,13 +63,11 @@ constexpr int kErrTimeoutEpilogue = 4;
 
 struct GroupLayer {
   int tiles_begin;   // first tile of this layer in the launch
-  int mt, nt, ns;    // m tiles, n tiles, splits (AGGREGATE) / samples (NORM)
+  int mt, nt, ns;    // m tiles, n tiles, samples (NORM; 1 otherwise)
   int kblocks;       // k-blocks of the whole K extent
   int M, N;          // output extent
   int ldo;           // leading dimension of the output
   void* out;         // PROJECT: AP (bf16); AGGREGATE: S; BACKPROJ: W
-  float* split_ws;   // AGGREGATE with ns > 1: ns partial copies of S
-  int* counters;     // AGGREGATE with ns > 1: arrivals per output tile
   int part_base;     // NORM: first partial slot of this layer
 };
 
@@ -76,16 +76,17 @@ struct GroupParams {
   CUtensorMap mapB[kMaxGroup];
   GroupLayer lay[kMaxGroup];
   int n_layers;
+  int total_tiles;
   int part_stride;   // NORM
   float* partials;   // NORM
   float lr;          // BACKPROJ
+  int cluster;       // AGGREGATE on a cluster: CTAs per output tile (K split)
   int* err;
 };
 
 template <int MODE>
 struct ModeTraits {
   static constexpr bool kAMn = (MODE == NORM || MODE == AGGREGATE);
-  static constexpr bool kA3d = (MODE == NORM);
   static constexpr bool kB3d = (MODE == NORM);
 };
 
@@ -95,7 +96,7 @@ struct Smem {
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStage = kABytes + kBBytes;
   static constexpr int kBarOff = STAGES * kStage;
-  static constexpr int kBytes = kBarOff + 256 + 1024;   // + barriers + alignment slack
+  static constexpr int kBytes = kBarOff + 512 + 1024;   // + barriers + alignment slack
 };
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
@@ -105,11 +106,36 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+struct TileCoord {
+  int g, m_t, n_t, s_t, kb0, kb1;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const GroupParams& p, int tile, int mode) {
+  TileCoord c;
+  int g = 0;
+  while (g + 1 < p.n_layers && tile >= p.lay[g + 1].tiles_begin) ++g;
+  const GroupLayer& L = p.lay[g];
+  int t = tile - L.tiles_begin;
+  c.g = g;
+  c.n_t = t % L.nt;
+  t /= L.nt;
+  c.m_t = t % L.mt;
+  c.s_t = t / L.mt;
+  c.kb0 = 0;
+  c.kb1 = L.kblocks;
+  (void)mode;
+  return c;
+}
+
+// Persistent: CTA b handles tiles b, b + gridDim.x, ...  The shared-memory stage ring
+// (index `it` counts k-blocks over all of this CTA's tiles) runs across tile
+// boundaries, and two TMEM accumulators let the epilogue of one tile overlap the
+// loads and MMAs of the next.
 template <int MODE, int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ GroupParams p) {
   using T = ModeTraits<MODE>;
   using S = Smem<BN, STAGES>;
-  constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+  constexpr uint32_t kTmemCols = 2 * BN;
   constexpr uint32_t kIdesc = ptx::idesc_bf16(kBM, BN, T::kAMn, true);
 
   extern __shared__ uint8_t smem_raw[];
@@ -117,40 +143,32 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
   uint64_t* empty = full + STAGES;
-  uint64_t* accfull = empty + STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 1);
-  float* red = reinterpret_cast<float*>(tmem_slot + 2);   // 4 floats
-  int* flag = reinterpret_cast<int*>(red + 4);
+  uint64_t* accfull = empty + STAGES;       // [2]
+  uint64_t* accempty = accfull + 2;         // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + 2);
+  float* red = reinterpret_cast<float*>(tmem_slot + 2);   // [2][4]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(red + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  // ---- which tile ----
-  int g = 0;
-  while (g + 1 < p.n_layers && static_cast<int>(blockIdx.x) >= p.lay[g + 1].tiles_begin) ++g;
-  const GroupLayer& L = p.lay[g];
-  int t = static_cast<int>(blockIdx.x) - L.tiles_begin;
-  const int n_t = t % L.nt;
-  t /= L.nt;
-  const int m_t = t % L.mt;
-  const int s_t = t / L.mt;
-  int kb0 = 0, kb1 = L.kblocks;
-  if (MODE == AGGREGATE) {
-    kb0 = static_cast<int>(static_cast<int64_t>(s_t) * L.kblocks / L.ns);
-    kb1 = static_cast<int>(static_cast<int64_t>(s_t + 1) * L.kblocks / L.ns);
-  }
-  const int nkb = kb1 - kb0;
-  const CUtensorMap* mapA = &p.mapA[g];
-  const CUtensorMap* mapB = &p.mapB[g];
+  auto wait = [&](uint64_t* bar, uint32_t parity) {
+    return ptx::mbar_wait_or_abort(bar, parity, kWaitLimitNs, abort_flag);
+  };
 
   if (warp == 0 && lane == 0) {
+    *abort_flag = 0;
     for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(&full[s], 1);
       ptx::mbar_init(&empty[s], 1);
     }
-    ptx::mbar_init(accfull, 1);
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&accfull[b], 1);
+      ptx::mbar_init(&accempty[b], 4);
+    }
     ptx::fence_mbar_init();
-    ptx::prefetch_tmap(mapA);
-    ptx::prefetch_tmap(mapB);
+    for (int g = 0; g < p.n_layers; ++g) {
+      ptx::prefetch_tmap(&p.mapA[g]);
+      ptx::prefetch_tmap(&p.mapB[g]);
+    }
   }
   if (warp == 1) {
     ptx::tmem_alloc(tmem_slot, kTmemCols);
@@ -164,42 +182,293 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      for (int k = 0; k < nkb; ++k) {
-        const int s = k % STAGES;
-        if (k >= STAGES && !ptx::mbar_wait(&empty[s], ((k / STAGES) & 1) ^ 1, kWaitLimitNs)) {
-          atomicOr(p.err, kErrTimeoutProducer);
-          break;
-        }
-        uint8_t* sa = smem + s * S::kStage;
-        uint8_t* sb = sa + S::kABytes;
-        ptx::mbar_arrive_expect_tx(&full[s], S::kStage);
-        const int kk = (kb0 + k) * kBK;
-        if (MODE == PROJECT || MODE == BACKPROJ) {
-          ptx::tma_load_2d(sa, mapA, &full[s], kk, m_t * kBM);
-        } else if (MODE == NORM) {
+      // A and Gout stream once per use; P, AP and dR are re-read by other tiles or
+      // by the next phase, so they are kept in L2 preferentially.
+      const uint64_t polA = (MODE == PROJECT || MODE == AGGREGATE) ? ptx::policy_evict_first()
+                                                                     : ptx::policy_evict_last();
+      const uint64_t polB = (MODE == AGGREGATE) ? ptx::policy_evict_first() : ptx::policy_evict_last();
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+        const TileCoord c = decode_tile(p, tile, MODE);
+        const CUtensorMap* mapA = &p.mapA[c.g];
+        const CUtensorMap* mapB = &p.mapB[c.g];
+        for (int kb = c.kb0; kb < c.kb1; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t use = it / STAGES;
+          if (use > 0 && !wait(&empty[s], (use - 1) & 1)) {
+            atomicOr(p.err, kErrTimeoutProducer);
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + s * S::kStage;
+          uint8_t* sb = sa + S::kABytes;
+          ptx::mbar_arrive_expect_tx(&full[s], S::kStage);
+          const int kk = kb * kBK;
+          if (MODE == PROJECT || MODE == BACKPROJ) {
+            ptx::tma_load_2d_hint(sa, mapA, &full[s], kk, c.m_t * kBM, polA);
+          } else if (MODE == NORM) {
 #pragma unroll
-          for (int c = 0; c < kBM / 64; ++c)
-            ptx::tma_load_3d(sa + c * 8192, mapA, &full[s], m_t * kBM + 64 * c, kk, s_t);
-        } else {
+            for (int q = 0; q < kBM / 64; ++q)
+              ptx::tma_load_3d_hint(sa + q * 8192, mapA, &full[s], c.m_t * kBM + 64 * q, kk, c.s_t, polA);
+          } else {
 #pragma unroll
-          for (int c = 0; c < kBM / 64; ++c)
-            ptx::tma_load_2d(sa + c * 8192, mapA, &full[s], m_t * kBM + 64 * c, kk);
-        }
+            for (int q = 0; q < kBM / 64; ++q)
+              ptx::tma_load_2d_hint(sa + q * 8192, mapA, &full[s], c.m_t * kBM + 64 * q, kk, polA);
+          }
 #pragma unroll
-        for (int c = 0; c < BN / 64; ++c) {
-          if (T::kB3d)
-            ptx::tma_load_3d(sb + c * 8192, mapB, &full[s], n_t * BN + 64 * c, kk, s_t);
-          else
-            ptx::tma_load_2d(sb + c * 8192, mapB, &full[s], n_t * BN + 64 * c, kk);
+          for (int q = 0; q < BN / 64; ++q) {
+            if (T::kB3d)
+              ptx::tma_load_3d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kk, c.s_t, polB);
+            else
+              ptx::tma_load_2d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kk, polB);
+          }
         }
       }
     }
   } else if (warp == 1) {
     // ---------------- UMMA issuer ----------------
     if (lane == 0) {
-      for (int k = 0; k < nkb; ++k) {
-        const int s = k % STAGES;
-        if (!ptx::mbar_wait(&full[s], (k / STAGES) & 1, kWaitLimitNs)) {
+      uint32_t it = 0, tc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++tc) {
+        const TileCoord c = decode_tile(p, tile, MODE);
+        const int b = tc & 1;
+        const uint32_t use = tc >> 1;
+        if (use > 0 && !wait(&accempty[b], (use - 1) & 1)) {
+          atomicOr(p.err, kErrTimeoutMma);
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d = tmem + b * BN;
+        for (int kb = c.kb0; kb < c.kb1; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!wait(&full[s], ph)) {
+            atomicOr(p.err, kErrTimeoutMma);
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a_base = ptx::smem_u32(smem + s * S::kStage);
+          const uint32_t b_base = a_base + S::kABytes;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            // K-major: the next 16 elements are 32 bytes further along the swizzled row;
+            // M/N-major: the next 16 K-rows are 16 x 128 bytes further.
+            const uint64_t ad = T::kAMn ? ptx::desc_sw128(a_base + k * 2048, 8192, 1024)
+                                        : ptx::desc_sw128(a_base + k * 32, 16, 1024);
+            const uint64_t bd = ptx::desc_sw128(b_base + k * 2048, 8192, 1024);
+            ptx::umma_bf16(d, ad, bd, kIdesc, (kb > c.kb0 || k > 0) ? 1u : 0u);
+          }
+          ptx::umma_commit(&empty[s]);
+        }
+        ptx::umma_commit(&accfull[b]);
+      }
+    }
+  } else {
+    // ---------------- epilogue: warps 2..5 ----------------
+    const int q = warp & 3;                       // TMEM lanes 32q .. 32q+31
+    const int row = q * 32 + lane;                // accumulator row of this thread
+    // The four epilogue warps walk every tile even after a failed wait (their waits then
+    // return at once), so the named barriers below are always reached by all of them.
+    uint32_t tc = 0;
+    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++tc) {
+      const TileCoord c = decode_tile(p, tile, MODE);
+      const GroupLayer& L = p.lay[c.g];
+      const int b = tc & 1;
+      const uint32_t use = tc >> 1;
+      const bool got = wait(&accfull[b], use & 1);
+      if (!got) atomicOr(p.err, kErrTimeoutEpilogue);
+      ptx::tc_fence_after();
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
+      const bool have = got && c.kb1 > c.kb0;
+
+      if (MODE == PROJECT) {
+        const int m = c.m_t * kBM + row;
+        __nv_bfloat16* AP = static_cast<__nv_bfloat16*>(L.out);
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          float v[32];
+          ptx::tmem_ld32(tbase + cc * 32, v);
+          if (have && m < L.M) {
+            uint4* dst = reinterpret_cast<uint4*>(AP + static_cast<size_t>(m) * L.ldo + c.n_t * BN + cc * 32);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              dst[u] = make_uint4(pack_bf16(v[8 * u + 0], v[8 * u + 1]), pack_bf16(v[8 * u + 2], v[8 * u + 3]),
+                                  pack_bf16(v[8 * u + 4], v[8 * u + 5]), pack_bf16(v[8 * u + 6], v[8 * u + 7]));
+          }
+        }
+      } else if (MODE == NORM) {
+        float ss = 0.0f;
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          float v[32];
+          ptx::tmem_ld32(tbase + cc * 32, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
+        }
+        if (!have) ss = 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        float* rb = red + (tc & 1) * 4;
+        if (lane == 0) rb[q] = ss;
+        epi_bar();
+        if (warp == 2 && lane == 0) {
+          const float tot = ((rb[0] + rb[1]) + rb[2]) + rb[3];
+          p.partials[static_cast<size_t>(c.s_t) * p.part_stride + L.part_base + c.m_t * L.nt + c.n_t] = tot;
+        }
+      } else if (MODE == AGGREGATE) {
+        const int m = c.m_t * kBM + row;
+        float* dst = static_cast<float*>(L.out);
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          float v[32];
+          ptx::tmem_ld32(tbase + cc * 32, v);
+          const int n0 = c.n_t * BN + cc * 32;
+          if (m < L.M) {
+            float* o = dst + static_cast<size_t>(m) * L.ldo + n0;
+            if (n0 + 32 <= L.N) {
+#pragma unroll
+              for (int u = 0; u < 8; ++u)
+                reinterpret_cast<float4*>(o)[u] =
+                    have ? make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3])
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+            } else {
+              for (int j = 0; j < 32 && n0 + j < L.N; ++j) o[j] = have ? v[j] : 0.0f;
+            }
+          }
+        }
+      } else {  // BACKPROJ: W -= lr * P dR
+        const int m = c.m_t * kBM + row;
+        float* Wm = static_cast<float*>(L.out) + static_cast<size_t>(m) * L.ldo;
+        const float lr = p.lr;
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          float v[32];
+          ptx::tmem_ld32(tbase + cc * 32, v);
+          const int n0 = c.n_t * BN + cc * 32;
+          if (have && m < L.M) {
+            if (n0 + 32 <= L.N) {
+              float4* w4 = reinterpret_cast<float4*>(Wm + n0);
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                float4 x = w4[u];
+                x.x = fmaf(-lr, v[4 * u + 0], x.x);
+                x.y = fmaf(-lr, v[4 * u + 1], x.y);
+                x.z = fmaf(-lr, v[4 * u + 2], x.z);
+                x.w = fmaf(-lr, v[4 * u + 3], x.w);
+                w4[u] = x;
+              }
+            } else {
+              for (int j = 0; j < 32 && n0 + j < L.N; ++j) Wm[n0 + j] = fmaf(-lr, v[j], Wm[n0 + j]);
+            }
+          }
+        }
+      }
+      // this accumulator may be overwritten by the tile after next
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&accempty[b]);
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---- aggregation with the K split across a thread-block cluster --------------------
+// For few output tiles (r x d_out is small next to K = B*T): the CS CTAs of a cluster
+// share one 128 x BN output tile of S and each runs 1/CS of the stacked token rows.
+// Their fp32 partial tiles meet in shared memory: after a cluster barrier, CTA k sums
+// rows [k*128/CS, (k+1)*128/CS) over the CS partials, read through distributed shared
+// memory in rank order (a fixed order: the result does not depend on timing), and
+// writes them to S.  No partial ever goes to global memory.
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __grid_constant__ GroupParams p) {
+  using S = Smem<BN, STAGES>;
+  constexpr uint32_t kTmemCols = BN;
+  constexpr uint32_t kIdesc = ptx::idesc_bf16(kBM, BN, true, true);
+  constexpr int kLd = BN + 4;   // staging row stride (floats): conflict-free row writes
+  static_assert(kBM * kLd * 4 <= STAGES * S::kStage, "staging must fit in the stage ring");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accfull = empty + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int CS = p.cluster;
+  const uint32_t rank = ptx::cluster_ctarank();
+  auto wait = [&](uint64_t* bar, uint32_t parity) {
+    return ptx::mbar_wait_or_abort(bar, parity, kWaitLimitNs, abort_flag);
+  };
+
+  // output tile of this cluster and this CTA's share of K
+  const TileCoord c = decode_tile(p, static_cast<int>(blockIdx.x) / CS, NORM);
+  const GroupLayer& L = p.lay[c.g];
+  const int kb0 = static_cast<int>(static_cast<int64_t>(rank) * L.kblocks / CS);
+  const int kb1 = static_cast<int>(static_cast<int64_t>(rank + 1) * L.kblocks / CS);
+
+  if (warp == 0 && lane == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    ptx::mbar_init(accfull, 1);
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&p.mapA[c.g]);
+    ptx::prefetch_tmap(&p.mapB[c.g]);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol = ptx::policy_evict_first();   // last use of AP and Gout in the step
+      const CUtensorMap* mapA = &p.mapA[c.g];
+      const CUtensorMap* mapB = &p.mapB[c.g];
+      for (int kb = kb0, it = 0; kb < kb1; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t use = it / STAGES;
+        if (use > 0 && !wait(&empty[s], (use - 1) & 1)) {
+          atomicOr(p.err, kErrTimeoutProducer);
+          break;
+        }
+        uint8_t* sa = smem + s * S::kStage;
+        uint8_t* sb = sa + S::kABytes;
+        ptx::mbar_arrive_expect_tx(&full[s], S::kStage);
+        const int kk = kb * kBK;
+#pragma unroll
+        for (int q = 0; q < kBM / 64; ++q)
+          ptx::tma_load_2d_hint(sa + q * 8192, mapA, &full[s], c.m_t * kBM + 64 * q, kk, pol);
+#pragma unroll
+        for (int q = 0; q < BN / 64; ++q)
+          ptx::tma_load_2d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kk, pol);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (int kb = kb0, it = 0; kb < kb1; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!wait(&full[s], ph)) {
           atomicOr(p.err, kErrTimeoutMma);
           break;
         }
@@ -207,145 +476,65 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         const uint32_t a_base = ptx::smem_u32(smem + s * S::kStage);
         const uint32_t b_base = a_base + S::kABytes;
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-          // K-major: next 16 elements are 32 bytes further along the swizzled row;
-          // M/N-major: next 16 K-rows are 16 x 128 bytes further.
-          const uint64_t ad = T::kAMn ? ptx::desc_sw128(a_base + kk * 2048, 8192, 1024)
-                                      : ptx::desc_sw128(a_base + kk * 32, 16, 1024);
-          const uint64_t bd = ptx::desc_sw128(b_base + kk * 2048, 8192, 1024);
-          ptx::umma_bf16(tmem, ad, bd, kIdesc, (k > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int k = 0; k < kBK / 16; ++k)
+          ptx::umma_bf16(tmem, ptx::desc_sw128(a_base + k * 2048, 8192, 1024),
+                         ptx::desc_sw128(b_base + k * 2048, 8192, 1024), kIdesc,
+                         (kb > kb0 || k > 0) ? 1u : 0u);
         ptx::umma_commit(&empty[s]);
       }
       ptx::umma_commit(accfull);
     }
   } else {
-    // ---------------- epilogue: warps 2..5 ----------------
-    const int q = warp & 3;                 // TMEM lanes 32q .. 32q+31
-    const int row = q * 32 + lane;          // accumulator row of this thread
-    const bool got = ptx::mbar_wait(accfull, 0, kWaitLimitNs);
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    // partial tile -> own shared memory (the stage ring is idle once the MMAs are done)
+    const bool got = wait(accfull, 0);
     if (!got) atomicOr(p.err, kErrTimeoutEpilogue);
     ptx::tc_fence_after();
+    float* stage = reinterpret_cast<float*>(smem);
     const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    const bool have = got && nkb > 0;
-
-    if (MODE == PROJECT) {
-      const int m = m_t * kBM + row;
-      __nv_bfloat16* AP = static_cast<__nv_bfloat16*>(L.out);
+    const bool have = got && kb1 > kb0;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        ptx::tmem_ld32(tbase + c * 32, v);
-        if (have && m < L.M) {
-          uint4* dst = reinterpret_cast<uint4*>(AP + static_cast<size_t>(m) * L.ldo + n_t * BN + c * 32);
+    for (int cc = 0; cc < BN / 32; ++cc) {
+      float v[32];
+      ptx::tmem_ld32(tbase + cc * 32, v);
+      float4* dst = reinterpret_cast<float4*>(stage + row * kLd + cc * 32);
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            dst[u] = make_uint4(pack_bf16(v[8 * u + 0], v[8 * u + 1]), pack_bf16(v[8 * u + 2], v[8 * u + 3]),
-                                pack_bf16(v[8 * u + 4], v[8 * u + 5]), pack_bf16(v[8 * u + 6], v[8 * u + 7]));
-        }
-      }
-    } else if (MODE == NORM) {
-      float ss = 0.0f;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        ptx::tmem_ld32(tbase + c * 32, v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
-      }
-      if (!have) ss = 0.0f;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      if (lane == 0) red[q] = ss;
-      epi_bar();
-      if (warp == 2 && lane == 0) {
-        const float tot = ((red[0] + red[1]) + red[2]) + red[3];
-        p.partials[static_cast<size_t>(s_t) * p.part_stride + L.part_base + m_t * L.nt + n_t] = tot;
-      }
-    } else if (MODE == AGGREGATE) {
-      const int m = m_t * kBM + row;
-      float* dst = (L.ns > 1) ? L.split_ws + static_cast<size_t>(s_t) * L.M * L.ldo
-                              : static_cast<float*>(L.out);
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        ptx::tmem_ld32(tbase + c * 32, v);
-        const int n0 = n_t * BN + c * 32;
-        if (m < L.M) {
-          float* o = dst + static_cast<size_t>(m) * L.ldo + n0;
-          if (n0 + 32 <= L.N) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              reinterpret_cast<float4*>(o)[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-          } else {
-            for (int j = 0; j < 32 && n0 + j < L.N; ++j) o[j] = v[j];
-          }
-        }
-      }
-      if (L.ns > 1) {
-        // Serial split-K fix-up: the last CTA of this output tile to arrive sums the
-        // partial copies in split order (0, 1, ...), so the result does not depend
-        // on which CTA arrives last.
-        __threadfence();
-        epi_bar();
-        if (warp == 2 && lane == 0) {
-          const int old = atomicAdd(&L.counters[m_t * L.nt + n_t], 1);
-          *flag = (old == L.ns - 1);
-        }
-        epi_bar();
-        if (*flag) {
-          __threadfence();
-          if (m < L.M) {
-            float* Sout = static_cast<float*>(L.out);
-            for (int c = 0; c < BN / 32; ++c) {
-              const int n0 = n_t * BN + c * 32;
-              for (int j = 0; j < 32; j += 4) {
-                if (n0 + j >= L.N) break;
-                const size_t o = static_cast<size_t>(m) * L.ldo + n0 + j;
-                float4 acc = *reinterpret_cast<const float4*>(L.split_ws + o);
-                for (int s = 1; s < L.ns; ++s) {
-                  const float4 x = *reinterpret_cast<const float4*>(
-                      L.split_ws + static_cast<size_t>(s) * L.M * L.ldo + o);
-                  acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
-                }
-                *reinterpret_cast<float4*>(Sout + o) = acc;
-              }
-            }
-          }
-          if (warp == 2 && lane == 0) L.counters[m_t * L.nt + n_t] = 0;
-        }
-      }
-    } else {  // BACKPROJ: W -= lr * P dR
-      const int m = m_t * kBM + row;
-      float* Wm = static_cast<float*>(L.out) + static_cast<size_t>(m) * L.ldo;
-      const float lr = p.lr;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        ptx::tmem_ld32(tbase + c * 32, v);
-        const int n0 = n_t * BN + c * 32;
-        if (have && m < L.M) {
-          if (n0 + 32 <= L.N) {
-            float4* w4 = reinterpret_cast<float4*>(Wm + n0);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              float4 x = w4[u];
-              x.x = fmaf(-lr, v[4 * u + 0], x.x);
-              x.y = fmaf(-lr, v[4 * u + 1], x.y);
-              x.z = fmaf(-lr, v[4 * u + 2], x.z);
-              x.w = fmaf(-lr, v[4 * u + 3], x.w);
-              w4[u] = x;
-            }
-          } else {
-            for (int j = 0; j < 32 && n0 + j < L.N; ++j) Wm[n0 + j] = fmaf(-lr, v[j], Wm[n0 + j]);
-          }
-        }
-      }
+      for (int u = 0; u < 8; ++u)
+        dst[u] = have ? make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3])
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
 
   ptx::tc_fence_before();
   __syncthreads();
+  __syncwarp();
+  ptx::cluster_sync();   // every partial tile of the cluster is in shared memory
+
+  if (warp >= 2) {
+    const int e = (warp - 2) * 32 + threadIdx.x % 32;
+    const int rows_per = kBM / CS;
+    const int r0 = static_cast<int>(rank) * rows_per;
+    const uint32_t stage_addr = ptx::smem_u32(smem);
+    float* Sout = static_cast<float*>(L.out);
+    const int n_f4 = rows_per * (BN / 4);
+    for (int idx = e; idx < n_f4; idx += 128) {
+      const int rr = r0 + idx / (BN / 4);
+      const int c4 = idx % (BN / 4);
+      const uint32_t off = static_cast<uint32_t>((rr * kLd + c4 * 4) * 4);
+      float4 acc = ptx::ld_dsmem_f4(ptx::mapa_shared(stage_addr + off, 0));
+      for (int j = 1; j < CS; ++j) {
+        const float4 x = ptx::ld_dsmem_f4(ptx::mapa_shared(stage_addr + off, j));
+        acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+      }
+      const int m = c.m_t * kBM + rr;
+      const int n = c.n_t * BN + c4 * 4;
+      if (m < L.M && n + 4 <= L.N)
+        *reinterpret_cast<float4*>(Sout + static_cast<size_t>(m) * L.ldo + n) = acc;
+    }
+  }
+  __syncwarp();
+  ptx::cluster_sync();   // no CTA leaves while another may still read its shared memory
   if (warp == 1) {
     __syncwarp();
     ptx::tc_fence_after();
@@ -372,17 +561,21 @@ __global__ void __launch_bounds__(256) gen_P_bf16_kernel(PTable t, uint64_t seed
   }
 }
 
-// ---- n_i, c_i, and AP rows of sample i scaled by c_i (all layers) -------------------
+// ---- n_i, c_i, and the clip folded into AP ------------------------------------------
+// Block (i, l): n_i = sqrt(sum of sample i's partial slots) in a fixed order (every
+// block of sample i computes the same bits), c_i = C/n_i if n_i > C else 1; block
+// (i, 0) records n_i and c_i, and block (i, l) rescales sample i's T rows of AP_l by
+// c_i in place, so the aggregation that follows is a plain GEMM:
+// sum_i c_i (A_i P)^T Gout_i = (diag(c) AP)^T Gout over the stacked rows.
 struct ApTable {
   __nv_bfloat16* AP[GRAPE_MAX_LAYERS];
 };
 
-__global__ void __launch_bounds__(256) clip_scale_kernel(ApTable t, int L, int r, int T, int part_stride,
-                                                         float C, const float* partials, float* norms,
-                                                         float* clip) {
+__global__ void __launch_bounds__(256) clip_scale_kernel(ApTable t, int r, int T, int part_stride, float C,
+                                                         const float* partials, float* norms, float* clip) {
   __shared__ float red[8];
   __shared__ float c_sh;
-  const int i = blockIdx.x;
+  const int i = blockIdx.x, l = blockIdx.y;
   const float* pp = partials + static_cast<size_t>(i) * part_stride;
   float ss = 0.0f;
   for (int k = threadIdx.x; k < part_stride; k += 256) ss += pp[k];
@@ -395,26 +588,26 @@ __global__ void __launch_bounds__(256) clip_scale_kernel(ApTable t, int L, int r
     for (int w = 0; w < 8; ++w) tot += red[w];
     const float n = sqrtf(tot);
     const float c = (n > C) ? C / n : 1.0f;
-    norms[i] = n;
-    clip[i] = c;
+    if (l == 0) {
+      norms[i] = n;
+      clip[i] = c;
+    }
     c_sh = c;
   }
   __syncthreads();
   const float c = c_sh;
   if (c == 1.0f) return;
+  uint4* rows = reinterpret_cast<uint4*>(t.AP[l] + static_cast<size_t>(i) * T * r);
   const size_t n8 = static_cast<size_t>(T) * r / 8;   // 8 bf16 per 16-byte vector
-  for (int l = 0; l < L; ++l) {
-    uint4* rows = reinterpret_cast<uint4*>(t.AP[l] + static_cast<size_t>(i) * T * r);
-    for (size_t k = threadIdx.x; k < n8; k += 256) {
-      uint4 x = rows[k];
-      __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&x);
+  for (size_t k = threadIdx.x; k < n8; k += 256) {
+    uint4 x = rows[k];
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&x);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float2 f = __bfloat1622float2(h[u]);
-        h[u] = __floats2bfloat162_rn(f.x * c, f.y * c);
-      }
-      rows[k] = x;
+    for (int u = 0; u < 4; ++u) {
+      const float2 f = __bfloat1622float2(h[u]);
+      h[u] = __floats2bfloat162_rn(f.x * c, f.y * c);
     }
+    rows[k] = x;
   }
 }
 
@@ -491,12 +684,15 @@ struct MapCache {
   }
 };
 
-constexpr int kBnProject = 128;    // r = 128: one N tile; larger r uses 256-wide tiles
 constexpr int kBnWide = 256;
-constexpr int kStagesProject = 4;
-constexpr int kStagesNorm = 4;
-constexpr int kStagesAgg = 4;
-constexpr int kStagesBack = 2;
+constexpr int kStagesProject128 = 3;   // 3 x 32 KB: two CTAs per SM
+constexpr int kStagesProject256 = 4;   // 4 x 48 KB
+constexpr int kStagesNorm = 4;         // 4 x 48 KB
+constexpr int kStagesAgg = 4;          // 4 x 48 KB
+constexpr int kBnBack = 128;
+constexpr int kStagesBack = 3;         // 3 x 32 KB: two CTAs per SM (TMEM 2 x 256 columns)
+constexpr int kBnAggCluster = 128;     // cluster-split aggregation: 6 x 32 KB
+constexpr int kStagesAggCluster = 6;
 
 struct HostState {
   int L = 0, r = 0, B = 0, T = 0;
@@ -509,10 +705,6 @@ struct HostState {
   std::vector<CUtensorMap> mapDR;       // dR as [r][d_out] (BACKPROJ B operand)
   // per-step maps, cached by pointer
   std::vector<MapCache> cacheA, cacheG3, cacheG2;
-  // aggregation split-K
-  std::vector<int> agg_ns;
-  std::vector<float*> agg_ws;
-  std::vector<int*> agg_cnt;
   int* err = nullptr;
   int bn_project = 128;
   GroupParams gp;   // host staging of one launch's kernel parameters
@@ -520,8 +712,21 @@ struct HostState {
 
 int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+// Persistent launch: as many CTAs as can be resident (shared memory and TMEM
+// columns both limit it), never more than there are tiles.
 template <int MODE, int BN, int STAGES>
-cudaError_t launch_group(const GroupParams& gp, int tiles, cudaStream_t st) {
+cudaError_t launch_group(GroupParams& gp, int tiles, cudaStream_t st) {
   using S = Smem<BN, STAGES>;
   static bool configured = false;
   if (!configured) {
@@ -530,7 +735,15 @@ cudaError_t launch_group(const GroupParams& gp, int tiles, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  tc_gemm_kernel<MODE, BN, STAGES><<<tiles, kThreads, S::kBytes, st>>>(gp);
+  gp.total_tiles = tiles;
+  if (tiles <= 0) return cudaSuccess;
+  int per_sm = (227 * 1024) / S::kBytes;
+  const int by_tmem = 512 / (2 * BN);
+  per_sm = per_sm < by_tmem ? per_sm : by_tmem;
+  per_sm = per_sm < 1 ? 1 : per_sm;
+  int grid = sm_count() * per_sm;
+  grid = grid < tiles ? grid : tiles;
+  tc_gemm_kernel<MODE, BN, STAGES><<<grid, kThreads, S::kBytes, st>>>(gp);
   return cudaGetLastError();
 }
 
@@ -590,28 +803,8 @@ bool tc_supported(int device, const grape_layer* layers, int n_layers, int r, in
 
 int tc_partials_per_sample(int r, int d_out) { return cdiv(r, kBM) * cdiv(d_out, kBnWide); }
 
-namespace {
-int agg_splits(int r, int d_out, int B, int T, int L) {
-  // aim for about two CTAs per SM over the whole launch group
-  const int tiles = cdiv(r, kBM) * cdiv(d_out, kBnWide) * (L < kMaxGroup ? L : kMaxGroup);
-  const int kblocks = cdiv(static_cast<int64_t>(B) * T, kBK);
-  int ns = cdiv(296, tiles);
-  if (ns > kblocks) ns = kblocks;
-  if (ns > 16) ns = 16;
-  return ns < 1 ? 1 : ns;
-}
-}  // namespace
-
-size_t tc_workspace_bytes(const StepShape& sh, const LayerWs* ws) {
-  size_t b = 256;  // error word
-  for (int l = 0; l < sh.L; ++l) {
-    const int ns = agg_splits(sh.r, ws[l].d_out, sh.B, sh.T, sh.L);
-    if (ns > 1) {
-      b += (static_cast<size_t>(ns) * sh.r * ws[l].d_out * 4 + 255) & ~size_t(255);
-      b += (static_cast<size_t>(cdiv(sh.r, kBM)) * cdiv(ws[l].d_out, kBnWide) * 4 + 255) & ~size_t(255);
-    }
-  }
-  return b;
+size_t tc_workspace_bytes(const StepShape&, const LayerWs*) {
+  return 256;  // error word
 }
 
 cudaError_t tc_init(const StepShape& sh, const LayerWs* ws, void* scratch, size_t bytes,
@@ -634,9 +827,6 @@ cudaError_t tc_init(const StepShape& sh, const LayerWs* ws, void* scratch, size_
   hs->cacheA.resize(sh.L);
   hs->cacheG3.resize(sh.L);
   hs->cacheG2.resize(sh.L);
-  hs->agg_ns.resize(sh.L);
-  hs->agg_ws.assign(sh.L, nullptr);
-  hs->agg_cnt.assign(sh.L, nullptr);
   const uint64_t rows = static_cast<uint64_t>(sh.B) * sh.T;
   for (int l = 0; l < sh.L; ++l) {
     hs->d_in.push_back(ws[l].d_in);
@@ -649,14 +839,6 @@ cudaError_t tc_init(const StepShape& sh, const LayerWs* ws, void* scratch, size_
     if (!ok) {
       delete hs;
       return cudaErrorInvalidValue;
-    }
-    const int ns = agg_splits(sh.r, ws[l].d_out, sh.B, sh.T, sh.L);
-    hs->agg_ns[l] = ns;
-    if (ns > 1) {
-      hs->agg_ws[l] = reinterpret_cast<float*>(base + off);
-      off += (static_cast<size_t>(ns) * sh.r * ws[l].d_out * 4 + 255) & ~size_t(255);
-      hs->agg_cnt[l] = reinterpret_cast<int*>(base + off);
-      off += (static_cast<size_t>(cdiv(sh.r, kBM)) * cdiv(ws[l].d_out, kBnWide) * 4 + 255) & ~size_t(255);
     }
   }
   if (off > bytes) {
@@ -723,8 +905,8 @@ cudaError_t tc_project(const StepShape& sh, const LayerWs* ws, const LayerIo* io
     return true;
   };
   if (hs.bn_project == 128)
-    return run_mode<PROJECT, 128, kStagesProject>(hs, sh.L, st, launches, fill, gp);
-  return run_mode<PROJECT, 256, kStagesProject>(hs, sh.L, st, launches, fill, gp);
+    return run_mode<PROJECT, 128, kStagesProject128>(hs, sh.L, st, launches, fill, gp);
+  return run_mode<PROJECT, 256, kStagesProject256>(hs, sh.L, st, launches, fill, gp);
 }
 
 cudaError_t tc_project_norm(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
@@ -760,41 +942,128 @@ cudaError_t tc_clip_scale(const StepShape& sh, const LayerWs* ws, const TcWorksp
                           int* launches) {
   ApTable t{};
   for (int l = 0; l < sh.L; ++l) t.AP[l] = static_cast<__nv_bfloat16*>(ws[l].AP);
-  clip_scale_kernel<<<sh.B, 256, 0, st>>>(t, sh.L, sh.r, sh.T, sh.part_stride, sh.C, partials, norms,
-                                          clip);
+  clip_scale_kernel<<<dim3(sh.B, sh.L), 256, 0, st>>>(t, sh.r, sh.T, sh.part_stride, sh.C, partials,
+                                                       norms, clip);
   ++*launches;
   return cudaGetLastError();
 }
 
+namespace {
+
+// How many clusters of `cs` CTAs of the aggregation kernel the device holds at once.
+template <int BN, int STAGES>
+int clusters_resident(int cs) {
+  static int cached[9] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
+  if (cs < 1 || cs > 8) return 0;
+  if (cached[cs] < 0) {
+    using S = Smem<BN, STAGES>;
+    cudaFuncSetAttribute(tc_agg_cluster_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         S::kBytes);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(cs);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = S::kBytes;
+    cudaLaunchAttribute a[1];
+    a[0].id = cudaLaunchAttributeClusterDimension;
+    a[0].val.clusterDim.x = cs;
+    a[0].val.clusterDim.y = 1;
+    a[0].val.clusterDim.z = 1;
+    cfg.attrs = a;
+    cfg.numAttrs = 1;
+    int n = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, tc_agg_cluster_kernel<BN, STAGES>, &cfg);
+    if (e != cudaSuccess) cudaGetLastError();
+    cached[cs] = (e == cudaSuccess) ? n : 0;
+  }
+  return cached[cs];
+}
+
+template <int BN, int STAGES>
+cudaError_t launch_agg_cluster(GroupParams& gp, int tiles, int cs, cudaStream_t st) {
+  using S = Smem<BN, STAGES>;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(tc_agg_cluster_kernel<BN, STAGES>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  gp.total_tiles = tiles;
+  gp.cluster = cs;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(tiles * cs);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = S::kBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute a[1];
+  a[0].id = cudaLaunchAttributeClusterDimension;
+  a[0].val.clusterDim.x = cs;
+  a[0].val.clusterDim.y = 1;
+  a[0].val.clusterDim.z = 1;
+  cfg.attrs = a;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc_agg_cluster_kernel<BN, STAGES>, gp);
+}
+
+}  // namespace
+
 cudaError_t tc_aggregate(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                          const TcWorkspace& tc, const float* clip, cudaStream_t st, int* launches) {
-  (void)clip;   // the clip factors were folded into AP by tc_clip_scale
+  (void)clip;   // folded into AP by tc_clip_scale
   HostState& hs = *static_cast<HostState*>(tc.host_state);
   GroupParams& gp = hs.gp;
-  std::memset(&gp, 0, sizeof(gp));
-  gp.err = hs.err;
   const int64_t rows = static_cast<int64_t>(sh.B) * sh.T;
-  auto fill = [&](int g, int l, int* tiles) {
-    gp.mapA[g] = hs.mapAP2[l];
-    if (!hs.cacheG2[l].get(io[l].G, &gp.mapB[g], [&](CUtensorMap* m) {
-          return map_2d(m, io[l].G, rows, ws[l].d_out, 64, 64);
-        }))
-      return false;
-    GroupLayer& L = gp.lay[g];
-    L.mt = cdiv(sh.r, kBM);
-    L.nt = cdiv(ws[l].d_out, kBnWide);
-    L.ns = hs.agg_ns[l];
-    L.kblocks = cdiv(rows, kBK);
-    L.M = sh.r;
-    L.N = ws[l].d_out;
-    L.ldo = ws[l].d_out;
-    L.out = ws[l].S;
-    L.split_ws = hs.agg_ws[l];
-    L.counters = hs.agg_cnt[l];
-    *tiles = L.mt * L.nt * L.ns;
-    return true;
-  };
-  return run_mode<AGGREGATE, kBnWide, kStagesAgg>(hs, sh.L, st, launches, fill, gp);
+  for (int l0 = 0; l0 < sh.L; l0 += kMaxGroup) {
+    const int n = (sh.L - l0) < kMaxGroup ? (sh.L - l0) : kMaxGroup;
+    // Output tiles of this group at the persistent kernel's width: with at least one
+    // tile per SM the persistent kernel runs K whole; with fewer, K is split over a
+    // cluster (the largest of 8, 4, 2 whose clusters are all resident at once).
+    int wide_tiles = 0;
+    for (int g = 0; g < n; ++g) wide_tiles += cdiv(sh.r, kBM) * cdiv(ws[l0 + g].d_out, kBnWide);
+    int cs = 1, narrow_tiles = 0;
+    if (wide_tiles < sm_count()) {
+      for (int g = 0; g < n; ++g) narrow_tiles += cdiv(sh.r, kBM) * cdiv(ws[l0 + g].d_out, kBnAggCluster);
+      for (int cand = 8; cand >= 2; cand /= 2)
+        if (narrow_tiles <= clusters_resident<kBnAggCluster, kStagesAggCluster>(cand)) {
+          cs = cand;
+          break;
+        }
+    }
+    const int bn = (cs > 1) ? kBnAggCluster : kBnWide;
+    if (std::getenv("GRAPE_DEBUG_PLAN"))
+      std::fprintf(stderr, "grape: aggregate layers %d..%d: %d wide tiles, cluster %d (resident clusters of 8/4/2: %d/%d/%d)\n",
+                   l0, l0 + n - 1, wide_tiles, cs, clusters_resident<kBnAggCluster, kStagesAggCluster>(8),
+                   clusters_resident<kBnAggCluster, kStagesAggCluster>(4),
+                   clusters_resident<kBnAggCluster, kStagesAggCluster>(2));
+    std::memset(&gp, 0, sizeof(gp));
+    gp.err = hs.err;
+    gp.n_layers = n;
+    int tiles = 0;
+    for (int g = 0; g < n; ++g) {
+      const int l = l0 + g;
+      gp.mapA[g] = hs.mapAP2[l];
+      if (!hs.cacheG2[l].get(io[l].G, &gp.mapB[g], [&](CUtensorMap* m) {
+            return map_2d(m, io[l].G, rows, ws[l].d_out, 64, 64);
+          }))
+        return cudaErrorInvalidValue;
+      GroupLayer& L = gp.lay[g];
+      L.tiles_begin = tiles;
+      L.mt = cdiv(sh.r, kBM);
+      L.nt = cdiv(ws[l].d_out, bn);
+      L.ns = 1;
+      L.kblocks = cdiv(rows, kBK);
+      L.M = sh.r;
+      L.N = ws[l].d_out;
+      L.ldo = ws[l].d_out;
+      L.out = ws[l].S;
+      tiles += L.mt * L.nt;
+    }
+    cudaError_t e = (cs > 1) ? launch_agg_cluster<kBnAggCluster, kStagesAggCluster>(gp, tiles, cs, st)
+                             : launch_group<AGGREGATE, kBnWide, kStagesAgg>(gp, tiles, st);
+    if (e != cudaSuccess) return e;
+    ++*launches;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t tc_backproject(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
@@ -809,7 +1078,7 @@ cudaError_t tc_backproject(const StepShape& sh, const LayerWs* ws, const LayerIo
     gp.mapB[g] = hs.mapDR[l];
     GroupLayer& L = gp.lay[g];
     L.mt = cdiv(ws[l].d_in, kBM);
-    L.nt = cdiv(ws[l].d_out, kBnWide);
+    L.nt = cdiv(ws[l].d_out, kBnBack);
     L.ns = 1;
     L.kblocks = cdiv(sh.r, kBK);
     L.M = ws[l].d_in;
@@ -819,7 +1088,7 @@ cudaError_t tc_backproject(const StepShape& sh, const LayerWs* ws, const LayerIo
     *tiles = L.mt * L.nt;
     return true;
   };
-  return run_mode<BACKPROJ, kBnWide, kStagesBack>(hs, sh.L, st, launches, fill, gp);
+  return run_mode<BACKPROJ, kBnBack, kStagesBack>(hs, sh.L, st, launches, fill, gp);
 }
 
 // ---------------------------------------------------------------------------------
@@ -931,8 +1200,8 @@ cudaError_t tc_layer_sqnorms_static(const void* A, const void* G, int d_in, int 
   L.N = r;
   L.ldo = r;
   L.out = AP;
-  e = (bnp == 128) ? launch_group<PROJECT, 128, kStagesProject>(gp, L.mt * L.nt, st)
-                   : launch_group<PROJECT, 256, kStagesProject>(gp, L.mt * L.nt, st);
+  e = (bnp == 128) ? launch_group<PROJECT, 128, kStagesProject128>(gp, L.mt * L.nt, st)
+                   : launch_group<PROJECT, 256, kStagesProject256>(gp, L.mt * L.nt, st);
   if (e != cudaSuccess) return e;
   // ||(A_i P)^T Gout_i||^2 per sample, as partial slots
   std::memset(&gp, 0, sizeof(gp));
