@@ -50,7 +50,8 @@ namespace {
 
 constexpr int kBM = 128;           // UMMA M (one CTA, TMEM lanes)
 constexpr int kBK = 64;            // K per stage: one 128-byte swizzle row of bf16
-constexpr int kThreads = 192;      // 6 warps
+constexpr int kThreads = 320;      // 10 warps: TMA, MMA, 8 epilogue
+constexpr int kEpiWarps = 8;       // two per TMEM lane quarter, each on half the columns
 constexpr int kMaxGroup = 16;      // layers per launch
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 
@@ -74,6 +75,7 @@ struct GroupLayer {
 struct GroupParams {
   CUtensorMap mapA[kMaxGroup];
   CUtensorMap mapB[kMaxGroup];
+  CUtensorMap mapW[kMaxGroup];   // BACKPROJ: W as fp32 (32-column x 128-row boxes)
   GroupLayer lay[kMaxGroup];
   int n_layers;
   int total_tiles;
@@ -90,16 +92,29 @@ struct ModeTraits {
   static constexpr bool kB3d = (MODE == NORM);
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int EXTRA = 0>
 struct Smem {
   static constexpr int kABytes = kBM * kBK * 2;
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStage = kABytes + kBBytes;
   static constexpr int kBarOff = STAGES * kStage;
-  static constexpr int kBytes = kBarOff + 512 + 1024;   // + barriers + alignment slack
+  // after the barriers, on a 1024-byte boundary (128-byte-swizzled TMA boxes live there)
+  static constexpr int kExtraOff = ((kBarOff + 512 + 1023) / 1024) * 1024;
+  static constexpr int kBytes = kExtraOff + EXTRA + 1024;  // + alignment slack
+  static_assert(kStage % 1024 == 0 && kExtraOff % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 };
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// BACKPROJ: two W tiles (128 rows x 128 fp32 columns, as four 128B-swizzled boxes of
+// 32 columns) so the TMA load of the next tile's W overlaps this tile's update.
+constexpr int kBnBack = 128;
+constexpr int kWBox = kBM * 128;                 // one 32-column box: 16 KB
+constexpr int kWTile = (kBnBack / 32) * kWBox;   // 64 KB
+template <int MODE>
+struct ModeExtra {
+  static constexpr int kBytes = (MODE == BACKPROJ) ? 2 * kWTile : 0;
+};
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -134,9 +149,10 @@ __device__ __forceinline__ TileCoord decode_tile(const GroupParams& p, int tile,
 template <int MODE, int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ GroupParams p) {
   using T = ModeTraits<MODE>;
-  using S = Smem<BN, STAGES>;
+  using S = Smem<BN, STAGES, ModeExtra<MODE>::kBytes>;
   constexpr uint32_t kTmemCols = 2 * BN;
   constexpr uint32_t kIdesc = ptx::idesc_bf16(kBM, BN, T::kAMn, true);
+  static_assert(BN % 128 == 0, "each epilogue warp takes BN/2 columns in 64-column loads");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -146,8 +162,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   uint64_t* accfull = empty + STAGES;       // [2]
   uint64_t* accempty = accfull + 2;         // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + 2);
-  float* red = reinterpret_cast<float*>(tmem_slot + 2);   // [2][4]
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(red + 8);
+  float* red = reinterpret_cast<float*>(tmem_slot + 2);   // [2][kEpiWarps]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(red + 2 * kEpiWarps);
+  uint64_t* wfull = reinterpret_cast<uint64_t*>(smem + S::kBarOff + 448);   // BACKPROJ [2]
+  uint64_t* wfree = wfull + 2;                                              // BACKPROJ [2]
+  static_assert(2 * STAGES * 8 + 4 * 8 + 8 + 2 * kEpiWarps * 4 + 4 <= 448, "barrier area");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto wait = [&](uint64_t* bar, uint32_t parity) {
@@ -162,12 +181,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&accfull[b], 1);
-      ptx::mbar_init(&accempty[b], 4);
+      ptx::mbar_init(&accempty[b], kEpiWarps);
+      ptx::mbar_init(&wfull[b], 1);
+      ptx::mbar_init(&wfree[b], 1);
     }
     ptx::fence_mbar_init();
     for (int g = 0; g < p.n_layers; ++g) {
       ptx::prefetch_tmap(&p.mapA[g]);
       ptx::prefetch_tmap(&p.mapB[g]);
+      if (MODE == BACKPROJ) ptx::prefetch_tmap(&p.mapW[g]);
     }
   }
   if (warp == 1) {
@@ -184,15 +206,32 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     if (lane == 0) {
       // A and Gout stream once per use; P, AP and dR are re-read by other tiles or
       // by the next phase, so they are kept in L2 preferentially.
-      const uint64_t polA = (MODE == PROJECT || MODE == AGGREGATE) ? ptx::policy_evict_first()
-                                                                     : ptx::policy_evict_last();
+      const uint64_t polA = (MODE == PROJECT || MODE == AGGREGATE || MODE == BACKPROJ)
+                                ? ptx::policy_evict_first()
+                                : ptx::policy_evict_last();
       const uint64_t polB = (MODE == AGGREGATE) ? ptx::policy_evict_first() : ptx::policy_evict_last();
-      uint32_t it = 0;
+      uint32_t it = 0, tcp = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+      for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++tcp) {
         const TileCoord c = decode_tile(p, tile, MODE);
         const CUtensorMap* mapA = &p.mapA[c.g];
         const CUtensorMap* mapB = &p.mapB[c.g];
+        if (MODE == BACKPROJ) {
+          // this tile's W into buffer tcp & 1, once the store of the tile before last
+          // has finished reading it
+          const int wb = tcp & 1;
+          const uint32_t wuse = tcp >> 1;
+          if (wuse > 0 && !wait(&wfree[wb], (wuse - 1) & 1)) {
+            atomicOr(p.err, kErrTimeoutProducer);
+            break;
+          }
+          uint8_t* wbuf = smem + S::kExtraOff + wb * kWTile;
+          ptx::mbar_arrive_expect_tx(&wfull[wb], kWTile);
+#pragma unroll
+          for (int q = 0; q < kBnBack / 32; ++q)
+            ptx::tma_load_2d_hint(wbuf + q * kWBox, &p.mapW[c.g], &wfull[wb], c.n_t * kBnBack + 32 * q,
+                                  c.m_t * kBM, polA);
+        }
         for (int kb = c.kb0; kb < c.kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t use = it / STAGES;
@@ -206,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
           ptx::mbar_arrive_expect_tx(&full[s], S::kStage);
           const int kk = kb * kBK;
           if (MODE == PROJECT || MODE == BACKPROJ) {
-            ptx::tma_load_2d_hint(sa, mapA, &full[s], kk, c.m_t * kBM, polA);
+            ptx::tma_load_2d_hint(sa, mapA, &full[s], kk, c.m_t * kBM, MODE == BACKPROJ ? polB : polA);
           } else if (MODE == NORM) {
 #pragma unroll
             for (int q = 0; q < kBM / 64; ++q)
@@ -267,10 +306,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       }
     }
   } else {
-    // ---------------- epilogue: warps 2..5 ----------------
+    // ---------------- epilogue: warps 2..9 ----------------
+    // Warp w reads TMEM lanes 32*(w%4).. (its lane quarter, a hardware rule) and half
+    // h = (w-2)/4 of the accumulator's columns, 64 columns per load.
+    const int ew = warp - 2;                      // 0..7
     const int q = warp & 3;                       // TMEM lanes 32q .. 32q+31
+    const int h = ew >> 2;                        // column half
     const int row = q * 32 + lane;                // accumulator row of this thread
-    // The four epilogue warps walk every tile even after a failed wait (their waits then
+    constexpr int kHalf = BN / 2;
+    // The epilogue warps walk every tile even after a failed wait (their waits then
     // return at once), so the named barriers below are always reached by all of them.
     uint32_t tc = 0;
     for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++tc) {
@@ -281,20 +325,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       const bool got = wait(&accfull[b], use & 1);
       if (!got) atomicOr(p.err, kErrTimeoutEpilogue);
       ptx::tc_fence_after();
-      const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * BN + h * kHalf;
+      const int col0 = c.n_t * BN + h * kHalf;    // first output column of this warp
       const bool have = got && c.kb1 > c.kb0;
 
       if (MODE == PROJECT) {
         const int m = c.m_t * kBM + row;
         __nv_bfloat16* AP = static_cast<__nv_bfloat16*>(L.out);
 #pragma unroll 1
-        for (int cc = 0; cc < BN / 32; ++cc) {
-          float v[32];
-          ptx::tmem_ld32(tbase + cc * 32, v);
+        for (int cc = 0; cc < kHalf; cc += 64) {
+          float v[64];
+          ptx::tmem_ld64(tbase + cc, v);
           if (have && m < L.M) {
-            uint4* dst = reinterpret_cast<uint4*>(AP + static_cast<size_t>(m) * L.ldo + c.n_t * BN + cc * 32);
+            uint4* dst = reinterpret_cast<uint4*>(AP + static_cast<size_t>(m) * L.ldo + col0 + cc);
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+            for (int u = 0; u < 8; ++u)
               dst[u] = make_uint4(pack_bf16(v[8 * u + 0], v[8 * u + 1]), pack_bf16(v[8 * u + 2], v[8 * u + 3]),
                                   pack_bf16(v[8 * u + 4], v[8 * u + 5]), pack_bf16(v[8 * u + 6], v[8 * u + 7]));
           }
@@ -302,68 +347,85 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       } else if (MODE == NORM) {
         float ss = 0.0f;
 #pragma unroll 1
-        for (int cc = 0; cc < BN / 32; ++cc) {
-          float v[32];
-          ptx::tmem_ld32(tbase + cc * 32, v);
+        for (int cc = 0; cc < kHalf; cc += 64) {
+          float v[64];
+          ptx::tmem_ld64(tbase + cc, v);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
+          for (int j = 0; j < 64; ++j) ss = fmaf(v[j], v[j], ss);
         }
         if (!have) ss = 0.0f;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        float* rb = red + (tc & 1) * 4;
-        if (lane == 0) rb[q] = ss;
+        float* rb = red + (tc & 1) * kEpiWarps;
+        if (lane == 0) rb[ew] = ss;
         epi_bar();
-        if (warp == 2 && lane == 0) {
-          const float tot = ((rb[0] + rb[1]) + rb[2]) + rb[3];
+        if (ew == 0 && lane == 0) {
+          float tot = 0.0f;
+#pragma unroll
+          for (int k = 0; k < kEpiWarps; ++k) tot += rb[k];
           p.partials[static_cast<size_t>(c.s_t) * p.part_stride + L.part_base + c.m_t * L.nt + c.n_t] = tot;
         }
       } else if (MODE == AGGREGATE) {
         const int m = c.m_t * kBM + row;
         float* dst = static_cast<float*>(L.out);
 #pragma unroll 1
-        for (int cc = 0; cc < BN / 32; ++cc) {
-          float v[32];
-          ptx::tmem_ld32(tbase + cc * 32, v);
-          const int n0 = c.n_t * BN + cc * 32;
+        for (int cc = 0; cc < kHalf; cc += 64) {
+          float v[64];
+          ptx::tmem_ld64(tbase + cc, v);
+          const int n0 = col0 + cc;
           if (m < L.M) {
             float* o = dst + static_cast<size_t>(m) * L.ldo + n0;
-            if (n0 + 32 <= L.N) {
+            if (n0 + 64 <= L.N) {
 #pragma unroll
-              for (int u = 0; u < 8; ++u)
+              for (int u = 0; u < 16; ++u)
                 reinterpret_cast<float4*>(o)[u] =
                     have ? make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3])
                          : make_float4(0.f, 0.f, 0.f, 0.f);
             } else {
-              for (int j = 0; j < 32 && n0 + j < L.N; ++j) o[j] = have ? v[j] : 0.0f;
+              for (int j = 0; j < 64 && n0 + j < L.N; ++j) o[j] = have ? v[j] : 0.0f;
             }
           }
         }
-      } else {  // BACKPROJ: W -= lr * P dR
-        const int m = c.m_t * kBM + row;
-        float* Wm = static_cast<float*>(L.out) + static_cast<size_t>(m) * L.ldo;
+      } else {  // BACKPROJ: W -= lr * P dR on the W tile in shared memory, then TMA store
+        const bool wgot = wait(&wfull[b], use & 1);
+        if (!wgot) atomicOr(p.err, kErrTimeoutEpilogue);
+        uint8_t* wbuf = smem + S::kExtraOff + b * kWTile;
         const float lr = p.lr;
 #pragma unroll 1
-        for (int cc = 0; cc < BN / 32; ++cc) {
-          float v[32];
-          ptx::tmem_ld32(tbase + cc * 32, v);
-          const int n0 = c.n_t * BN + cc * 32;
-          if (have && m < L.M) {
-            if (n0 + 32 <= L.N) {
-              float4* w4 = reinterpret_cast<float4*>(Wm + n0);
+        for (int cc = 0; cc < kHalf; cc += 64) {
+          float v[64];
+          ptx::tmem_ld64(tbase + cc, v);
+          if (have && wgot) {
+            // columns h*kHalf + cc + [0, 64): two 32-column boxes; 16-byte unit u of
+            // row `row` sits at unit u ^ (row & 7) (128-byte swizzle)
+#pragma unroll
+            for (int bx = 0; bx < 2; ++bx) {
+              uint8_t* box = wbuf + ((h * kHalf + cc) / 32 + bx) * kWBox + row * 128;
 #pragma unroll
               for (int u = 0; u < 8; ++u) {
-                float4 x = w4[u];
-                x.x = fmaf(-lr, v[4 * u + 0], x.x);
-                x.y = fmaf(-lr, v[4 * u + 1], x.y);
-                x.z = fmaf(-lr, v[4 * u + 2], x.z);
-                x.w = fmaf(-lr, v[4 * u + 3], x.w);
-                w4[u] = x;
+                float4* w4 = reinterpret_cast<float4*>(box + ((u ^ (row & 7)) * 16));
+                float4 x = *w4;
+                const int j = bx * 32 + u * 4;
+                x.x = fmaf(-lr, v[j + 0], x.x);
+                x.y = fmaf(-lr, v[j + 1], x.y);
+                x.z = fmaf(-lr, v[j + 2], x.z);
+                x.w = fmaf(-lr, v[j + 3], x.w);
+                *w4 = x;
               }
-            } else {
-              for (int j = 0; j < 32 && n0 + j < L.N; ++j) Wm[n0 + j] = fmaf(-lr, v[j], Wm[n0 + j]);
             }
           }
+        }
+        ptx::fence_proxy_async_smem();   // the W tile is next read by the TMA store
+        epi_bar();
+        if (ew == 0 && lane == 0) {
+          if (have && wgot) {
+#pragma unroll
+            for (int q2 = 0; q2 < kBnBack / 32; ++q2)
+              ptx::tma_store_2d(&p.mapW[c.g], wbuf + q2 * kWBox, c.n_t * kBnBack + 32 * q2, c.m_t * kBM);
+            ptx::bulk_commit_group();
+            ptx::bulk_wait_group_read0();
+          }
+          ptx::mbar_arrive(&wfree[b]);
         }
       }
       // this accumulator may be overwritten by the tile after next
@@ -373,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     }
   }
 
+  if (MODE == BACKPROJ && warp == 2 && lane == 0) ptx::bulk_wait_group0();   // W stores complete
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -396,6 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
   constexpr uint32_t kIdesc = ptx::idesc_bf16(kBM, BN, true, true);
   constexpr int kLd = BN + 4;   // staging row stride (floats): conflict-free row writes
   static_assert(kBM * kLd * 4 <= STAGES * S::kStage, "staging must fit in the stage ring");
+  static_assert(BN % 128 == 0, "each epilogue warp stages BN/2 columns in 64-column loads");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -485,22 +549,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
       ptx::umma_commit(accfull);
     }
   } else {
-    const int q = warp & 3;
+    const int q = warp & 3;                 // TMEM lane quarter
+    const int h = (warp - 2) >> 2;          // column half
     const int row = q * 32 + lane;
     // partial tile -> own shared memory (the stage ring is idle once the MMAs are done)
     const bool got = wait(accfull, 0);
     if (!got) atomicOr(p.err, kErrTimeoutEpilogue);
     ptx::tc_fence_after();
     float* stage = reinterpret_cast<float*>(smem);
-    const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * (BN / 2);
     const bool have = got && kb1 > kb0;
 #pragma unroll 1
-    for (int cc = 0; cc < BN / 32; ++cc) {
-      float v[32];
-      ptx::tmem_ld32(tbase + cc * 32, v);
-      float4* dst = reinterpret_cast<float4*>(stage + row * kLd + cc * 32);
+    for (int cc = 0; cc < BN / 2; cc += 64) {
+      float v[64];
+      ptx::tmem_ld64(tbase + cc, v);
+      float4* dst = reinterpret_cast<float4*>(stage + row * kLd + h * (BN / 2) + cc);
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
+      for (int u = 0; u < 16; ++u)
         dst[u] = have ? make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3])
                       : make_float4(0.f, 0.f, 0.f, 0.f);
     }
@@ -518,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
     const uint32_t stage_addr = ptx::smem_u32(smem);
     float* Sout = static_cast<float*>(L.out);
     const int n_f4 = rows_per * (BN / 4);
-    for (int idx = e; idx < n_f4; idx += 128) {
+    for (int idx = e; idx < n_f4; idx += 32 * kEpiWarps) {
       const int rr = r0 + idx / (BN / 4);
       const int c4 = idx % (BN / 4);
       const uint32_t off = static_cast<uint32_t>((rr * kLd + c4 * 4) * 4);
@@ -642,6 +707,19 @@ bool map_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint3
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 row-major [rows][cols] as a 2-D map with a (32 x 128) box, 128-byte swizzle.
+bool map_2d_f32(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {32, kBM};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // bf16 [B][T][cols] as a 3-D map with a (64 x 64 x 1) box: rows past T read as zero.
 bool map_3d(CUtensorMap* m, const void* ptr, uint64_t B, uint64_t T, uint64_t cols) {
   auto enc = encode_fn();
@@ -689,8 +767,7 @@ constexpr int kStagesProject128 = 3;   // 3 x 32 KB: two CTAs per SM
 constexpr int kStagesProject256 = 4;   // 4 x 48 KB
 constexpr int kStagesNorm = 4;         // 4 x 48 KB
 constexpr int kStagesAgg = 4;          // 4 x 48 KB
-constexpr int kBnBack = 128;
-constexpr int kStagesBack = 3;         // 3 x 32 KB: two CTAs per SM (TMEM 2 x 256 columns)
+constexpr int kStagesBack = 2;         // 2 x 32 KB stages + 2 x 64 KB W tiles
 constexpr int kBnAggCluster = 128;     // cluster-split aggregation: 6 x 32 KB
 constexpr int kStagesAggCluster = 6;
 
@@ -704,7 +781,7 @@ struct HostState {
   std::vector<CUtensorMap> mapAP2;      // AP as [B*T][r] (AGGREGATE A operand)
   std::vector<CUtensorMap> mapDR;       // dR as [r][d_out] (BACKPROJ B operand)
   // per-step maps, cached by pointer
-  std::vector<MapCache> cacheA, cacheG3, cacheG2;
+  std::vector<MapCache> cacheA, cacheG3, cacheG2, cacheW;
   int* err = nullptr;
   int bn_project = 128;
   GroupParams gp;   // host staging of one launch's kernel parameters
@@ -727,7 +804,7 @@ int sm_count() {
 // columns both limit it), never more than there are tiles.
 template <int MODE, int BN, int STAGES>
 cudaError_t launch_group(GroupParams& gp, int tiles, cudaStream_t st) {
-  using S = Smem<BN, STAGES>;
+  using S = Smem<BN, STAGES, ModeExtra<MODE>::kBytes>;
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<MODE, BN, STAGES>,
@@ -827,6 +904,7 @@ cudaError_t tc_init(const StepShape& sh, const LayerWs* ws, void* scratch, size_
   hs->cacheA.resize(sh.L);
   hs->cacheG3.resize(sh.L);
   hs->cacheG2.resize(sh.L);
+  hs->cacheW.resize(sh.L);
   const uint64_t rows = static_cast<uint64_t>(sh.B) * sh.T;
   for (int l = 0; l < sh.L; ++l) {
     hs->d_in.push_back(ws[l].d_in);
@@ -1076,6 +1154,10 @@ cudaError_t tc_backproject(const StepShape& sh, const LayerWs* ws, const LayerIo
   auto fill = [&](int g, int l, int* tiles) {
     gp.mapA[g] = hs.mapP_k[l];
     gp.mapB[g] = hs.mapDR[l];
+    if (!hs.cacheW[l].get(io[l].W, &gp.mapW[g], [&](CUtensorMap* m) {
+          return map_2d_f32(m, io[l].W, ws[l].d_in, ws[l].d_out);
+        }))
+      return false;
     GroupLayer& L = gp.lay[g];
     L.mt = cdiv(ws[l].d_in, kBM);
     L.nt = cdiv(ws[l].d_out, kBnBack);

@@ -1,0 +1,92 @@
+"""Data-parallel orchestration on two gloo ranks (CPU, no GPU).
+
+dp_step (random_gradient_projection_b200/data_parallel.py) runs, on every rank,
+accumulate -> all-reduce of every S_l -> apply(batch_total = B * world).  Here each
+rank drives a stand-in context that computes its shard with the fp64 oracle, so the
+test checks the orchestration itself: which tensors are reduced, in which order, and
+the global batch used for the average.  Two ranks of 3 samples each must reproduce the
+single-process oracle step on all 6 samples, and the two replicas must agree exactly.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle.grape_oracle as O
+import workloads as W
+
+
+def _workload():
+    return W.Workload("dp", ((24, 16), (16, 12)), r=8, B=6, T=5, dtype="f32", C=0.9,
+                      sigma=0.7, steps=2)
+
+
+class OracleShard:
+    """Implements the methods dp_step calls, for the samples `rows` of the batch."""
+
+    def __init__(self, w, rows, W0):
+        self.w, self.rows = w, list(rows)
+        self.layers = list(w.layers)
+        self.B = len(self.rows)
+        self.h = O.Hyper.of(w)
+        self.state = O.State.init(W0, w.r)
+        self.S = None
+
+    def accumulate(self, A, Gout, step, stream=None):
+        Ps = [O.projection_matrix(self.h.seed, l, step, di, self.h.r)
+              for l, (di, _) in enumerate(self.layers)]
+        R = O.projected_per_sample(A, Gout, Ps, range(self.B))
+        norms = [np.sqrt(sum(np.sum(R[i][l] ** 2) for l in range(len(Ps)))) for i in range(self.B)]
+        c = [O.clip_factor(n, self.h.C) for n in norms]
+        self.P = Ps
+        self.S = [torch.from_numpy(sum(c[i] * R[i][l] for i in range(self.B)).copy())
+                  for l in range(len(Ps))]
+
+    def S_tensor(self, l):
+        return self.S[l]
+
+    def apply(self, Wt, step, batch_total, stream=None):
+        t = step + 1
+        for l, (di, do) in enumerate(self.layers):
+            xi = O.noise_matrix(self.h.seed, l, step, self.h.r, do)
+            g = (self.S[l].numpy() + self.h.sigma * self.h.C * xi) / batch_total
+            self.state.m[l], self.state.v[l], d = O.adam(self.state.m[l], self.state.v[l], g, t,
+                                                         self.h.beta1, self.h.beta2, self.h.eps)
+            Wt[l] -= torch.from_numpy(self.h.lr * (self.P[l] @ d))
+
+
+def _rank(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    from random_gradient_projection_b200.data_parallel import dp_step
+    w = _workload()
+    per = w.B // world
+    rows = range(rank * per, (rank + 1) * per)
+    W0 = W.make_weights(w)
+    g = OracleShard(w, rows, W0)
+    Wt = [torch.from_numpy(x.astype(np.float64)) for x in W0]
+    for s in range(w.steps):
+        x = W.make_step_inputs(w, s, samples=list(rows))
+        A = [x.as_f64(a) for a in x.A]
+        G = [x.as_f64(gg) for gg in x.Gout]
+        dp_step(g, A, G, Wt, s)
+    out[rank] = [t.numpy().copy() for t in Wt]
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_rank_dp_step_equals_full_batch_oracle():
+    world = 2
+    port = 29500 + os.getpid() % 1000
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_rank, args=(world, port, out), nprocs=world, start_method="spawn", join=True)
+    w = _workload()
+    ref = O.run(w, w.steps)["state"]
+    for l in range(w.n_layers):
+        assert np.array_equal(out[0][l], out[1][l])          # replicas identical
+        assert np.allclose(out[0][l], ref.W[l], rtol=0, atol=1e-13), l
