@@ -215,7 +215,7 @@ int run_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_total
   const grape::LayerWs* ws = ctx->ws.data();
   int rc = phase(ctx, GRAPE_PHASE_ADAM, "noise + adam", st, [&](int* n) {
     *n = 1;
-    return grape::noise_adam(sh, ws, u, tc, st);
+    return grape::noise_adam(sh, ws, u, tc, tc, st);
   });
   if (rc) return rc;
   return phase(ctx, GRAPE_PHASE_BACKPROJECT, "back-project", st, [&](int* n) {

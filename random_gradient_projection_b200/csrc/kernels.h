@@ -60,8 +60,9 @@ cudaError_t finalize_clip(const StepShape& sh, const float* partials, float* nor
                           cudaStream_t st);
 cudaError_t simt_aggregate(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                            const float* clip, cudaStream_t st);
+// pdl: launch as a programmatic dependent of the previous kernel (tensor-core path).
 cudaError_t noise_adam(const StepShape& sh, const LayerWs* ws, const UpdateScalars& u,
-                       bool dR_bf16, cudaStream_t st);
+                       bool dR_bf16, bool pdl, cudaStream_t st);
 cudaError_t simt_backproject(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                              float lr, cudaStream_t st);
 int simt_partials_per_sample(int r, int d_out);

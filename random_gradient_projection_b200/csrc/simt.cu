@@ -212,6 +212,10 @@ __global__ void __launch_bounds__(kThreads) aggregate_kernel(StepShape sh, Layer
 // xi_l[e] = z(seed, l, s, stream 1, e), e = j*d_out + n.  One thread per block of 4.
 __global__ void __launch_bounds__(256) noise_adam_kernel(StepShape sh, LayerTable tab,
                                                          UpdateScalars u, int dR_bf16) {
+  // When launched as a programmatic dependent (tensor-core path): let the back-projection
+  // be scheduled, then wait for S.  Both are no-ops after an ordinary launch.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int l = blockIdx.y;
   const LayerWs& w = tab.ws[l];
   const int64_t n = static_cast<int64_t>(sh.r) * w.d_out;
@@ -366,12 +370,24 @@ cudaError_t simt_aggregate(const StepShape& sh, const LayerWs* ws, const LayerIo
 }
 
 cudaError_t noise_adam(const StepShape& sh, const LayerWs* ws, const UpdateScalars& u, bool dR_bf16,
-                       cudaStream_t st) {
+                       bool pdl, cudaStream_t st) {
   const LayerTable t = make_table(sh, ws, nullptr);
   const int64_t q = (static_cast<int64_t>(sh.r) * max_d_out(sh, ws) + 3) / 4;
   dim3 grid(cdiv(q, 256) < 592 ? cdiv(q, 256) : 592, sh.L);
-  noise_adam_kernel<<<grid, 256, 0, st>>>(sh, t, u, dR_bf16 ? 1 : 0);
-  return cudaGetLastError();
+  if (!pdl) {
+    noise_adam_kernel<<<grid, 256, 0, st>>>(sh, t, u, dR_bf16 ? 1 : 0);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute a[1];
+  a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = a;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, noise_adam_kernel, sh, t, u, dR_bf16 ? 1 : 0);
 }
 
 cudaError_t simt_backproject(const StepShape& sh, const LayerWs* ws, const LayerIo* io, float lr,

@@ -54,6 +54,7 @@ constexpr int kThreads = 320;      // 10 warps: TMA, MMA, 8 epilogue
 constexpr int kEpiWarps = 8;       // two per TMEM lane quarter, each on half the columns
 constexpr int kMaxGroup = 16;      // layers per launch
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
+constexpr uint64_t kDrainLimitNs = 1000000000ull;   // after an abort: wait for loads in flight
 
 enum Mode : int { PROJECT = 0, NORM = 1, AGGREGATE = 2, BACKPROJ = 3 };
 
@@ -172,6 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   auto wait = [&](uint64_t* bar, uint32_t parity) {
     return ptx::mbar_wait_or_abort(bar, parity, kWaitLimitNs, abort_flag);
   };
+  ptx::griddep_launch_dependents();
 
   if (warp == 0 && lane == 0) {
     *abort_flag = 0;
@@ -210,13 +212,70 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                                 ? ptx::policy_evict_first()
                                 : ptx::policy_evict_last();
       const uint64_t polB = (MODE == AGGREGATE) ? ptx::policy_evict_first() : ptx::policy_evict_last();
+      auto load_a = [&](const TileCoord& c, int kb, int s) {
+        uint8_t* sa = smem + s * S::kStage;
+        const CUtensorMap* mapA = &p.mapA[c.g];
+        const int kk = kb * kBK;
+        if (MODE == PROJECT || MODE == BACKPROJ) {
+          ptx::tma_load_2d_hint(sa, mapA, &full[s], kk, c.m_t * kBM, MODE == BACKPROJ ? polB : polA);
+        } else if (MODE == NORM) {
+#pragma unroll
+          for (int q = 0; q < kBM / 64; ++q)
+            ptx::tma_load_3d_hint(sa + q * 8192, mapA, &full[s], c.m_t * kBM + 64 * q, kk, c.s_t, polA);
+        } else {
+#pragma unroll
+          for (int q = 0; q < kBM / 64; ++q)
+            ptx::tma_load_2d_hint(sa + q * 8192, mapA, &full[s], c.m_t * kBM + 64 * q, kk, polA);
+        }
+      };
+      auto load_b = [&](const TileCoord& c, int kb, int s) {
+        uint8_t* sb = smem + s * S::kStage + S::kABytes;
+        const CUtensorMap* mapB = &p.mapB[c.g];
+        const int kk = kb * kBK;
+#pragma unroll
+        for (int q = 0; q < BN / 64; ++q) {
+          if (T::kB3d)
+            ptx::tma_load_3d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kk, c.s_t, polB);
+          else
+            ptx::tma_load_2d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kk, polB);
+        }
+      };
+      auto load_w = [&](const TileCoord& c, int wb) {
+        uint8_t* wbuf = smem + S::kExtraOff + wb * kWTile;
+        ptx::mbar_arrive_expect_tx(&wfull[wb], kWTile);
+#pragma unroll
+        for (int q = 0; q < kBnBack / 32; ++q)
+          ptx::tma_load_2d_hint(wbuf + q * kWBox, &p.mapW[c.g], &wfull[wb], c.n_t * kBnBack + 32 * q,
+                                c.m_t * kBM, polA);
+      };
+
+      // Before waiting for the previous kernel of the step, load what predates the step:
+      // A (PROJECT) or Gout (NORM, AGGREGATE) for the first stages, W of the first tile
+      // (BACKPROJ).  P, AP and dR are written earlier in this step and load after the wait.
+      constexpr int kEarly = (MODE == PROJECT) ? 0 : (MODE == BACKPROJ ? -1 : 1);
+      uint32_t pre = 0, wissued = 0;
+      if (kEarly >= 0) {
+        for (int tile = blockIdx.x; pre < static_cast<uint32_t>(STAGES) && tile < p.total_tiles;
+             tile += gridDim.x) {
+          const TileCoord c = decode_tile(p, tile, MODE);
+          for (int kb = c.kb0; kb < c.kb1 && pre < static_cast<uint32_t>(STAGES); ++kb, ++pre) {
+            ptx::mbar_arrive_expect_tx(&full[pre], S::kStage);
+            if (kEarly == 0) load_a(c, kb, pre);
+            else load_b(c, kb, pre);
+          }
+        }
+      }
+      if (MODE == BACKPROJ && static_cast<int>(blockIdx.x) < p.total_tiles) {
+        load_w(decode_tile(p, blockIdx.x, MODE), 0);
+        wissued = 1;
+      }
+      ptx::griddep_wait();
+
       uint32_t it = 0, tcp = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++tcp) {
         const TileCoord c = decode_tile(p, tile, MODE);
-        const CUtensorMap* mapA = &p.mapA[c.g];
-        const CUtensorMap* mapB = &p.mapB[c.g];
-        if (MODE == BACKPROJ) {
+        if (MODE == BACKPROJ && tcp > 0) {
           // this tile's W into buffer tcp & 1, once the store of the tile before last
           // has finished reading it
           const int wb = tcp & 1;
@@ -225,44 +284,34 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             atomicOr(p.err, kErrTimeoutProducer);
             break;
           }
-          uint8_t* wbuf = smem + S::kExtraOff + wb * kWTile;
-          ptx::mbar_arrive_expect_tx(&wfull[wb], kWTile);
-#pragma unroll
-          for (int q = 0; q < kBnBack / 32; ++q)
-            ptx::tma_load_2d_hint(wbuf + q * kWBox, &p.mapW[c.g], &wfull[wb], c.n_t * kBnBack + 32 * q,
-                                  c.m_t * kBM, polA);
+          load_w(c, wb);
+          ++wissued;
         }
         for (int kb = c.kb0; kb < c.kb1; ++kb, ++it) {
           const int s = it % STAGES;
+          if (it < pre) {   // its early operand is already on the way
+            if (kEarly == 0) load_b(c, kb, s);
+            else load_a(c, kb, s);
+            continue;
+          }
           const uint32_t use = it / STAGES;
           if (use > 0 && !wait(&empty[s], (use - 1) & 1)) {
             atomicOr(p.err, kErrTimeoutProducer);
             ok = false;
             break;
           }
-          uint8_t* sa = smem + s * S::kStage;
-          uint8_t* sb = sa + S::kABytes;
           ptx::mbar_arrive_expect_tx(&full[s], S::kStage);
-          const int kk = kb * kBK;
-          if (MODE == PROJECT || MODE == BACKPROJ) {
-            ptx::tma_load_2d_hint(sa, mapA, &full[s], kk, c.m_t * kBM, MODE == BACKPROJ ? polB : polA);
-          } else if (MODE == NORM) {
-#pragma unroll
-            for (int q = 0; q < kBM / 64; ++q)
-              ptx::tma_load_3d_hint(sa + q * 8192, mapA, &full[s], c.m_t * kBM + 64 * q, kk, c.s_t, polA);
-          } else {
-#pragma unroll
-            for (int q = 0; q < kBM / 64; ++q)
-              ptx::tma_load_2d_hint(sa + q * 8192, mapA, &full[s], c.m_t * kBM + 64 * q, kk, polA);
-          }
-#pragma unroll
-          for (int q = 0; q < BN / 64; ++q) {
-            if (T::kB3d)
-              ptx::tma_load_3d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kk, c.s_t, polB);
-            else
-              ptx::tma_load_2d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kk, polB);
-          }
+          load_a(c, kb, s);
+          load_b(c, kb, s);
         }
+      }
+      if (*abort_flag) {
+        // leave no TMA load in flight into this CTA's shared memory
+        for (uint32_t k = it > STAGES ? it - STAGES : 0; k < it; ++k)
+          ptx::mbar_wait(&full[k % STAGES], (k / STAGES) & 1, kDrainLimitNs);
+        if (MODE == BACKPROJ)
+          for (uint32_t k = wissued > 2 ? wissued - 2 : 0; k < wissued; ++k)
+            ptx::mbar_wait(&wfull[k & 1], (k >> 1) & 1, kDrainLimitNs);
       }
     }
   } else if (warp == 1) {
@@ -472,6 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int CS = p.cluster;
+  ptx::griddep_launch_dependents();
   const uint32_t rank = ptx::cluster_ctarank();
   auto wait = [&](uint64_t* bar, uint32_t parity) {
     return ptx::mbar_wait_or_abort(bar, parity, kWaitLimitNs, abort_flag);
@@ -508,24 +558,42 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
       const uint64_t pol = ptx::policy_evict_first();   // last use of AP and Gout in the step
       const CUtensorMap* mapA = &p.mapA[c.g];
       const CUtensorMap* mapB = &p.mapB[c.g];
+      // Gout predates the step: its first stages load before waiting for the clip kernel;
+      // AP (rescaled by that kernel) loads after.
+      const int pre = (kb1 - kb0) < STAGES ? (kb1 - kb0) : STAGES;
+      for (int it = 0; it < pre; ++it) {
+        uint8_t* sb = smem + it * S::kStage + S::kABytes;
+        ptx::mbar_arrive_expect_tx(&full[it], S::kStage);
+#pragma unroll
+        for (int q = 0; q < BN / 64; ++q)
+          ptx::tma_load_2d_hint(sb + q * 8192, mapB, &full[it], c.n_t * BN + 64 * q, (kb0 + it) * kBK, pol);
+      }
+      ptx::griddep_wait();
+      uint32_t issued = pre;
       for (int kb = kb0, it = 0; kb < kb1; ++kb, ++it) {
         const int s = it % STAGES;
-        const uint32_t use = it / STAGES;
-        if (use > 0 && !wait(&empty[s], (use - 1) & 1)) {
-          atomicOr(p.err, kErrTimeoutProducer);
-          break;
-        }
         uint8_t* sa = smem + s * S::kStage;
         uint8_t* sb = sa + S::kABytes;
-        ptx::mbar_arrive_expect_tx(&full[s], S::kStage);
         const int kk = kb * kBK;
+        if (it >= pre) {
+          const uint32_t use = it / STAGES;
+          if (use > 0 && !wait(&empty[s], (use - 1) & 1)) {
+            atomicOr(p.err, kErrTimeoutProducer);
+            break;
+          }
+          ++issued;
+          ptx::mbar_arrive_expect_tx(&full[s], S::kStage);
+#pragma unroll
+          for (int q = 0; q < BN / 64; ++q)
+            ptx::tma_load_2d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kk, pol);
+        }
 #pragma unroll
         for (int q = 0; q < kBM / 64; ++q)
           ptx::tma_load_2d_hint(sa + q * 8192, mapA, &full[s], c.m_t * kBM + 64 * q, kk, pol);
-#pragma unroll
-        for (int q = 0; q < BN / 64; ++q)
-          ptx::tma_load_2d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kk, pol);
       }
+      if (*abort_flag)
+        for (uint32_t k = issued > STAGES ? issued - STAGES : 0; k < issued; ++k)
+          ptx::mbar_wait(&full[k % STAGES], (k / STAGES) & 1, kDrainLimitNs);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -614,6 +682,7 @@ struct PTable {
 };
 
 __global__ void __launch_bounds__(256) gen_P_bf16_kernel(PTable t, uint64_t seed, uint32_t step, int r) {
+  ptx::griddep_launch_dependents();
   const int l = blockIdx.y;
   const int64_t nq = static_cast<int64_t>(t.d_in[l]) * r / 4;   // r is a multiple of 64
   const float scale = rsqrtf(static_cast<float>(r));
@@ -640,6 +709,8 @@ __global__ void __launch_bounds__(256) clip_scale_kernel(ApTable t, int r, int T
                                                          const float* partials, float* norms, float* clip) {
   __shared__ float red[8];
   __shared__ float c_sh;
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();   // the norm partials, and AP no longer read by the norm kernel
   const int i = blockIdx.x, l = blockIdx.y;
   const float* pp = partials + static_cast<size_t>(i) * part_stride;
   float ss = 0.0f;
@@ -789,6 +860,23 @@ struct HostState {
 
 int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
+// Launch as a programmatic dependent of the previous kernel in the stream (the kernel
+// itself waits with griddepcontrol.wait before it reads that kernel's outputs).
+template <class Kern, class... Args>
+cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute a[1];
+  a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = a;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 int sm_count() {
   static int n = 0;
   if (n == 0) {
@@ -820,8 +908,7 @@ cudaError_t launch_group(GroupParams& gp, int tiles, cudaStream_t st) {
   per_sm = per_sm < 1 ? 1 : per_sm;
   int grid = sm_count() * per_sm;
   grid = grid < tiles ? grid : tiles;
-  tc_gemm_kernel<MODE, BN, STAGES><<<grid, kThreads, S::kBytes, st>>>(gp);
-  return cudaGetLastError();
+  return launch_pdl(tc_gemm_kernel<MODE, BN, STAGES>, dim3(grid), dim3(kThreads), S::kBytes, st, gp);
 }
 
 // Build and launch the groups of one mode.  fill(g, l, gp) sets maps and the layer record
@@ -1020,10 +1107,9 @@ cudaError_t tc_clip_scale(const StepShape& sh, const LayerWs* ws, const TcWorksp
                           int* launches) {
   ApTable t{};
   for (int l = 0; l < sh.L; ++l) t.AP[l] = static_cast<__nv_bfloat16*>(ws[l].AP);
-  clip_scale_kernel<<<dim3(sh.B, sh.L), 256, 0, st>>>(t, sh.r, sh.T, sh.part_stride, sh.C, partials,
-                                                       norms, clip);
   ++*launches;
-  return cudaGetLastError();
+  return launch_pdl(clip_scale_kernel, dim3(sh.B, sh.L), dim3(256), 0, st, t, sh.r, sh.T, sh.part_stride,
+                    sh.C, partials, norms, clip);
 }
 
 namespace {
@@ -1073,13 +1159,15 @@ cudaError_t launch_agg_cluster(GroupParams& gp, int tiles, int cs, cudaStream_t 
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = S::kBytes;
   cfg.stream = st;
-  cudaLaunchAttribute a[1];
+  cudaLaunchAttribute a[2];
   a[0].id = cudaLaunchAttributeClusterDimension;
   a[0].val.clusterDim.x = cs;
   a[0].val.clusterDim.y = 1;
   a[0].val.clusterDim.z = 1;
+  a[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = a;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, tc_agg_cluster_kernel<BN, STAGES>, gp);
 }
 

@@ -162,6 +162,16 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---- programmatic dependent launch ----------------------------------------------------
+// Let the next kernel in the stream be scheduled (it still waits for this one to finish
+// before it touches this kernel's outputs).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until the previous kernel in the stream has completed and its memory is visible
+// (returns at once when this kernel was not launched as a programmatic dependent).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---- thread-block clusters / distributed shared memory -----------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
