@@ -341,6 +341,26 @@ def main(argv=None):
     ms_per_step = ms / args.steps
     samples_per_s = world * w.B * args.steps / (ms / 1e3)
 
+    # ---- the same steps from a cold L2: a 256 MB write before each step, each step timed
+    # alone with events (the write is outside the timed intervals) ------------------------
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    cold_ms = 0.0
+    n_cold = min(args.steps, 50)
+    for _ in range(n_cold):
+        flush.fill_(step & 0xFF)
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        one(step)
+        c1.record(stream)
+        step += 1
+        torch.cuda.synchronize()
+        cold_ms += c0.elapsed_time(c1)
+    if world > 1:
+        t = torch.tensor([cold_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        cold_ms = float(t.item())
+    del flush
+
     # ---- per-phase device time (same K steps, events between phases) --------------------
     g.profile(True)
     for _ in range(args.steps):
@@ -421,7 +441,10 @@ def main(argv=None):
                        "path": path_name, "parallelism": f"dp{world}",
                        "l2": f"inputs rotate over {INPUT_SETS} distinct sets of "
                              f"{set_bytes / 1e6:.0f} MB each (> 126 MB L2)",
-                       "tokens_per_s": samples_per_s * w.T},
+                       "tokens_per_s": samples_per_s * w.T,
+                       "cold_l2": {"ms_per_step": cold_ms / n_cold,
+                                   "value": world * w.B * n_cold / (cold_ms / 1e3),
+                                   "how": f"{n_cold} steps, each after a 256 MB write, timed one by one"}},
             "roofline": {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,
                          "unit": unit, "frac": achieved / peak, "traffic": traffic,
                          "peak_source": pk["source"] if bound != "alu" else
