@@ -14,13 +14,17 @@
 // with Gradient Random Projection": per-sample projection, norms for clipping,
 // aggregation, and the projected update of the parameters).
 //
-// CTA layout (192 threads): warp 0 issues TMA loads into a ring of shared-memory
-// stages (128-byte swizzle), warp 1 owns the TMEM allocation and one of its
-// threads issues tcgen05.mma (M = 128, N = BN, K = 16 per instruction) into a
-// 128 x BN fp32 TMEM accumulator, warps 2-5 read the accumulator back with
-// tcgen05.ld (each warp its 32 TMEM lanes) and run the epilogue.  Stage reuse
-// is tracked with mbarriers (TMA completion -> full, tcgen05.commit -> empty);
-// every wait is bounded and reports a timeout through an error word.
+// CTA layout (352 threads, one CTA per SM: the runtime places a single CTA of a kernel
+// that allocates TMEM on each SM): warps 0 and 10 issue the TMA loads of the A and the
+// B operand into a ring of shared-memory stages (128-byte swizzle) -- one issuing
+// thread per operand, because one thread's TMA stream tops out near 6 TB/s of SM
+// ingress over the whole GPU while two reach about 11 TB/s; warp 1 owns the TMEM
+// allocation and one of its threads issues tcgen05.mma (M = 128, N = BN, K = 16 per
+// instruction) into one of two 128 x BN fp32 TMEM accumulators; warps 2-9 read the
+// accumulator back with tcgen05.ld (each warp its 32 TMEM lanes) and run the
+// epilogue.  Stage reuse is tracked with mbarriers (TMA completion -> fullA / fullB,
+// tcgen05.commit -> empty); every wait is bounded and reports a timeout through an
+// error word.
 //
 // Operands: A, P (as the A operand of BACKPROJ) are K-major tiles of 128 rows x
 // 64 bf16; AP^T (NORM / AGGREGATE) and every B operand (P, Gout, dR) are
@@ -50,8 +54,9 @@ namespace {
 
 constexpr int kBM = 128;           // UMMA M (one CTA, TMEM lanes)
 constexpr int kBK = 64;            // K per stage: one 128-byte swizzle row of bf16
-constexpr int kThreads = 320;      // 10 warps: TMA, MMA, 8 epilogue
 constexpr int kEpiWarps = 8;       // two per TMEM lane quarter, each on half the columns
+constexpr int kProdBWarp = 2 + kEpiWarps;        // warp 0: TMA A, 1: MMA, 2..9: epilogue, 10: TMA B
+constexpr int kThreads = 32 * (kProdBWarp + 1);  // 352
 constexpr int kMaxGroup = 16;      // layers per launch
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr uint64_t kDrainLimitNs = 1000000000ull;   // after an abort: wait for loads in flight
@@ -158,8 +163,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
-  uint64_t* empty = full + STAGES;
+  uint64_t* fullA = reinterpret_cast<uint64_t*>(smem + S::kBarOff);   // A operand landed
+  uint64_t* fullB = fullA + STAGES;                                     // B operand landed
+  uint64_t* empty = fullB + STAGES;
   uint64_t* accfull = empty + STAGES;       // [2]
   uint64_t* accempty = accfull + 2;         // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + 2);
@@ -167,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   volatile int* abort_flag = reinterpret_cast<volatile int*>(red + 2 * kEpiWarps);
   uint64_t* wfull = reinterpret_cast<uint64_t*>(smem + S::kBarOff + 448);   // BACKPROJ [2]
   uint64_t* wfree = wfull + 2;                                              // BACKPROJ [2]
-  static_assert(2 * STAGES * 8 + 4 * 8 + 8 + 2 * kEpiWarps * 4 + 4 <= 448, "barrier area");
+  static_assert(3 * STAGES * 8 + 4 * 8 + 8 + 2 * kEpiWarps * 4 + 4 <= 448, "barrier area");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto wait = [&](uint64_t* bar, uint32_t parity) {
@@ -178,7 +184,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   if (warp == 0 && lane == 0) {
     *abort_flag = 0;
     for (int s = 0; s < STAGES; ++s) {
-      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&fullA[s], 1);
+      ptx::mbar_init(&fullB[s], 1);
       ptx::mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -203,9 +210,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ---------------- TMA producer ----------------
+  if (warp == 0 || warp == kProdBWarp) {
+    // ---------------- TMA producers: warp 0 the A operand, warp 10 the B operand ----------------
     if (lane == 0) {
+      const bool isA = (warp == 0);
       // A and Gout stream once per use; P, AP and dR are re-read by other tiles or
       // by the next phase, so they are kept in L2 preferentially.
       const uint64_t polA = (MODE == PROJECT || MODE == AGGREGATE || MODE == BACKPROJ)
@@ -217,15 +225,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         const CUtensorMap* mapA = &p.mapA[c.g];
         const int kk = kb * kBK;
         if (MODE == PROJECT || MODE == BACKPROJ) {
-          ptx::tma_load_2d_hint(sa, mapA, &full[s], kk, c.m_t * kBM, MODE == BACKPROJ ? polB : polA);
+          ptx::tma_load_2d_hint(sa, mapA, &fullA[s], kk, c.m_t * kBM, MODE == BACKPROJ ? polB : polA);
         } else if (MODE == NORM) {
 #pragma unroll
           for (int q = 0; q < kBM / 64; ++q)
-            ptx::tma_load_3d_hint(sa + q * 8192, mapA, &full[s], c.m_t * kBM + 64 * q, kk, c.s_t, polA);
+            ptx::tma_load_3d_hint(sa + q * 8192, mapA, &fullA[s], c.m_t * kBM + 64 * q, kk, c.s_t, polA);
         } else {
 #pragma unroll
           for (int q = 0; q < kBM / 64; ++q)
-            ptx::tma_load_2d_hint(sa + q * 8192, mapA, &full[s], c.m_t * kBM + 64 * q, kk, polA);
+            ptx::tma_load_2d_hint(sa + q * 8192, mapA, &fullA[s], c.m_t * kBM + 64 * q, kk, polA);
         }
       };
       auto load_b = [&](const TileCoord& c, int kb, int s) {
@@ -235,9 +243,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
 #pragma unroll
         for (int q = 0; q < BN / 64; ++q) {
           if (T::kB3d)
-            ptx::tma_load_3d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kk, c.s_t, polB);
+            ptx::tma_load_3d_hint(sb + q * 8192, mapB, &fullB[s], c.n_t * BN + 64 * q, kk, c.s_t, polB);
           else
-            ptx::tma_load_2d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kk, polB);
+            ptx::tma_load_2d_hint(sb + q * 8192, mapB, &fullB[s], c.n_t * BN + 64 * q, kk, polB);
         }
       };
       auto load_w = [&](const TileCoord& c, int wb) {
@@ -249,33 +257,25 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                                 c.m_t * kBM, polA);
       };
 
-      // Before waiting for the previous kernel of the step, load what predates the step:
-      // A (PROJECT) or Gout (NORM, AGGREGATE) for the first stages, W of the first tile
-      // (BACKPROJ).  P, AP and dR are written earlier in this step and load after the wait.
-      constexpr int kEarly = (MODE == PROJECT) ? 0 : (MODE == BACKPROJ ? -1 : 1);
-      uint32_t pre = 0, wissued = 0;
-      if (kEarly >= 0) {
-        for (int tile = blockIdx.x; pre < static_cast<uint32_t>(STAGES) && tile < p.total_tiles;
-             tile += gridDim.x) {
-          const TileCoord c = decode_tile(p, tile, MODE);
-          for (int kb = c.kb0; kb < c.kb1 && pre < static_cast<uint32_t>(STAGES); ++kb, ++pre) {
-            ptx::mbar_arrive_expect_tx(&full[pre], S::kStage);
-            if (kEarly == 0) load_a(c, kb, pre);
-            else load_b(c, kb, pre);
-          }
-        }
-      }
-      if (MODE == BACKPROJ && static_cast<int>(blockIdx.x) < p.total_tiles) {
+      // The operand that predates the step -- A (PROJECT) or Gout (NORM, AGGREGATE) --
+      // streams without waiting for the previous kernel of the step; P, AP and dR are
+      // written earlier in this step and load after the wait.  W of the first tile
+      // (BACKPROJ) also loads before it.
+      const bool predates = isA ? (MODE == PROJECT) : (MODE == NORM || MODE == AGGREGATE);
+      uint64_t* full = isA ? fullA : fullB;
+      const uint32_t bytes = isA ? S::kABytes : S::kBBytes;
+      uint32_t wissued = 0;
+      if (MODE == BACKPROJ && !isA && static_cast<int>(blockIdx.x) < p.total_tiles) {
         load_w(decode_tile(p, blockIdx.x, MODE), 0);
         wissued = 1;
       }
-      ptx::griddep_wait();
+      if (!predates) ptx::griddep_wait();
 
       uint32_t it = 0, tcp = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++tcp) {
         const TileCoord c = decode_tile(p, tile, MODE);
-        if (MODE == BACKPROJ && tcp > 0) {
+        if (MODE == BACKPROJ && !isA && tcp > 0) {
           // this tile's W into buffer tcp & 1, once the store of the tile before last
           // has finished reading it
           const int wb = tcp & 1;
@@ -289,27 +289,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         }
         for (int kb = c.kb0; kb < c.kb1; ++kb, ++it) {
           const int s = it % STAGES;
-          if (it < pre) {   // its early operand is already on the way
-            if (kEarly == 0) load_b(c, kb, s);
-            else load_a(c, kb, s);
-            continue;
-          }
           const uint32_t use = it / STAGES;
           if (use > 0 && !wait(&empty[s], (use - 1) & 1)) {
             atomicOr(p.err, kErrTimeoutProducer);
             ok = false;
             break;
           }
-          ptx::mbar_arrive_expect_tx(&full[s], S::kStage);
-          load_a(c, kb, s);
-          load_b(c, kb, s);
+          ptx::mbar_arrive_expect_tx(&full[s], bytes);
+          if (isA)
+            load_a(c, kb, s);
+          else
+            load_b(c, kb, s);
         }
       }
       if (*abort_flag) {
-        // leave no TMA load in flight into this CTA's shared memory
+        // leave none of this thread's TMA loads in flight into this CTA's shared memory
         for (uint32_t k = it > STAGES ? it - STAGES : 0; k < it; ++k)
           ptx::mbar_wait(&full[k % STAGES], (k / STAGES) & 1, kDrainLimitNs);
-        if (MODE == BACKPROJ)
+        if (MODE == BACKPROJ && !isA)
           for (uint32_t k = wissued > 2 ? wissued - 2 : 0; k < wissued; ++k)
             ptx::mbar_wait(&wfull[k & 1], (k >> 1) & 1, kDrainLimitNs);
       }
@@ -332,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         for (int kb = c.kb0; kb < c.kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
-          if (!wait(&full[s], ph)) {
+          if (!wait(&fullA[s], ph) || !wait(&fullB[s], ph)) {
             atomicOr(p.err, kErrTimeoutMma);
             ok = false;
             break;
@@ -354,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         ptx::umma_commit(&accfull[b]);
       }
     }
-  } else {
+  } else if (warp < 2 + kEpiWarps) {
     // ---------------- epilogue: warps 2..9 ----------------
     // Warp w reads TMEM lanes 32*(w%4).. (its lane quarter, a hardware rule) and half
     // h = (w-2)/4 of the accumulator's columns, 64 columns per load.
@@ -513,8 +510,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
-  uint64_t* empty = full + STAGES;
+  uint64_t* fullA = reinterpret_cast<uint64_t*>(smem + S::kBarOff);   // AP stage landed
+  uint64_t* fullB = fullA + STAGES;                                     // Gout stage landed
+  uint64_t* empty = fullB + STAGES;
   uint64_t* accfull = empty + STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
@@ -536,7 +534,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
   if (warp == 0 && lane == 0) {
     *abort_flag = 0;
     for (int s = 0; s < STAGES; ++s) {
-      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&fullA[s], 1);
+      ptx::mbar_init(&fullB[s], 1);
       ptx::mbar_init(&empty[s], 1);
     }
     ptx::mbar_init(accfull, 1);
@@ -553,43 +552,30 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == 0 || warp == kProdBWarp) {
+    // warp 0 loads AP (rescaled by the clip kernel, so after the wait for it); warp 10
+    // loads Gout, which predates the step, without that wait.
     if (lane == 0) {
+      const bool isA = (warp == 0);
       const uint64_t pol = ptx::policy_evict_first();   // last use of AP and Gout in the step
-      const CUtensorMap* mapA = &p.mapA[c.g];
-      const CUtensorMap* mapB = &p.mapB[c.g];
-      // Gout predates the step: its first stages load before waiting for the clip kernel;
-      // AP (rescaled by that kernel) loads after.
-      const int pre = (kb1 - kb0) < STAGES ? (kb1 - kb0) : STAGES;
-      for (int it = 0; it < pre; ++it) {
-        uint8_t* sb = smem + it * S::kStage + S::kABytes;
-        ptx::mbar_arrive_expect_tx(&full[it], S::kStage);
-#pragma unroll
-        for (int q = 0; q < BN / 64; ++q)
-          ptx::tma_load_2d_hint(sb + q * 8192, mapB, &full[it], c.n_t * BN + 64 * q, (kb0 + it) * kBK, pol);
-      }
-      ptx::griddep_wait();
-      uint32_t issued = pre;
-      for (int kb = kb0, it = 0; kb < kb1; ++kb, ++it) {
-        const int s = it % STAGES;
-        uint8_t* sa = smem + s * S::kStage;
-        uint8_t* sb = sa + S::kABytes;
-        const int kk = kb * kBK;
-        if (it >= pre) {
-          const uint32_t use = it / STAGES;
-          if (use > 0 && !wait(&empty[s], (use - 1) & 1)) {
-            atomicOr(p.err, kErrTimeoutProducer);
-            break;
-          }
-          ++issued;
-          ptx::mbar_arrive_expect_tx(&full[s], S::kStage);
-#pragma unroll
-          for (int q = 0; q < BN / 64; ++q)
-            ptx::tma_load_2d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kk, pol);
+      const CUtensorMap* map = isA ? &p.mapA[c.g] : &p.mapB[c.g];
+      uint64_t* full = isA ? fullA : fullB;
+      const uint32_t bytes = isA ? S::kABytes : S::kBBytes;
+      const int chunks = isA ? kBM / 64 : BN / 64;
+      const int col0 = isA ? c.m_t * kBM : c.n_t * BN;
+      if (isA) ptx::griddep_wait();
+      uint32_t issued = 0;
+      for (int kb = kb0; kb < kb1; ++kb, ++issued) {
+        const int s = issued % STAGES;
+        const uint32_t use = issued / STAGES;
+        if (use > 0 && !wait(&empty[s], (use - 1) & 1)) {
+          atomicOr(p.err, kErrTimeoutProducer);
+          break;
         }
-#pragma unroll
-        for (int q = 0; q < kBM / 64; ++q)
-          ptx::tma_load_2d_hint(sa + q * 8192, mapA, &full[s], c.m_t * kBM + 64 * q, kk, pol);
+        uint8_t* dst = smem + s * S::kStage + (isA ? 0 : S::kABytes);
+        ptx::mbar_arrive_expect_tx(&full[s], bytes);
+        for (int q = 0; q < chunks; ++q)
+          ptx::tma_load_2d_hint(dst + q * 8192, map, &full[s], col0 + 64 * q, kb * kBK, pol);
       }
       if (*abort_flag)
         for (uint32_t k = issued > STAGES ? issued - STAGES : 0; k < issued; ++k)
@@ -600,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
       for (int kb = kb0, it = 0; kb < kb1; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
-        if (!wait(&full[s], ph)) {
+        if (!wait(&fullA[s], ph) || !wait(&fullB[s], ph)) {
           atomicOr(p.err, kErrTimeoutMma);
           break;
         }
@@ -616,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
       }
       ptx::umma_commit(accfull);
     }
-  } else {
+  } else if (warp < 2 + kEpiWarps) {
     const int q = warp & 3;                 // TMEM lane quarter
     const int h = (warp - 2) >> 2;          // column half
     const int row = q * 32 + lane;
@@ -644,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
   __syncwarp();
   ptx::cluster_sync();   // every partial tile of the cluster is in shared memory
 
-  if (warp >= 2) {
+  if (warp >= 2 && warp < 2 + kEpiWarps) {
     const int e = (warp - 2) * 32 + threadIdx.x % 32;
     const int rows_per = kBM / CS;
     const int r0 = static_cast<int>(rank) * rows_per;
@@ -834,11 +820,12 @@ struct MapCache {
 };
 
 constexpr int kBnWide = 256;
-constexpr int kStagesProject128 = 3;   // 3 x 32 KB: two CTAs per SM
+// One CTA per SM, so each ring takes most of the 227 KB of shared memory.
+constexpr int kStagesProject128 = 6;   // 6 x 32 KB
 constexpr int kStagesProject256 = 4;   // 4 x 48 KB
 constexpr int kStagesNorm = 4;         // 4 x 48 KB
 constexpr int kStagesAgg = 4;          // 4 x 48 KB
-constexpr int kStagesBack = 2;         // 2 x 32 KB stages + 2 x 64 KB W tiles
+constexpr int kStagesBack = 3;         // 3 x 32 KB stages + 2 x 64 KB W tiles
 constexpr int kBnAggCluster = 128;     // cluster-split aggregation: 6 x 32 KB
 constexpr int kStagesAggCluster = 6;
 
@@ -888,24 +875,27 @@ int sm_count() {
   return n;
 }
 
-// Persistent launch: as many CTAs as can be resident (shared memory and TMEM
-// columns both limit it), never more than there are tiles.
+// Persistent launch: as many CTAs as the runtime keeps resident at once (one per SM
+// for a kernel that allocates TMEM), never more than there are tiles.  A larger grid
+// would run its surplus CTAs as a second wave behind the first.
 template <int MODE, int BN, int STAGES>
 cudaError_t launch_group(GroupParams& gp, int tiles, cudaStream_t st) {
   using S = Smem<BN, STAGES, ModeExtra<MODE>::kBytes>;
-  static bool configured = false;
-  if (!configured) {
+  static int per_sm = 0;
+  if (per_sm == 0) {
     cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<MODE, BN, STAGES>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tc_gemm_kernel<MODE, BN, STAGES>, kThreads,
+                                                        S::kBytes);
+    if (e != cudaSuccess) {
+      per_sm = 0;
+      return e;
+    }
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;   // does not fit on an SM
   }
   gp.total_tiles = tiles;
   if (tiles <= 0) return cudaSuccess;
-  int per_sm = (227 * 1024) / S::kBytes;
-  const int by_tmem = 512 / (2 * BN);
-  per_sm = per_sm < by_tmem ? per_sm : by_tmem;
-  per_sm = per_sm < 1 ? 1 : per_sm;
   int grid = sm_count() * per_sm;
   grid = grid < tiles ? grid : tiles;
   return launch_pdl(tc_gemm_kernel<MODE, BN, STAGES>, dim3(grid), dim3(kThreads), S::kBytes, st, gp);
