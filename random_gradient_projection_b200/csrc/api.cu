@@ -315,7 +315,7 @@ int grape_create(const grape_layer* layers, int32_t n_layers, int32_t r, double 
   const bool tc = resolved == GRAPE_PATH_TC;
   const size_t ap_el = tc ? 2 : 4;
   Arena ar;
-  struct Offs { size_t P32, Pt16, P16, AP, S, m, v, dR; };
+  struct Offs { size_t P32, P16, AP, S, m, v, dR; };
   std::vector<Offs> offs(n_layers);
   int part = 0;
   ctx->ws.resize(n_layers);
@@ -323,7 +323,6 @@ int grape_create(const grape_layer* layers, int32_t n_layers, int32_t r, double 
     const size_t di = layers[l].d_in, dout = layers[l].d_out;
     Offs& o = offs[l];
     o.P32 = tc ? SIZE_MAX : ar.take(di * r * 4);
-    o.Pt16 = tc ? ar.take(di * r * 2) : SIZE_MAX;
     o.P16 = tc ? ar.take(di * r * 2) : SIZE_MAX;
     o.AP = ar.take(static_cast<size_t>(B) * T * r * ap_el);
     o.S = ar.take(r * dout * 4);
@@ -364,7 +363,6 @@ int grape_create(const grape_layer* layers, int32_t n_layers, int32_t r, double 
     grape::LayerWs& w = ctx->ws[l];
     const Offs& o = offs[l];
     w.P32 = reinterpret_cast<float*>(at(o.P32));
-    w.Pt16 = reinterpret_cast<__nv_bfloat16*>(at(o.Pt16));
     w.P16 = reinterpret_cast<__nv_bfloat16*>(at(o.P16));
     w.AP = at(o.AP);
     w.S = reinterpret_cast<float*>(at(o.S));

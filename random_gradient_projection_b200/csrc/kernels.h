@@ -13,7 +13,6 @@ namespace grape {
 struct LayerWs {
   int d_in, d_out;
   float* P32;              // d_in x r fp32        (CUDA-core path)
-  __nv_bfloat16* Pt16;     // r x d_in bf16 = P^T  (tensor-core path: projection operand)
   __nv_bfloat16* P16;      // d_in x r bf16 = P    (tensor-core path: back-projection operand)
   void* AP;                // B*T x r: fp32 (CUDA-core) / bf16 (tensor-core)
   float* S;                // r x d_out  sum_i c_i R_i

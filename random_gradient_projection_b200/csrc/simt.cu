@@ -82,8 +82,7 @@ __device__ __forceinline__ float block_sum(float x) {
 
 // ---- a1: P_l = z(seed, l, s, stream 0, e) / sqrt(r), e = k*r + j -------------
 // One thread per block of four elements; blockIdx.y = layer.
-__global__ void __launch_bounds__(256) generate_P_kernel(StepShape sh, LayerTable tab, uint32_t step,
-                                                         int want32, int want16) {
+__global__ void __launch_bounds__(256) generate_P_kernel(StepShape sh, LayerTable tab, uint32_t step) {
   const int l = blockIdx.y;
   const LayerWs& w = tab.ws[l];
   const int64_t n = static_cast<int64_t>(w.d_in) * sh.r;
@@ -98,14 +97,7 @@ __global__ void __launch_bounds__(256) generate_P_kernel(StepShape sh, LayerTabl
     for (int u = 0; u < 4; ++u) {
       const int64_t e = 4 * q + u;
       if (e >= n) break;
-      const float p = zz[u] * scale;
-      const int k = static_cast<int>(e / sh.r), j = static_cast<int>(e % sh.r);
-      if (want32) w.P32[e] = p;
-      if (want16) {
-        const __nv_bfloat16 b = __float2bfloat16_rn(p);
-        w.P16[e] = b;
-        w.Pt16[static_cast<int64_t>(j) * w.d_in + k] = b;
-      }
+      w.P32[e] = zz[u] * scale;
     }
   }
 }
@@ -209,42 +201,87 @@ __global__ void __launch_bounds__(kThreads) aggregate_kernel(StepShape sh, Layer
 }
 
 // ---- a6: g = (S + sigma C xi) / batch; Adam in the projected space ----------------
-// xi_l[e] = z(seed, l, s, stream 1, e), e = j*d_out + n.  One thread per block of 4.
+// xi_l[e] = z(seed, l, s, stream 1, e), e = j*d_out + n.  One thread per block of four
+// consecutive elements (float4 accesses when r*d_out is a multiple of 4; every buffer
+// of the library's arena starts on a 256-byte boundary).
+//
+// After a programmatic (PDL) launch the aggregation that writes S may still be
+// running, so S is read only after griddepcontrol.wait.  m and v were last written by
+// this kernel in the previous step, and every step begins with an ordinary launch
+// (the generation of P) that waits for all earlier work, so they -- and the noise,
+// which depends on nothing -- are read and drawn before the wait.
 __global__ void __launch_bounds__(256) noise_adam_kernel(StepShape sh, LayerTable tab,
                                                          UpdateScalars u, int dR_bf16) {
-  // When launched as a programmatic dependent (tensor-core path): let the back-projection
-  // be scheduled, then wait for S.  Both are no-ops after an ordinary launch.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int l = blockIdx.y;
   const LayerWs& w = tab.ws[l];
   const int64_t n = static_cast<int64_t>(sh.r) * w.d_out;
-  const int64_t nq = (n + 3) / 4;
+  const int64_t q = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (4 * q >= n) return;
+  const bool vec = (n % 4) == 0;
   const float noise_scale = sh.sigma_C;
+  float xi[4] = {0.f, 0.f, 0.f, 0.f};
+  if (noise_scale != 0.0f) {
+    const float4 z = gaussian4(sh.seed, static_cast<uint32_t>(l), u.step, kStreamNoise,
+                               static_cast<uint32_t>(q));
+    xi[0] = z.x; xi[1] = z.y; xi[2] = z.z; xi[3] = z.w;
+  }
+  float m[4] = {0.f, 0.f, 0.f, 0.f}, v[4] = {0.f, 0.f, 0.f, 0.f}, S[4] = {0.f, 0.f, 0.f, 0.f};
+  const int cnt = static_cast<int>((n - 4 * q) < 4 ? (n - 4 * q) : 4);
+  if (vec) {
+    const float4 m4 = reinterpret_cast<const float4*>(w.m)[q];
+    const float4 v4 = reinterpret_cast<const float4*>(w.v)[q];
+    m[0] = m4.x; m[1] = m4.y; m[2] = m4.z; m[3] = m4.w;
+    v[0] = v4.x; v[1] = v4.y; v[2] = v4.z; v[3] = v4.w;
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k < cnt) {
+        m[k] = w.m[4 * q + k];
+        v[k] = w.v[4 * q + k];
+      }
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (vec) {
+    const float4 s4 = reinterpret_cast<const float4*>(w.S)[q];
+    S[0] = s4.x; S[1] = s4.y; S[2] = s4.z; S[3] = s4.w;
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k < cnt) S[k] = w.S[4 * q + k];
+  }
   const float b1 = sh.beta1, b2 = sh.beta2;
   const float ob1 = sh.one_minus_beta1, ob2 = sh.one_minus_beta2;
-  for (int64_t q = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; q < nq;
-       q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    float xi[4] = {0.f, 0.f, 0.f, 0.f};
-    if (noise_scale != 0.0f) {
-      const float4 z = gaussian4(sh.seed, static_cast<uint32_t>(l), u.step, kStreamNoise,
-                                 static_cast<uint32_t>(q));
-      xi[0] = z.x; xi[1] = z.y; xi[2] = z.z; xi[3] = z.w;
+  float d[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float g = fmaf(noise_scale, xi[k], S[k]) * u.inv_batch;
+    m[k] = fmaf(b1, m[k], ob1 * g);
+    v[k] = fmaf(b2, v[k], ob2 * g * g);
+    d[k] = (m[k] * u.inv_bc1) / (sqrtf(v[k] * u.inv_bc2) + sh.eps);
+  }
+  if (vec) {
+    reinterpret_cast<float4*>(w.m)[q] = make_float4(m[0], m[1], m[2], m[3]);
+    reinterpret_cast<float4*>(w.v)[q] = make_float4(v[0], v[1], v[2], v[3]);
+    if (dR_bf16) {
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(d[0], d[1]);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(d[2], d[3]);
+      reinterpret_cast<uint2*>(w.dR)[q] =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+    } else {
+      reinterpret_cast<float4*>(w.dR)[q] = make_float4(d[0], d[1], d[2], d[3]);
     }
+  } else {
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
+      if (k >= cnt) continue;
       const int64_t e = 4 * q + k;
-      if (e >= n) break;
-      const float g = fmaf(noise_scale, xi[k], w.S[e]) * u.inv_batch;
-      const float m = fmaf(b1, w.m[e], ob1 * g);
-      const float v = fmaf(b2, w.v[e], ob2 * g * g);
-      w.m[e] = m;
-      w.v[e] = v;
-      const float d = (m * u.inv_bc1) / (sqrtf(v * u.inv_bc2) + sh.eps);
+      w.m[e] = m[k];
+      w.v[e] = v[k];
       if (dR_bf16)
-        static_cast<__nv_bfloat16*>(w.dR)[e] = __float2bfloat16_rn(d);
+        static_cast<__nv_bfloat16*>(w.dR)[e] = __float2bfloat16_rn(d[k]);
       else
-        static_cast<float*>(w.dR)[e] = d;
+        static_cast<float*>(w.dR)[e] = d[k];
     }
   }
 }
@@ -333,9 +370,9 @@ cudaError_t simt_generate_P(const StepShape& sh, const LayerWs* ws, uint32_t ste
     const int64_t q = (static_cast<int64_t>(ws[l].d_in) * sh.r + 3) / 4;
     most = q > most ? q : most;
   }
-  const int want32 = ws[0].P32 != nullptr, want16 = ws[0].P16 != nullptr;
+  if (ws[0].P32 == nullptr) return cudaErrorInvalidValue;   // fp32 P lives on the CUDA-core path only
   dim3 grid(cdiv(most, 256) < 1184 ? cdiv(most, 256) : 1184, sh.L);
-  generate_P_kernel<<<grid, 256, 0, st>>>(sh, t, step, want32, want16);
+  generate_P_kernel<<<grid, 256, 0, st>>>(sh, t, step);
   return cudaGetLastError();
 }
 
@@ -373,7 +410,7 @@ cudaError_t noise_adam(const StepShape& sh, const LayerWs* ws, const UpdateScala
                        bool pdl, cudaStream_t st) {
   const LayerTable t = make_table(sh, ws, nullptr);
   const int64_t q = (static_cast<int64_t>(sh.r) * max_d_out(sh, ws) + 3) / 4;
-  dim3 grid(cdiv(q, 256) < 592 ? cdiv(q, 256) : 592, sh.L);
+  dim3 grid(cdiv(q, 256), sh.L);   // one thread per four elements (no grid-stride loop)
   if (!pdl) {
     noise_adam_kernel<<<grid, 256, 0, st>>>(sh, t, u, dR_bf16 ? 1 : 0);
     return cudaGetLastError();

@@ -14,17 +14,17 @@
 // with Gradient Random Projection": per-sample projection, norms for clipping,
 // aggregation, and the projected update of the parameters).
 //
-// CTA layout (352 threads, one CTA per SM: the runtime places a single CTA of a kernel
-// that allocates TMEM on each SM): warps 0 and 10 issue the TMA loads of the A and the
-// B operand into a ring of shared-memory stages (128-byte swizzle) -- one issuing
-// thread per operand, because one thread's TMA stream tops out near 6 TB/s of SM
-// ingress over the whole GPU while two reach about 11 TB/s; warp 1 owns the TMEM
-// allocation and one of its threads issues tcgen05.mma (M = 128, N = BN, K = 16 per
-// instruction) into one of two 128 x BN fp32 TMEM accumulators; warps 2-9 read the
-// accumulator back with tcgen05.ld (each warp its 32 TMEM lanes) and run the
-// epilogue.  Stage reuse is tracked with mbarriers (TMA completion -> fullA / fullB,
-// tcgen05.commit -> empty); every wait is bounded and reports a timeout through an
-// error word.
+// CTA layout (416 threads, one CTA per SM: the runtime places a single CTA of a kernel
+// that allocates TMEM on each SM): four producer warps (0, 10, 11, 12) issue the TMA
+// loads into a ring of shared-memory stages (128-byte swizzle), producer p filling the
+// stages of k-block iterations it = p (mod 4) -- the TMA stream of one issuing thread
+// moves about 25 GB/s of L2-resident data into an SM and four such streams about
+// 86 GB/s, so the issue is spread; warp 1 owns the TMEM allocation and one of its
+// threads issues tcgen05.mma (M = 128, N = BN, K = 16 per instruction) into one of
+// two 128 x BN fp32 TMEM accumulators; warps 2-9 read the accumulator back with
+// tcgen05.ld (each warp its 32 TMEM lanes) and run the epilogue.  Stage reuse is
+// tracked with mbarriers (TMA completion -> full, tcgen05.commit -> empty); every
+// wait is bounded and reports a timeout through an error word.
 //
 // Operands: A, P (as the A operand of BACKPROJ) are K-major tiles of 128 rows x
 // 64 bf16; AP^T (NORM / AGGREGATE) and every B operand (P, Gout, dR) are
@@ -55,8 +55,20 @@ namespace {
 constexpr int kBM = 128;           // UMMA M (one CTA, TMEM lanes)
 constexpr int kBK = 64;            // K per stage: one 128-byte swizzle row of bf16
 constexpr int kEpiWarps = 8;       // two per TMEM lane quarter, each on half the columns
-constexpr int kProdBWarp = 2 + kEpiWarps;        // warp 0: TMA A, 1: MMA, 2..9: epilogue, 10: TMA B
-constexpr int kThreads = 32 * (kProdBWarp + 1);  // 352
+constexpr int kProducers = 4;                    // TMA-issuing warps: 0 and 10, 11, 12
+// A ring of STAGES stages is filled by min(kProducers, STAGES) of them.  An mbarrier
+// parity wait tells only adjacent phases apart: a producer waiting for phase u-1 of
+// empty[s] must know that phase u-2 is complete, and its own previous wait (kP
+// iterations earlier) guarantees that only when kP <= STAGES.
+template <int STAGES>
+struct RingProducers {
+  static constexpr int kCount = STAGES < kProducers ? STAGES : kProducers;
+};
+constexpr int kThreads = 32 * (2 + kEpiWarps + kProducers - 1);   // 416
+// producer index of a warp (0 .. kProducers-1), or -1 for the MMA and epilogue warps
+__device__ __forceinline__ int producer_of(int warp) {
+  return warp == 0 ? 0 : (warp >= 2 + kEpiWarps ? warp - (2 + kEpiWarps) + 1 : -1);
+}
 constexpr int kMaxGroup = 16;      // layers per launch
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr uint64_t kDrainLimitNs = 1000000000ull;   // after an abort: wait for loads in flight
@@ -163,9 +175,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* fullA = reinterpret_cast<uint64_t*>(smem + S::kBarOff);   // A operand landed
-  uint64_t* fullB = fullA + STAGES;                                     // B operand landed
-  uint64_t* empty = fullB + STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
+  uint64_t* empty = full + STAGES;
   uint64_t* accfull = empty + STAGES;       // [2]
   uint64_t* accempty = accfull + 2;         // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + 2);
@@ -173,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   volatile int* abort_flag = reinterpret_cast<volatile int*>(red + 2 * kEpiWarps);
   uint64_t* wfull = reinterpret_cast<uint64_t*>(smem + S::kBarOff + 448);   // BACKPROJ [2]
   uint64_t* wfree = wfull + 2;                                              // BACKPROJ [2]
-  static_assert(3 * STAGES * 8 + 4 * 8 + 8 + 2 * kEpiWarps * 4 + 4 <= 448, "barrier area");
+  static_assert(2 * STAGES * 8 + 4 * 8 + 8 + 2 * kEpiWarps * 4 + 4 <= 448, "barrier area");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto wait = [&](uint64_t* bar, uint32_t parity) {
@@ -184,8 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   if (warp == 0 && lane == 0) {
     *abort_flag = 0;
     for (int s = 0; s < STAGES; ++s) {
-      ptx::mbar_init(&fullA[s], 1);
-      ptx::mbar_init(&fullB[s], 1);
+      ptx::mbar_init(&full[s], 1);
       ptx::mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -210,10 +220,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0 || warp == kProdBWarp) {
-    // ---------------- TMA producers: warp 0 the A operand, warp 10 the B operand ----------------
-    if (lane == 0) {
-      const bool isA = (warp == 0);
+  if (producer_of(warp) >= 0) {
+    // ---------------- TMA producers ----------------
+    constexpr int kNP = RingProducers<STAGES>::kCount;
+    static_assert(kNP >= 1 && kNP <= STAGES, "parity waits need at most STAGES producers");
+    if (lane == 0 && producer_of(warp) < kNP) {
+      const int pi = producer_of(warp);
       // A and Gout stream once per use; P, AP and dR are re-read by other tiles or
       // by the next phase, so they are kept in L2 preferentially.
       const uint64_t polA = (MODE == PROJECT || MODE == AGGREGATE || MODE == BACKPROJ)
@@ -225,15 +237,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         const CUtensorMap* mapA = &p.mapA[c.g];
         const int kk = kb * kBK;
         if (MODE == PROJECT || MODE == BACKPROJ) {
-          ptx::tma_load_2d_hint(sa, mapA, &fullA[s], kk, c.m_t * kBM, MODE == BACKPROJ ? polB : polA);
+          ptx::tma_load_2d_hint(sa, mapA, &full[s], kk, c.m_t * kBM, MODE == BACKPROJ ? polB : polA);
         } else if (MODE == NORM) {
 #pragma unroll
           for (int q = 0; q < kBM / 64; ++q)
-            ptx::tma_load_3d_hint(sa + q * 8192, mapA, &fullA[s], c.m_t * kBM + 64 * q, kk, c.s_t, polA);
+            ptx::tma_load_3d_hint(sa + q * 8192, mapA, &full[s], c.m_t * kBM + 64 * q, kk, c.s_t, polA);
         } else {
 #pragma unroll
           for (int q = 0; q < kBM / 64; ++q)
-            ptx::tma_load_2d_hint(sa + q * 8192, mapA, &fullA[s], c.m_t * kBM + 64 * q, kk, polA);
+            ptx::tma_load_2d_hint(sa + q * 8192, mapA, &full[s], c.m_t * kBM + 64 * q, kk, polA);
         }
       };
       auto load_b = [&](const TileCoord& c, int kb, int s) {
@@ -243,9 +255,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
 #pragma unroll
         for (int q = 0; q < BN / 64; ++q) {
           if (T::kB3d)
-            ptx::tma_load_3d_hint(sb + q * 8192, mapB, &fullB[s], c.n_t * BN + 64 * q, kk, c.s_t, polB);
+            ptx::tma_load_3d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kk, c.s_t, polB);
           else
-            ptx::tma_load_2d_hint(sb + q * 8192, mapB, &fullB[s], c.n_t * BN + 64 * q, kk, polB);
+            ptx::tma_load_2d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kk, polB);
         }
       };
       auto load_w = [&](const TileCoord& c, int wb) {
@@ -258,24 +270,27 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       };
 
       // The operand that predates the step -- A (PROJECT) or Gout (NORM, AGGREGATE) --
-      // streams without waiting for the previous kernel of the step; P, AP and dR are
-      // written earlier in this step and load after the wait.  W of the first tile
-      // (BACKPROJ) also loads before it.
-      const bool predates = isA ? (MODE == PROJECT) : (MODE == NORM || MODE == AGGREGATE);
-      uint64_t* full = isA ? fullA : fullB;
-      const uint32_t bytes = isA ? S::kABytes : S::kBBytes;
+      // of a producer's first stage loads before waiting for the previous kernel of the
+      // step; P, AP and dR are written earlier in this step and load after the wait.
+      // Producer 0 also loads W of the first tile (BACKPROJ) before it, and every W tile.
+      bool waited = false;
+      auto ensure_wait = [&]() {
+        if (!waited) {
+          ptx::griddep_wait();
+          waited = true;
+        }
+      };
       uint32_t wissued = 0;
-      if (MODE == BACKPROJ && !isA && static_cast<int>(blockIdx.x) < p.total_tiles) {
+      if (MODE == BACKPROJ && pi == 0 && static_cast<int>(blockIdx.x) < p.total_tiles) {
         load_w(decode_tile(p, blockIdx.x, MODE), 0);
         wissued = 1;
       }
-      if (!predates) ptx::griddep_wait();
 
-      uint32_t it = 0, tcp = 0;
+      uint32_t it = 0, tcp = 0, issued_end = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++tcp) {
         const TileCoord c = decode_tile(p, tile, MODE);
-        if (MODE == BACKPROJ && !isA && tcp > 0) {
+        if (MODE == BACKPROJ && pi == 0 && tcp > 0) {
           // this tile's W into buffer tcp & 1, once the store of the tile before last
           // has finished reading it
           const int wb = tcp & 1;
@@ -288,6 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
           ++wissued;
         }
         for (int kb = c.kb0; kb < c.kb1; ++kb, ++it) {
+          if (static_cast<int>(it % kNP) != pi) continue;
           const int s = it % STAGES;
           const uint32_t use = it / STAGES;
           if (use > 0 && !wait(&empty[s], (use - 1) & 1)) {
@@ -295,18 +311,29 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             ok = false;
             break;
           }
-          ptx::mbar_arrive_expect_tx(&full[s], bytes);
-          if (isA)
+          ptx::mbar_arrive_expect_tx(&full[s], S::kStage);
+          if (MODE == PROJECT) {
             load_a(c, kb, s);
-          else
+            ensure_wait();
             load_b(c, kb, s);
+          } else if (MODE == NORM || MODE == AGGREGATE) {
+            load_b(c, kb, s);
+            ensure_wait();
+            load_a(c, kb, s);
+          } else {
+            ensure_wait();
+            load_a(c, kb, s);
+            load_b(c, kb, s);
+          }
+          issued_end = it + 1;
         }
       }
       if (*abort_flag) {
         // leave none of this thread's TMA loads in flight into this CTA's shared memory
-        for (uint32_t k = it > STAGES ? it - STAGES : 0; k < it; ++k)
-          ptx::mbar_wait(&full[k % STAGES], (k / STAGES) & 1, kDrainLimitNs);
-        if (MODE == BACKPROJ && !isA)
+        for (uint32_t k = issued_end > STAGES ? issued_end - STAGES : 0; k < issued_end; ++k)
+          if (static_cast<int>(k % kNP) == pi)
+            ptx::mbar_wait(&full[k % STAGES], (k / STAGES) & 1, kDrainLimitNs);
+        if (MODE == BACKPROJ && pi == 0)
           for (uint32_t k = wissued > 2 ? wissued - 2 : 0; k < wissued; ++k)
             ptx::mbar_wait(&wfull[k & 1], (k >> 1) & 1, kDrainLimitNs);
       }
@@ -329,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         for (int kb = c.kb0; kb < c.kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
-          if (!wait(&fullA[s], ph) || !wait(&fullB[s], ph)) {
+          if (!wait(&full[s], ph)) {
             atomicOr(p.err, kErrTimeoutMma);
             ok = false;
             break;
@@ -510,9 +537,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* fullA = reinterpret_cast<uint64_t*>(smem + S::kBarOff);   // AP stage landed
-  uint64_t* fullB = fullA + STAGES;                                     // Gout stage landed
-  uint64_t* empty = fullB + STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
+  uint64_t* empty = full + STAGES;
   uint64_t* accfull = empty + STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
@@ -534,8 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
   if (warp == 0 && lane == 0) {
     *abort_flag = 0;
     for (int s = 0; s < STAGES; ++s) {
-      ptx::mbar_init(&fullA[s], 1);
-      ptx::mbar_init(&fullB[s], 1);
+      ptx::mbar_init(&full[s], 1);
       ptx::mbar_init(&empty[s], 1);
     }
     ptx::mbar_init(accfull, 1);
@@ -552,41 +577,52 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0 || warp == kProdBWarp) {
-    // warp 0 loads AP (rescaled by the clip kernel, so after the wait for it); warp 10
-    // loads Gout, which predates the step, without that wait.
-    if (lane == 0) {
-      const bool isA = (warp == 0);
+  if (producer_of(warp) >= 0) {
+    // Producer p fills the stages of iterations it = p (mod kNP).  Gout predates the
+    // step and loads before the wait for the clip kernel; AP (rescaled by it) after.
+    constexpr int kNP = RingProducers<STAGES>::kCount;
+    static_assert(kNP >= 1 && kNP <= STAGES, "parity waits need at most STAGES producers");
+    if (lane == 0 && producer_of(warp) < kNP) {
+      const int pi = producer_of(warp);
       const uint64_t pol = ptx::policy_evict_first();   // last use of AP and Gout in the step
-      const CUtensorMap* map = isA ? &p.mapA[c.g] : &p.mapB[c.g];
-      uint64_t* full = isA ? fullA : fullB;
-      const uint32_t bytes = isA ? S::kABytes : S::kBBytes;
-      const int chunks = isA ? kBM / 64 : BN / 64;
-      const int col0 = isA ? c.m_t * kBM : c.n_t * BN;
-      if (isA) ptx::griddep_wait();
-      uint32_t issued = 0;
-      for (int kb = kb0; kb < kb1; ++kb, ++issued) {
-        const int s = issued % STAGES;
-        const uint32_t use = issued / STAGES;
+      const CUtensorMap* mapA = &p.mapA[c.g];
+      const CUtensorMap* mapB = &p.mapB[c.g];
+      bool waited = false;
+      uint32_t issued_end = 0;
+      for (int kb = kb0, it = 0; kb < kb1; ++kb, ++it) {
+        if (it % kNP != pi) continue;
+        const int s = it % STAGES;
+        const uint32_t use = it / STAGES;
         if (use > 0 && !wait(&empty[s], (use - 1) & 1)) {
           atomicOr(p.err, kErrTimeoutProducer);
           break;
         }
-        uint8_t* dst = smem + s * S::kStage + (isA ? 0 : S::kABytes);
-        ptx::mbar_arrive_expect_tx(&full[s], bytes);
-        for (int q = 0; q < chunks; ++q)
-          ptx::tma_load_2d_hint(dst + q * 8192, map, &full[s], col0 + 64 * q, kb * kBK, pol);
+        uint8_t* sa = smem + s * S::kStage;
+        uint8_t* sb = sa + S::kABytes;
+        ptx::mbar_arrive_expect_tx(&full[s], S::kStage);
+#pragma unroll
+        for (int q = 0; q < BN / 64; ++q)
+          ptx::tma_load_2d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kb * kBK, pol);
+        if (!waited) {
+          ptx::griddep_wait();
+          waited = true;
+        }
+#pragma unroll
+        for (int q = 0; q < kBM / 64; ++q)
+          ptx::tma_load_2d_hint(sa + q * 8192, mapA, &full[s], c.m_t * kBM + 64 * q, kb * kBK, pol);
+        issued_end = it + 1;
       }
       if (*abort_flag)
-        for (uint32_t k = issued > STAGES ? issued - STAGES : 0; k < issued; ++k)
-          ptx::mbar_wait(&full[k % STAGES], (k / STAGES) & 1, kDrainLimitNs);
+        for (uint32_t k2 = issued_end > STAGES ? issued_end - STAGES : 0; k2 < issued_end; ++k2)
+          if (static_cast<int>(k2 % kNP) == pi)
+            ptx::mbar_wait(&full[k2 % STAGES], (k2 / STAGES) & 1, kDrainLimitNs);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       for (int kb = kb0, it = 0; kb < kb1; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
-        if (!wait(&fullA[s], ph) || !wait(&fullB[s], ph)) {
+        if (!wait(&full[s], ph)) {
           atomicOr(p.err, kErrTimeoutMma);
           break;
         }
@@ -614,12 +650,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
     const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * (BN / 2);
     const bool have = got && kb1 > kb0;
 #pragma unroll 1
-    for (int cc = 0; cc < BN / 2; cc += 64) {
-      float v[64];
-      ptx::tmem_ld64(tbase + cc, v);
+    for (int cc = 0; cc < BN / 2; cc += 32) {
+      float v[32];
+      ptx::tmem_ld32(tbase + cc, v);
       float4* dst = reinterpret_cast<float4*>(stage + row * kLd + h * (BN / 2) + cc);
 #pragma unroll
-      for (int u = 0; u < 16; ++u)
+      for (int u = 0; u < 8; ++u)
         dst[u] = have ? make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3])
                       : make_float4(0.f, 0.f, 0.f, 0.f);
     }
@@ -721,15 +757,26 @@ __global__ void __launch_bounds__(256) clip_scale_kernel(ApTable t, int r, int T
   if (c == 1.0f) return;
   uint4* rows = reinterpret_cast<uint4*>(t.AP[l] + static_cast<size_t>(i) * T * r);
   const size_t n8 = static_cast<size_t>(T) * r / 8;   // 8 bf16 per 16-byte vector
-  for (size_t k = threadIdx.x; k < n8; k += 256) {
-    uint4 x = rows[k];
-    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&x);
+  constexpr int kBatch = 8;                            // loads in flight per thread
+  for (size_t k0 = threadIdx.x; k0 < n8; k0 += 256 * kBatch) {
+    uint4 x[kBatch];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float2 f = __bfloat1622float2(h[u]);
-      h[u] = __floats2bfloat162_rn(f.x * c, f.y * c);
+    for (int u = 0; u < kBatch; ++u) {
+      const size_t k = k0 + static_cast<size_t>(u) * 256;
+      if (k < n8) x[u] = rows[k];
     }
-    rows[k] = x;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const size_t k = k0 + static_cast<size_t>(u) * 256;
+      if (k >= n8) continue;
+      __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&x[u]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h[e]);
+        h[e] = __floats2bfloat162_rn(f.x * c, f.y * c);
+      }
+      rows[k] = x[u];
+    }
   }
 }
 
