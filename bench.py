@@ -38,7 +38,17 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-INPUT_SETS = 4
+INPUT_SETS = 4          # distinct per-step input sets (2 when one set exceeds 1 GB)
+L2_BYTES = 126 * 1000 * 1000
+
+
+def layer_summary(w) -> str:
+    """'4x1024x1024' for a uniform stack, else the count and the distinct shapes."""
+    shapes = sorted(set(w.layers), key=w.layers.index)
+    if len(shapes) == 1:
+        return f"{w.n_layers}x{shapes[0][0]}x{shapes[0][1]}"
+    return f"{w.n_layers} layers of " + ", ".join(f"{a}x{b}" for a, b in shapes)
+
 
 
 def parse(argv=None):
@@ -247,7 +257,7 @@ def run_reference(args, rank: int, world: int):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "layers": f"{w.n_layers}x{w.layers[0][0]}x{w.layers[0][1]}",
+        "config": {"workload": w.name, "layers": layer_summary(w),
                    "r": w.r, "B": w.B, "T": w.T, "tokens_per_s": value * w.T},
         "cpu_baseline": {"value": value, "unit": "samples/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
@@ -292,8 +302,9 @@ def main(argv=None):
 
     # distinct per-step input sets; ranks draw different samples (input seed only)
     win = w.replace(seed=w.seed + 7919 * rank)
+    n_sets = INPUT_SETS if w.input_bytes() < (1 << 30) else 2
     sets = []
-    for k in range(INPUT_SETS):
+    for k in range(n_sets):
         x = WL.make_step_inputs(win, k, threads=16)
         conv = (lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)) \
             if w.dtype == "bf16" else torch.from_numpy
@@ -301,7 +312,7 @@ def main(argv=None):
     set_bytes = w.input_bytes()
 
     def one(s):
-        A, G = sets[s % INPUT_SETS]
+        A, G = sets[s % n_sets]
         if world > 1:
             dp_step(g, A, G, Wd, s)
         else:
@@ -436,11 +447,14 @@ def main(argv=None):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic",
-            "config": {"workload": w.name, "layers": f"{w.n_layers}x{w.layers[0][0]}x{w.layers[0][1]}",
+            "config": {"workload": w.name, "layers": layer_summary(w),
                        "r": w.r, "B_per_gpu": w.B, "global_batch": w.B * world, "T": w.T,
                        "path": path_name, "parallelism": f"dp{world}",
-                       "l2": f"inputs rotate over {INPUT_SETS} distinct sets of "
-                             f"{set_bytes / 1e6:.0f} MB each (> 126 MB L2)",
+                       "l2": (f"inputs rotate over {n_sets} distinct sets of "
+                              f"{set_bytes / 1e6:.0f} MB each (> 126 MB L2)")
+                             if set_bytes > L2_BYTES else
+                             (f"inputs ({n_sets} sets of {set_bytes / 1e6:.3f} MB) fit in L2; "
+                              "cold_l2 times steps after a 256 MB write"),
                        "tokens_per_s": samples_per_s * w.T,
                        "cold_l2": {"ms_per_step": cold_ms / n_cold,
                                    "value": world * w.B * n_cold / (cold_ms / 1e3),
