@@ -186,11 +186,23 @@ class Hyper:
     beta1: float = 0.9
     beta2: float = 0.999
     eps: float = 1e-8
+    refresh: int = 1     # projection-refresh period K: P of step s is drawn with key floor(s / K)
 
     @classmethod
     def of(cls, w) -> "Hyper":
         return cls(r=w.r, C=w.C, sigma=w.sigma, seed=w.seed, lr=w.lr, beta1=w.beta1,
-                   beta2=w.beta2, eps=w.eps)
+                   beta2=w.beta2, eps=w.eps, refresh=getattr(w, "refresh", 1))
+
+    def projection_key(self, step: int) -> int:
+        """Step field of P's Philox counter at step s.
+
+        Reading: "regenerated on the fly from a seed" (design choice 1 of
+        "Metodología") leaves the refresh schedule open.  K = 1 re-draws P every
+        step; K > 1 keeps one random subspace for K consecutive steps (as GaLore
+        keeps its SVD subspace between refreshes), with m and v carried across
+        refreshes unchanged.  The noise is drawn per step whatever K is.
+        """
+        return step // self.refresh
 
 
 @dataclasses.dataclass
@@ -216,7 +228,7 @@ ProjectionFn = Callable[[int, int, int, int], np.ndarray]   # (layer, step, d_in
 
 
 def default_projection(h: Hyper) -> ProjectionFn:
-    return lambda layer, step, d_in, r: projection_matrix(h.seed, layer, step, d_in, r)
+    return lambda layer, step, d_in, r: projection_matrix(h.seed, layer, h.projection_key(step), d_in, r)
 
 
 def projected_per_sample(A: Sequence[np.ndarray], Gout: Sequence[np.ndarray],
@@ -281,10 +293,47 @@ def sample_norms(A: Sequence[np.ndarray], Gout: Sequence[np.ndarray], step_index
     n = A[0].shape[0]
     tot = np.zeros(n)
     for l in range(L):
-        P = projection_matrix(h.seed, l, step_index, d_in[l], h.r)
+        P = projection_matrix(h.seed, l, h.projection_key(step_index), d_in[l], h.r)
         for j in range(n):
             tot[j] += float(np.sum(project(P, per_sample_gradient(A[l][j], Gout[l][j])) ** 2))
     return np.sqrt(tot)
+
+
+# --------------------------------------------------------------------------
+# Hutchinson estimate of a per-sample gradient norm (DP-SGD-RC)
+#
+# Source: "DP-SGD-RC" technical summary on the same site (gist.science,
+# 2605.24879), sections "Metodología: DP-SGD-RC" (the trace identity and the
+# Hutchinson estimator) and "Flujo Algorítmico" step 3 (the norm-estimation
+# routine, applied per sample).  ||A^T G||_F^2 = tr(O) with O = (A^T G)(A^T G)^T;
+# Hutchinson's estimator sums p_j^T O p_j over the k columns p_j of a Gaussian
+# matrix.  Reading: the sketch acts on the activation width (d_in), and its
+# entries are N(0, 1/k), the same scale as DP-GRAPE's P, so the sum is unbiased
+# with no further factor.
+# --------------------------------------------------------------------------
+
+def hutchinson_sqnorm(A_i: np.ndarray, Gout_i: np.ndarray, P: np.ndarray) -> float:
+    """sum_j P[:, j]^T O P[:, j] with O = G G^T, G = A_i^T Gout_i (d_in x d_out).
+
+    O is formed explicitly (d_in x d_in, fp64): the definition written out, not
+    the factored ||(A_i P)^T Gout_i||^2 that the kernels compute."""
+    G = per_sample_gradient(A_i, Gout_i)
+    O = G @ G.T
+    return float(sum(P[:, j] @ O @ P[:, j] for j in range(P.shape[1])))
+
+
+def hutchinson_sample_sqnorms(A: Sequence[np.ndarray], Gout: Sequence[np.ndarray], step_index: int,
+                              h: Hyper, d_in: Sequence[int]) -> np.ndarray:
+    """Per-sample estimate of sum_l ||A_{i,l}^T Gout_{i,l}||_F^2 with k = h.r sketch
+    columns per layer, P_l drawn as DP-GRAPE draws it (key floor(s / K))."""
+    L = len(A)
+    n = A[0].shape[0]
+    tot = np.zeros(n)
+    for l in range(L):
+        P = projection_matrix(h.seed, l, h.projection_key(step_index), d_in[l], h.r)
+        for j in range(n):
+            tot[j] += hutchinson_sqnorm(A[l][j], Gout[l][j], P)
+    return tot
 
 
 def run(workload, steps: int, samples: Optional[Sequence[int]] = None,

@@ -326,10 +326,94 @@ def pin_projection_before_privatization(O):
     assert not np.allclose(naive[0], out["S"][0], rtol=1e-3)
 
 
+# --------------------------------------------------------------------------
+# projection-refresh period K
+# --------------------------------------------------------------------------
+
+def _rank(M, tol=1e-9):
+    sv = np.linalg.svd(M, compute_uv=False)
+    return int(np.sum(sv > tol * sv[0]))
+
+
+def pin_refresh_fixed_subspace(O):
+    """K >= number of steps keeps one P for the whole run, so W_T - W_0 = -lr P sum_s dR_s
+    has rank <= r (the GaLore-style fixed subspace); with K = 1 a fresh P every step lets
+    the rank grow past r.  A property of the update, not of the key arithmetic."""
+    layers = ((12, 10),)
+    B, T, steps, r = 3, 4, 4, 2
+    h_fixed = O.Hyper(r=r, C=1e9, sigma=0.0, seed=5, lr=1e-2, refresh=steps)
+    h_fresh = O.Hyper(r=r, C=1e9, sigma=0.0, seed=5, lr=1e-2, refresh=1)
+    _, _, W0 = _tiny_problem(0, B, T, layers)
+    st_fixed, st_fresh = O.State.init(W0, r), O.State.init(W0, r)
+    for s in range(steps):
+        A, G, _ = _tiny_problem(20 + s, B, T, layers, scale=0.5)
+        O.step(st_fixed, A, G, s, h_fixed)
+        O.step(st_fresh, A, G, s, h_fresh)
+    assert _rank(st_fixed.W[0] - W0[0]) <= r
+    assert _rank(st_fresh.W[0] - W0[0]) > r
+
+
+def pin_refresh_period_two(O):
+    """K = 2: steps 0 and 1 project with the same P, step 2 with another, and the noise
+    still changes every step."""
+    A, G, W0 = _tiny_problem(3)
+    h = O.Hyper(r=2, C=0.5, sigma=1.0, seed=8, refresh=2)
+    st = O.State.init(W0, h.r)
+    P = [O.step(st, A, G, s, h)["P"][0] for s in range(3)]
+    assert np.array_equal(P[0], P[1]) and not np.allclose(P[1], P[2])
+    assert not np.allclose(O.noise_matrix(h.seed, 0, 0, 2, 4), O.noise_matrix(h.seed, 0, 1, 2, 4))
+
+
+# --------------------------------------------------------------------------
+# Hutchinson norm estimate (DP-SGD-RC)
+# --------------------------------------------------------------------------
+
+def pin_hutchinson_identity_sketch(O):
+    """With the identity as the sketch (k = d_in columns e_j) the estimator is the trace
+    itself: exactly ||A^T G||_F^2."""
+    rng = np.random.default_rng(11)
+    A, G = rng.standard_normal((5, 7)), rng.standard_normal((5, 3))
+    exact = float(np.sum((A.T @ G) ** 2))
+    assert math.isclose(O.hutchinson_sqnorm(A, G, np.eye(7)), exact, rel_tol=1e-12)
+
+
+def pin_hutchinson_unbiased(O):
+    """Gaussian sketch with N(0, 1/k) entries: the mean of N independent estimates is within
+    4 standard deviations of ||A^T G||_F^2, the variance of one estimate being
+    2 ||O||_F^2 / k for O = (A^T G)(A^T G)^T."""
+    rng = np.random.default_rng(12)
+    A, G = rng.standard_normal((6, 9)), rng.standard_normal((6, 4))
+    Gm = A.T @ G
+    exact = float(np.sum(Gm ** 2))
+    k, N = 3, 4000
+    est = np.array([O.hutchinson_sqnorm(A, G, rng.standard_normal((9, k)) / math.sqrt(k)) for _ in range(N)])
+    sd = math.sqrt(2.0 * float(np.sum((Gm @ Gm.T) ** 2)) / k / N)
+    assert abs(est.mean() - exact) < 4 * sd, (est.mean(), exact, sd)
+    # and the spread matches the closed form (within 10 %)
+    assert abs(est.std() / math.sqrt(2.0 * float(np.sum((Gm @ Gm.T) ** 2)) / k) - 1) < 0.1
+
+
+def pin_hutchinson_factored(O):
+    """The explicit-O estimator equals ||(A P)^T G||_F^2 computed with loops, the factored
+    form the per-sample norm kernels evaluate."""
+    rng = np.random.default_rng(13)
+    A, G, P = rng.standard_normal((4, 6)), rng.standard_normal((4, 5)), rng.standard_normal((6, 3))
+    f = 0.0
+    for j in range(3):
+        for n in range(5):
+            acc = 0.0
+            for t in range(4):
+                ap = sum(A[t, q] * P[q, j] for q in range(6))
+                acc += ap * G[t, n]
+            f += acc * acc
+    assert math.isclose(O.hutchinson_sqnorm(A, G, P), f, rel_tol=1e-12)
+
+
 ALL_PINS = [
     pin_philox_vs_aten, pin_box_muller_definition, pin_normal_statistics,
     pin_projection_scale, pin_projection_layout, pin_factored_bruteforce,
     pin_identity_projection_is_dp_adam, pin_clipping_bound, pin_sigma_zero,
     pin_adam_first_step, pin_no_privacy_reduction, pin_backprojection_unbiased,
-    pin_projection_before_privatization,
+    pin_projection_before_privatization, pin_refresh_fixed_subspace, pin_refresh_period_two,
+    pin_hutchinson_identity_sketch, pin_hutchinson_unbiased, pin_hutchinson_factored,
 ]

@@ -73,6 +73,14 @@ MUTATIONS = {
                          "state.W[l] = state.W[l] + h.lr * (Ps[l] @ d)"),
     "backproject_no_lr": ("state.W[l] = state.W[l] - h.lr * (Ps[l] @ d)",
                           "state.W[l] = state.W[l] - (Ps[l] @ d)"),
+    # projection-refresh period
+    "refresh_ignored": ("return step // self.refresh", "return step"),
+    "refresh_off_by_one": ("return step // self.refresh", "return (step + 1) // self.refresh"),
+    # Hutchinson estimate
+    "hutch_wrong_gram": ("O = G @ G.T", "O = G @ G.T + np.eye(G.shape[0])"),
+    "hutch_first_column": ("for j in range(P.shape[1])))", "for j in range(1)))"),
+    "hutch_transposed_sketch": ("return float(sum(P[:, j] @ O @ P[:, j] for j in range(P.shape[1])))",
+                                "return float(sum(P[:, j] @ O.T @ O @ P[:, j] for j in range(P.shape[1])))"),
 }
 
 # cheap pins first: a mutation stops at the first pin that fails

@@ -68,6 +68,7 @@ class Workload:
     scale_sigma: float = 1.0              # LogNormal(0, scale_sigma) per-sample scale
     mask_p: float = 1.0                   # Bernoulli keep probability of a loss token
     w_std: float = 0.02
+    refresh: int = 1                      # projection-refresh period K (P keyed on step // K)
 
     @property
     def n_layers(self) -> int:
