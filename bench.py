@@ -34,6 +34,9 @@ import numpy as np  # noqa: E402
 import workloads as WL  # noqa: E402
 
 METRIC = "DP-GRAPE step samples/s (tokens/s) on 1 B200; % of tensor-pipe/HBM roofline"
+# --mode sqnorms: the Hutchinson per-sample gradient-norm estimate alone (grape_sqnorms)
+METRIC_SQNORMS = ("Hutchinson per-sample gradient-norm estimates/s (samples/s) on 1 B200; "
+                  "% of tensor-pipe/HBM roofline")
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_HBM_GBS = 6650.0
@@ -58,6 +61,8 @@ def parse(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="mlp4x1024", choices=sorted(WL.WORKLOADS))
+    ap.add_argument("--mode", default="step", choices=["step", "sqnorms"],
+                    help="step: the whole DP-GRAPE step; sqnorms: per-sample norm estimates only")
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -167,6 +172,15 @@ def phase_work(w, path: str):
     return out
 
 
+def sqnorms_work(w):
+    """Work of the norm estimate alone: FLOPs of AP = A P and of the per-sample
+    (A_i P)^T Gout_i, bytes of A and Gout read once and of the B outputs."""
+    el = 4 if w.dtype == "f32" else 2
+    flops = sum(2 * w.B * w.T * w.r * (di + do) for di, do in w.layers)
+    byts = sum(w.B * w.T * (di + do) * el for di, do in w.layers) + 4 * w.B
+    return flops, byts
+
+
 def step_work(w):
     """The method's own work per step: FLOPs of the factored projection and back-projection,
     bytes of A and Gout read once, W read + written, m and v read + written."""
@@ -182,12 +196,12 @@ def kernel_source_sha(path: str) -> str:
     return hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
 
 
-def traffic_for(kernel: str, workload: str, path: str):
+def traffic_for(kernel: str, workload: str, path: str, mode: str = "step"):
     try:
         t = json.load(open(TRAFFIC_FILE))
     except Exception:  # noqa: BLE001
         return None
-    rec = t.get(f"{path}:{kernel}:{workload}")
+    rec = t.get(f"{path}:{kernel}:{workload}" + ("" if mode == "step" else f":{mode}"))
     if not rec or rec.get("source_sha") != kernel_source_sha(path):
         return None
     return rec.get("dram_bytes_per_launch")
@@ -197,7 +211,7 @@ def traffic_for(kernel: str, workload: str, path: str):
 # the oracle on the host cores (baseline arm and cpu_baseline)
 # ---------------------------------------------------------------------------------------
 
-def oracle_samples_per_s(w, target_s: float, max_steps: int = 1000, sub_batch=None):
+def oracle_samples_per_s(w, target_s: float, max_steps: int = 1000, sub_batch=None, mode="step"):
     """Time the fp64 oracle, as it stands, on samples of the workload's batch.
 
     Each timed call is one oracle step over ``sub_batch`` samples (the whole batch by
@@ -218,7 +232,10 @@ def oracle_samples_per_s(w, target_s: float, max_steps: int = 1000, sub_batch=No
         A = [x.as_f64(a) for a in x.A]
         G = [x.as_f64(g) for g in x.Gout]
         t0 = time.perf_counter()
-        O.step(st, A, G, s, h)
+        if mode == "sqnorms":
+            O.sample_norms(A, G, s, h, [di for di, _ in w.layers])
+        else:
+            O.step(st, A, G, s, h)
         spent += time.perf_counter() - t0
         done += nb
         s += 1
@@ -232,7 +249,7 @@ def run_reference(args, rank: int, world: int):
     w = WL.get(args.workload)
     sub = max(1, min(w.B, 4))
     # warm-up calls (untimed), then K timed calls of a bounded sub-batch each
-    oracle_samples_per_s(w, 0.0, max_steps=max(1, args.warmup), sub_batch=sub)
+    oracle_samples_per_s(w, 0.0, max_steps=max(1, args.warmup), sub_batch=sub, mode=args.mode)
     import oracle.grape_oracle as O
     h = O.Hyper.of(w)
     st = O.State.init(WL.make_weights(w), w.r)
@@ -242,7 +259,10 @@ def run_reference(args, rank: int, world: int):
         A = [x.as_f64(a) for a in x.A]
         G = [x.as_f64(g) for g in x.Gout]
         t0 = time.perf_counter()
-        O.step(st, A, G, s, h)
+        if args.mode == "sqnorms":
+            O.sample_norms(A, G, s, h, [di for di, _ in w.layers])
+        else:
+            O.step(st, A, G, s, h)
         times.append(time.perf_counter() - t0)
     total = sum(times)
     value = sub * len(times) / total
@@ -253,7 +273,8 @@ def run_reference(args, rank: int, world: int):
         cores = os.cpu_count() or 1
     sample = f"{sub} of {w.B} samples per step, all {w.n_layers} layers, fp64 numpy oracle"
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "samples/s",
+        "impl": "reference", "metric": METRIC if args.mode == "step" else METRIC_SQNORMS,
+        "value": value, "unit": "samples/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -311,9 +332,13 @@ def main(argv=None):
         sets.append(([conv(a).to(dev) for a in x.A], [conv(a).to(dev) for a in x.Gout]))
     set_bytes = w.input_bytes()
 
+    sq_out = torch.empty(w.B, dtype=torch.float32, device=dev)
+
     def one(s):
         A, G = sets[s % n_sets]
-        if world > 1:
+        if args.mode == "sqnorms":
+            g.sqnorms(A, G, s, out=sq_out)     # per-sample estimates only (no exchange needed)
+        elif world > 1:
             dp_step(g, A, G, Wd, s)
         else:
             g.step(A, G, Wd, s)
@@ -404,8 +429,8 @@ def main(argv=None):
         bound, unit = "alu", "TFLOP/s"
         achieved = work[dom]["flops"] / avg_s / 1e12
         peak = 148 * 128 * 2 * pk["sm_max_mhz"] * 1e6 / 1e12
-    traffic = traffic_for(dom, w.name, path_name)
-    flops, byts = step_work(w)
+    traffic = traffic_for(dom, w.name, path_name, args.mode)
+    flops, byts = step_work(w) if args.mode == "step" else sqnorms_work(w)
     t_roof = max(flops / (pk["bf16_tflops"] * 1e12), byts / (pk["hbm_gbs"] * 1e9))
 
     # ---- end to end through the public API: host buffers, copies in the timed region ----
@@ -417,12 +442,27 @@ def main(argv=None):
         hostG = [torch.from_numpy(a.view(np.int16) if w.dtype == "bf16" else a).pin_memory()
                  for a in x.Gout]
         norms = torch.empty(w.B, dtype=torch.float32).pin_memory()
-        g.step_host(hostA, hostG, Wd, step, norms)    # first call allocates the staging
+        if args.mode == "sqnorms":
+            # public call with device buffers: copy the step's inputs in, estimate, copy out
+            dA, dG = sets[0]
+
+            def e2e_one(s):
+                for d, h_ in zip(dA, hostA):
+                    d.view(torch.int16 if w.dtype == "bf16" else d.dtype).copy_(h_, non_blocking=True)
+                for d, h_ in zip(dG, hostG):
+                    d.view(torch.int16 if w.dtype == "bf16" else d.dtype).copy_(h_, non_blocking=True)
+                g.sqnorms(dA, dG, s, out=sq_out)
+                norms.copy_(sq_out, non_blocking=True)
+                torch.cuda.current_stream().synchronize()
+        else:
+            def e2e_one(s):
+                g.step_host(hostA, hostG, Wd, s, norms)   # synchronises its stream
+        e2e_one(step)    # first call allocates the staging
         step += 1
         barrier()
         t0 = time.perf_counter()
         for _ in range(args.e2e_steps):
-            g.step_host(hostA, hostG, Wd, step, norms)   # synchronises its stream
+            e2e_one(step)
             step += 1
         el = time.perf_counter() - t0
         if world > 1:
@@ -431,25 +471,29 @@ def main(argv=None):
             el = float(t.item())
         e2e = {"value": world * w.B * args.e2e_steps / el, "unit": "samples/s",
                "h2d_bytes_per_step": set_bytes, "d2h_bytes_per_step": 4 * w.B,
-               "steps": args.e2e_steps, "note": "grape_step_host: pinned host A/Gout copied in, "
-                                                "per-sample norms copied out, every step"}
+               "steps": args.e2e_steps,
+               "note": ("grape_step_host: pinned host A/Gout copied in, per-sample norms copied out, "
+                        "every step") if args.mode == "step" else
+                       ("pinned host A/Gout copied in, grape_sqnorms, the B estimates copied out, "
+                        "every step")}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, n, secs, cores = oracle_samples_per_s(w, args.cpu_seconds)
+        v, n, secs, cores = oracle_samples_per_s(w, args.cpu_seconds, mode=args.mode)
         cpu = {"value": v, "unit": "samples/s", "cores": cores, "kind": "oracle",
                "sample": f"{n} samples ({n // w.B} full steps of B={w.B}) of {w.name}, "
                          f"{secs:.1f} s of fp64 numpy oracle time"}
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": samples_per_s, "unit": "samples/s", "n_gpus": world,
+            "metric": METRIC if args.mode == "step" else METRIC_SQNORMS,
+            "value": samples_per_s, "unit": "samples/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic",
             "config": {"workload": w.name, "layers": layer_summary(w),
                        "r": w.r, "B_per_gpu": w.B, "global_batch": w.B * world, "T": w.T,
-                       "path": path_name, "parallelism": f"dp{world}",
+                       "path": path_name, "parallelism": f"dp{world}", "mode": args.mode,
                        "l2": (f"inputs rotate over {n_sets} distinct sets of "
                               f"{set_bytes / 1e6:.0f} MB each (> 126 MB L2)")
                              if set_bytes > L2_BYTES else

@@ -125,6 +125,35 @@ GRAPE_API int grape_accumulate(grape_ctx* ctx, const void* const* A, const void*
 GRAPE_API int grape_S_ptr(grape_ctx* ctx, int32_t layer, float** S_dev);
 GRAPE_API int grape_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_total, void* stream);
 
+/* Projection-refresh period K >= 1 (default 1).  P_l of step s is drawn with
+ * the step field of its Philox counter set to floor(s / K) instead of s, so one
+ * random subspace serves K consecutive steps (the refresh schedule is left
+ * open by design choice 1 of "Metodologia: DP-GRAPE" in the technical summary
+ * of "Memory-Efficient Differentially Private Training with Gradient Random
+ * Projection": P is "regenerated from a seed").  The noise is still drawn per
+ * step, and m and v carry over a refresh unchanged.  A step whose key equals
+ * that of the P already in the library's scratch does not regenerate it.
+ * Setting the period makes the next step draw P afresh.  The scratch is shared
+ * by every call on the handle: a caller that alternates streams orders them.
+ * Errors: GRAPE_EINVAL when K < 1 or ctx is NULL. */
+GRAPE_API int grape_set_refresh_period(grape_ctx* ctx, int32_t period);
+
+/* Per-sample squared norm estimates only: for every sample i,
+ *   sqnorms_dev[i] = sum_l || (A_{i,l} P_l)^T Gout_{i,l} ||_F^2,
+ * with P_l the step's projection (entries N(0, 1/r), key as for grape_step).
+ * This is the Hutchinson estimate of the full per-sample gradient norm
+ * sum_l ||A_{i,l}^T Gout_{i,l}||_F^2 with k = r Gaussian sketch columns
+ * ("Metodologia: DP-SGD-RC" and step 3 of its "Flujo Algoritmico", technical
+ * summary of DP-SGD-RC, gist.science 2605.24879): unbiased, with variance
+ * 2 ||O||_F^2 / r per layer for O = (A^T G)(A^T G)^T.  No clip, aggregation,
+ * noise or update runs, and m, v, W and the step's norms are untouched.
+ *  A[l], Gout[l]  device inputs, same layouts as grape_step
+ *  sqnorms_dev    device pointer to B floats (written)
+ * Enqueued on `stream`; returns before the results are ready.
+ * Errors: GRAPE_EINVAL for bad pointers or step; GRAPE_ECUDA for a launch error. */
+GRAPE_API int grape_sqnorms(grape_ctx* ctx, const void* const* A, const void* const* Gout, int64_t step,
+                            float* sqnorms_dev, void* stream);
+
 /* Checkpoint / resume of the projected Adam moments of one layer (r x d_out
  * fp32 each, device pointers), enqueued on `stream`.  P is not state: it is
  * regenerated from (seed, layer, step). */

@@ -48,6 +48,10 @@ struct grape_ctx {
   // staging for grape_step_host (allocated on first use)
   std::vector<void*> stage_A, stage_G;
   int64_t last_step = -1;
+  // projection refresh: P of step s is drawn with key s / refresh; p_key is the key of
+  // the P now in the scratch (-1: none), so a step with the same key skips generating it
+  uint32_t refresh = 1;
+  int64_t p_key = -1;
   double beta1 = 0.9, beta2 = 0.999;   // as given (bias corrections are formed in double)
   std::string err;
   // measurement
@@ -141,43 +145,51 @@ int phase(grape_ctx* ctx, int id, const char* what, cudaStream_t st, F&& launch)
   return GRAPE_OK;
 }
 
+// Generate P when its key changed, then AP = A P and the per-sample norm partials.
+int run_project_norm(grape_ctx* ctx, const grape::LayerIo* io, int64_t step, cudaStream_t st) {
+  const grape::StepShape& sh = ctx->sh;
+  const grape::LayerWs* ws = ctx->ws.data();
+  const uint32_t key = static_cast<uint32_t>(step) / ctx->refresh;
+  const bool gen = static_cast<int64_t>(key) != ctx->p_key;
+  int rc;
+  if (gen) {
+    ctx->p_key = -1;   // the scratch is being rewritten
+    rc = phase(ctx, GRAPE_PHASE_GEN_P, "generate P", st, [&](int* n) {
+      if (ctx->path == GRAPE_PATH_TC) return grape::tc_generate_P(sh, ws, ctx->tc, key, st, n);
+      *n = 1;
+      return grape::simt_generate_P(sh, ws, key, st);
+    });
+    if (rc) return rc;
+    ctx->p_key = key;
+  }
+  if (ctx->path == GRAPE_PATH_TC) {
+    const grape::TcWorkspace& tc = ctx->tc;
+    rc = phase(ctx, GRAPE_PHASE_PROJECT, "project", st,
+               [&](int* n) { return grape::tc_project(sh, ws, io, tc, st, n, !gen); });
+    if (rc) return rc;
+    return phase(ctx, GRAPE_PHASE_NORM, "per-sample norms", st, [&](int* n) {
+      return grape::tc_project_norm(sh, ws, io, tc, ctx->partials, st, n);
+    });
+  }
+  rc = phase(ctx, GRAPE_PHASE_PROJECT, "project", st, [&](int* n) {
+    *n = 1;
+    return grape::simt_project_ap(sh, ws, io, st);
+  });
+  if (rc) return rc;
+  return phase(ctx, GRAPE_PHASE_NORM, "per-sample norms", st, [&](int* n) {
+    *n = 1;
+    return grape::simt_project_norm(sh, ws, io, ctx->partials, st);
+  });
+}
+
 int run_accumulate(grape_ctx* ctx, const void* const* A, const void* const* G, int64_t step,
                    cudaStream_t st) {
   std::vector<grape::LayerIo> io(ctx->sh.L);
   for (int l = 0; l < ctx->sh.L; ++l) io[l] = grape::LayerIo{A[l], G[l], nullptr};
   const grape::StepShape& sh = ctx->sh;
   const grape::LayerWs* ws = ctx->ws.data();
-  const uint32_t s = static_cast<uint32_t>(step);
-  int rc;
-  if (ctx->path == GRAPE_PATH_TC) {
-    const grape::TcWorkspace& tc = ctx->tc;
-    rc = phase(ctx, GRAPE_PHASE_GEN_P, "generate P", st,
-               [&](int* n) { return grape::tc_generate_P(sh, ws, tc, s, st, n); });
-    if (rc) return rc;
-    rc = phase(ctx, GRAPE_PHASE_PROJECT, "project", st,
-               [&](int* n) { return grape::tc_project(sh, ws, io.data(), tc, st, n); });
-    if (rc) return rc;
-    rc = phase(ctx, GRAPE_PHASE_NORM, "per-sample norms", st, [&](int* n) {
-      return grape::tc_project_norm(sh, ws, io.data(), tc, ctx->partials, st, n);
-    });
-    if (rc) return rc;
-  } else {
-    rc = phase(ctx, GRAPE_PHASE_GEN_P, "generate P", st, [&](int* n) {
-      *n = 1;
-      return grape::simt_generate_P(sh, ws, s, st);
-    });
-    if (rc) return rc;
-    rc = phase(ctx, GRAPE_PHASE_PROJECT, "project", st, [&](int* n) {
-      *n = 1;
-      return grape::simt_project_ap(sh, ws, io.data(), st);
-    });
-    if (rc) return rc;
-    rc = phase(ctx, GRAPE_PHASE_NORM, "per-sample norms", st, [&](int* n) {
-      *n = 1;
-      return grape::simt_project_norm(sh, ws, io.data(), ctx->partials, st);
-    });
-    if (rc) return rc;
-  }
+  int rc = run_project_norm(ctx, io.data(), step, st);
+  if (rc) return rc;
   rc = phase(ctx, GRAPE_PHASE_CLIP, "clip", st, [&](int* n) {
     if (ctx->path == GRAPE_PATH_TC)
       return grape::tc_clip_scale(sh, ws, ctx->tc, ctx->partials, ctx->norms, ctx->clip, st, n);
@@ -479,6 +491,34 @@ int grape_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_tot
   rc = validate_io(ctx, nullptr, nullptr, W, false, true);
   if (rc) return rc;
   return run_apply(ctx, W, step, batch_total, static_cast<cudaStream_t>(stream));
+}
+
+int grape_set_refresh_period(grape_ctx* ctx, int32_t period) {
+  if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  if (period < 1) return ctx->fail(GRAPE_EINVAL, "refresh period must be >= 1");
+  ctx->refresh = static_cast<uint32_t>(period);
+  ctx->p_key = -1;   // the next step draws P afresh
+  return GRAPE_OK;
+}
+
+int grape_sqnorms(grape_ctx* ctx, const void* const* A, const void* const* Gout, int64_t step,
+                  float* sqnorms_dev, void* stream) {
+  if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  int rc = check_step_index(ctx, step);
+  if (rc) return rc;
+  rc = validate_io(ctx, A, Gout, nullptr, true, false);
+  if (rc) return rc;
+  if (!sqnorms_dev || (reinterpret_cast<uintptr_t>(sqnorms_dev) & 3u) != 0)
+    return ctx->fail(GRAPE_EINVAL, "sqnorms_dev must be a non-null, 4-byte aligned device pointer");
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::vector<grape::LayerIo> io(ctx->sh.L);
+  for (int l = 0; l < ctx->sh.L; ++l) io[l] = grape::LayerIo{A[l], Gout[l], nullptr};
+  rc = run_project_norm(ctx, io.data(), step, st);
+  if (rc) return rc;
+  return phase(ctx, GRAPE_PHASE_CLIP, "sum norm partials", st, [&](int* n) {
+    *n = 1;
+    return grape::sum_partials(ctx->sh, ctx->partials, sqnorms_dev, st);
+  });
 }
 
 int grape_get_state(grape_ctx* ctx, int32_t layer, float* m_dev, float* v_dev, void* stream) {

@@ -50,11 +50,14 @@ struct UpdateScalars {
 
 // ---- CUDA-core (SIMT, fp32) kernels: simt.cu --------------------------------
 // Each enqueues on `st` and returns cudaGetLastError().
-cudaError_t simt_generate_P(const StepShape& sh, const LayerWs* ws, uint32_t step, cudaStream_t st);
+// `key`: the step field of P's Philox counter (the step, or step / refresh period).
+cudaError_t simt_generate_P(const StepShape& sh, const LayerWs* ws, uint32_t key, cudaStream_t st);
 cudaError_t simt_project_ap(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                             cudaStream_t st);
 cudaError_t simt_project_norm(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                               float* partials, cudaStream_t st);
+// Per-sample squared norms: each sample's partial slots summed in a fixed order (no clip).
+cudaError_t sum_partials(const StepShape& sh, const float* partials, float* sqnorms, cudaStream_t st);
 cudaError_t finalize_clip(const StepShape& sh, const float* partials, float* norms, float* clip,
                           cudaStream_t st);
 cudaError_t simt_aggregate(const StepShape& sh, const LayerWs* ws, const LayerIo* io,

@@ -174,6 +174,18 @@ __global__ void __launch_bounds__(kThreads) clip_kernel(StepShape sh, const floa
   }
 }
 
+// ---- per-sample squared norms alone (the Hutchinson estimate): the sum of a sample's
+// partial slots over all layers, in the same fixed order, with no clip ----------------
+__global__ void __launch_bounds__(kThreads) sum_partials_kernel(StepShape sh, const float* partials,
+                                                                float* sqnorms) {
+  const int i = blockIdx.x;
+  const float* p = partials + static_cast<size_t>(i) * sh.part_stride;
+  float ss = 0.0f;
+  for (int k = threadIdx.x; k < sh.part_stride; k += kThreads) ss += p[k];
+  const float tot = block_sum(ss);
+  if (threadIdx.x == 0) sqnorms[i] = tot;
+}
+
 // ---- a5: S_l = sum_i c_i R_i = sum over stacked rows of c_{row/T} AP[row]^T Gout[row] --
 __global__ void __launch_bounds__(kThreads) aggregate_kernel(StepShape sh, LayerTable tab,
                                                              const float* clip) {
@@ -395,6 +407,11 @@ cudaError_t simt_project_norm(const StepShape& sh, const LayerWs* ws, const Laye
 cudaError_t finalize_clip(const StepShape& sh, const float* partials, float* norms, float* clip,
                           cudaStream_t st) {
   clip_kernel<<<sh.B, kThreads, 0, st>>>(sh, partials, norms, clip);
+  return cudaGetLastError();
+}
+
+cudaError_t sum_partials(const StepShape& sh, const float* partials, float* sqnorms, cudaStream_t st) {
+  sum_partials_kernel<<<sh.B, kThreads, 0, st>>>(sh, partials, sqnorms);
   return cudaGetLastError();
 }
 

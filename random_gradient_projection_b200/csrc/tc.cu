@@ -896,8 +896,11 @@ int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
 // Launch as a programmatic dependent of the previous kernel in the stream (the kernel
 // itself waits with griddepcontrol.wait before it reads that kernel's outputs).
+// A programmatic dependent launch when `pdl`, else an ordinary one (the first kernel of a
+// step is ordinary: it waits for all earlier work, which the early loads rely on).
 template <class Kern, class... Args>
-cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+cudaError_t launch_maybe_pdl(bool pdl, Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             Args... args) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -907,8 +910,13 @@ cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStre
   a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   a[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = a;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+template <class Kern, class... Args>
+cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  return launch_maybe_pdl(true, kernel, grid, block, smem, st, args...);
 }
 
 int sm_count() {
@@ -926,7 +934,7 @@ int sm_count() {
 // for a kernel that allocates TMEM), never more than there are tiles.  A larger grid
 // would run its surplus CTAs as a second wave behind the first.
 template <int MODE, int BN, int STAGES>
-cudaError_t launch_group(GroupParams& gp, int tiles, cudaStream_t st) {
+cudaError_t launch_group(GroupParams& gp, int tiles, cudaStream_t st, bool pdl = true) {
   using S = Smem<BN, STAGES, ModeExtra<MODE>::kBytes>;
   static int per_sm = 0;
   if (per_sm == 0) {
@@ -945,14 +953,16 @@ cudaError_t launch_group(GroupParams& gp, int tiles, cudaStream_t st) {
   if (tiles <= 0) return cudaSuccess;
   int grid = sm_count() * per_sm;
   grid = grid < tiles ? grid : tiles;
-  return launch_pdl(tc_gemm_kernel<MODE, BN, STAGES>, dim3(grid), dim3(kThreads), S::kBytes, st, gp);
+  return launch_maybe_pdl(pdl, tc_gemm_kernel<MODE, BN, STAGES>, dim3(grid), dim3(kThreads), S::kBytes, st, gp);
 }
 
 // Build and launch the groups of one mode.  fill(g, l, gp) sets maps and the layer record
 // (except tiles_begin) and returns the tile count of layer l.
+// `pdl_first` = false makes the first launch an ordinary one (used when it is the step's
+// first kernel); later groups always follow a kernel of the same step.
 template <int MODE, int BN, int STAGES, class Fill>
 cudaError_t run_mode(const HostState& hs, int L, cudaStream_t st, int* launches, const Fill& fill,
-                     GroupParams& gp) {
+                     GroupParams& gp, bool pdl_first = true) {
   for (int l0 = 0; l0 < L; l0 += kMaxGroup) {
     const int n = (L - l0) < kMaxGroup ? (L - l0) : kMaxGroup;
     gp.n_layers = n;
@@ -963,7 +973,7 @@ cudaError_t run_mode(const HostState& hs, int L, cudaStream_t st, int* launches,
       gp.lay[g].tiles_begin = tiles;
       tiles += t;
     }
-    cudaError_t e = launch_group<MODE, BN, STAGES>(gp, tiles, st);
+    cudaError_t e = launch_group<MODE, BN, STAGES>(gp, tiles, st, l0 == 0 ? pdl_first : true);
     if (e != cudaSuccess) return e;
     ++*launches;
   }
@@ -1082,7 +1092,7 @@ cudaError_t tc_generate_P(const StepShape& sh, const LayerWs* ws, const TcWorksp
 }
 
 cudaError_t tc_project(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
-                       const TcWorkspace& tc, cudaStream_t st, int* launches) {
+                       const TcWorkspace& tc, cudaStream_t st, int* launches, bool first_in_step) {
   HostState& hs = *static_cast<HostState*>(tc.host_state);
   GroupParams& gp = hs.gp;
   std::memset(&gp, 0, sizeof(gp));
@@ -1107,8 +1117,8 @@ cudaError_t tc_project(const StepShape& sh, const LayerWs* ws, const LayerIo* io
     return true;
   };
   if (hs.bn_project == 128)
-    return run_mode<PROJECT, 128, kStagesProject128>(hs, sh.L, st, launches, fill, gp);
-  return run_mode<PROJECT, 256, kStagesProject256>(hs, sh.L, st, launches, fill, gp);
+    return run_mode<PROJECT, 128, kStagesProject128>(hs, sh.L, st, launches, fill, gp, !first_in_step);
+  return run_mode<PROJECT, 256, kStagesProject256>(hs, sh.L, st, launches, fill, gp, !first_in_step);
 }
 
 cudaError_t tc_project_norm(const StepShape& sh, const LayerWs* ws, const LayerIo* io,

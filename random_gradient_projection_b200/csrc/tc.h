@@ -25,10 +25,13 @@ void tc_release(TcWorkspace* tc);
 int* tc_error_word(const TcWorkspace& tc);
 // The phases of the tensor-core path; each enqueues on `st`, adds the number of
 // kernels it launched to *launches and returns the first CUDA error.
+// `key` is the step field of P's Philox counter (the step, or step / refresh period).
 cudaError_t tc_generate_P(const StepShape& sh, const LayerWs* ws, const TcWorkspace& tc,
-                          uint32_t step, cudaStream_t st, int* launches);
+                          uint32_t key, cudaStream_t st, int* launches);
+// `first_in_step`: no P was generated this step (it is still valid from an earlier one),
+// so the projection is the step's first kernel and is launched as an ordinary launch.
 cudaError_t tc_project(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
-                       const TcWorkspace& tc, cudaStream_t st, int* launches);
+                       const TcWorkspace& tc, cudaStream_t st, int* launches, bool first_in_step);
 cudaError_t tc_project_norm(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                             const TcWorkspace& tc, float* partials, cudaStream_t st, int* launches);
 cudaError_t tc_clip_scale(const StepShape& sh, const LayerWs* ws, const TcWorkspace& tc,

@@ -29,7 +29,7 @@ EXPORTS = (
     "grape_apply", "grape_get_state", "grape_set_state", "grape_debug", "grape_device_bytes",
     "grape_path_of", "grape_last_error", "grape_global_error", "grape_destroy",
     "grape_philox_words", "grape_gaussian", "grape_profile", "grape_profile_read",
-    "grape_launch_count", "grape_layer_sqnorms_static",
+    "grape_launch_count", "grape_layer_sqnorms_static", "grape_set_refresh_period", "grape_sqnorms",
 )
 PHASES = ("gen_P", "project", "norm", "clip", "aggregate", "adam", "backproject")
 
@@ -77,6 +77,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "grape_profile_read": ([vp, vp, vp], i32),
         "grape_launch_count": ([vp, ctypes.POINTER(u64)], i32),
         "grape_layer_sqnorms_static": ([vp, vp, i32, i32, i32, i32, i32, u64, u32, u32, vp, vp], i32),
+        "grape_set_refresh_period": ([vp, i32], i32),
+        "grape_sqnorms": ([vp, pp, pp, i64, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -152,6 +154,14 @@ def grape_step_host(ctx: int, A_host, Gout_host, W, step: int, norms_host=None, 
 
 def grape_accumulate(ctx: int, A, Gout, step: int, stream=None):
     _check(lib().grape_accumulate(ctx, _array(A), _array(Gout), step, _stream(stream)), ctx)
+
+
+def grape_set_refresh_period(ctx: int, period: int):
+    _check(lib().grape_set_refresh_period(ctx, period), ctx)
+
+
+def grape_sqnorms(ctx: int, A, Gout, step: int, sqnorms_dev, stream=None):
+    _check(lib().grape_sqnorms(ctx, _array(A), _array(Gout), step, _ptr(sqnorms_dev), _stream(stream)), ctx)
 
 
 def grape_S_ptr(ctx: int, layer: int) -> int:
@@ -255,8 +265,23 @@ class GrapeStep:
 
     @classmethod
     def for_workload(cls, w, path=GRAPE_PATH_AUTO, B=None):
-        return cls(w.layers, w.r, w.C, w.sigma, w.seed, B or w.B, w.T, w.dtype, w.lr, w.beta1,
-                   w.beta2, w.eps, path)
+        g = cls(w.layers, w.r, w.C, w.sigma, w.seed, B or w.B, w.T, w.dtype, w.lr, w.beta1,
+                w.beta2, w.eps, path)
+        if getattr(w, "refresh", 1) != 1:
+            g.set_refresh_period(w.refresh)
+        return g
+
+    def set_refresh_period(self, period: int):
+        grape_set_refresh_period(self.ctx, period)
+
+    def sqnorms(self, A, Gout, step: int, out=None, stream=None):
+        """Per-sample squared norm estimates sum_l ||(A_il P_l)^T Gout_il||^2 (B floats on
+        the device); `out` is a torch float32 tensor of B elements, or one is allocated."""
+        if out is None:
+            import torch
+            out = torch.empty(self.B, dtype=torch.float32, device=A[0].device)
+        grape_sqnorms(self.ctx, A, Gout, step, out, stream)
+        return out
 
     def close(self):
         if self.ctx:

@@ -68,3 +68,10 @@ def test_generator_entry_points_validate(lib):
         grape.grape_philox_words(0, 0, 0, 0, 16, 8, stream=0)   # misaligned output
     assert e.value.code == grape.GRAPE_EINVAL
     grape.grape_gaussian(0, 0, 0, 0, 0, 0, stream=0)              # empty request is a no-op
+
+
+def test_refresh_and_sqnorms_validate_the_handle(lib):
+    """Both reject a NULL handle on the host, before any device work."""
+    assert lib.grape_set_refresh_period(None, 2) == 1          # GRAPE_EINVAL
+    assert b"ctx" in lib.grape_global_error()
+    assert lib.grape_sqnorms(None, None, None, 0, None, None) == 1
