@@ -300,6 +300,22 @@ def sample_norms(A: Sequence[np.ndarray], Gout: Sequence[np.ndarray], step_index
 
 
 # --------------------------------------------------------------------------
+# Loss-token masks
+#
+# The pages are silent about masking: a mask is a property of the workload
+# (tokens that carry no loss).  Reading: a masked token contributes nothing to
+# the sample's gradient, exactly as if its output gradient row were zero; the
+# gradient of a linear layer is a sum over tokens (A_i^T Gout_i = sum_t
+# a_t^T g_t), so dropping such tokens is an exact rewrite, not an approximation.
+# --------------------------------------------------------------------------
+
+def apply_token_mask(Gout: Sequence[np.ndarray], mask: np.ndarray) -> List[np.ndarray]:
+    """Gout_l with the rows of masked tokens set to zero; ``mask`` has shape (B, T), nonzero = kept."""
+    keep = (np.asarray(mask) != 0)[:, :, None]
+    return [np.where(keep, g, 0.0) for g in Gout]
+
+
+# --------------------------------------------------------------------------
 # Hutchinson estimate of a per-sample gradient norm (DP-SGD-RC)
 #
 # Source: "DP-SGD-RC" technical summary on the same site (gist.science,

@@ -365,6 +365,40 @@ def pin_refresh_period_two(O):
 
 
 # --------------------------------------------------------------------------
+# token masks
+# --------------------------------------------------------------------------
+
+def pin_masked_tokens_drop_out(O):
+    """A step on masked inputs equals the step on each sample's kept tokens alone, moved
+    to the front and zero-padded to a shorter T: the gradient is a sum over tokens, so
+    the step may not depend on T or on where the dropped tokens were."""
+    layers = ((7, 5), (6, 4))
+    B, T, T_cap = 3, 9, 5
+    A, G, W0 = _tiny_problem(31, B, T, layers, scale=0.8)
+    rng = np.random.default_rng(32)
+    mask = rng.random((B, T)) < 0.45
+    mask[0, :] = False                        # a sample with no live token
+    mask[1, :T_cap] = True; mask[1, T_cap:] = False   # one exactly at the capacity
+    h = O.Hyper(r=3, C=0.6, sigma=0.7, seed=9)
+    st_full = O.State.init(W0, h.r)
+    out_full = O.step(st_full, A, O.apply_token_mask(G, mask), 0, h)
+    Ac = [np.zeros((B, T_cap, a.shape[2])) for a in A]
+    Gc = [np.zeros((B, T_cap, g.shape[2])) for g in G]
+    for i in range(B):
+        live = np.flatnonzero(mask[i])
+        assert len(live) <= T_cap
+        for l in range(len(layers)):
+            Ac[l][i, :len(live)] = A[l][i, live]
+            Gc[l][i, :len(live)] = G[l][i, live]
+    st_c = O.State.init(W0, h.r)
+    out_c = O.step(st_c, Ac, Gc, 0, h)
+    assert np.allclose(out_full["norms"], out_c["norms"], rtol=1e-12, atol=0)
+    assert out_full["norms"][0] == 0.0 and out_full["clip"][0] == 1.0
+    for l in range(len(layers)):
+        assert np.allclose(st_full.W[l], st_c.W[l], rtol=0, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
 # Hutchinson norm estimate (DP-SGD-RC)
 # --------------------------------------------------------------------------
 
@@ -416,4 +450,5 @@ ALL_PINS = [
     pin_adam_first_step, pin_no_privacy_reduction, pin_backprojection_unbiased,
     pin_projection_before_privatization, pin_refresh_fixed_subspace, pin_refresh_period_two,
     pin_hutchinson_identity_sketch, pin_hutchinson_unbiased, pin_hutchinson_factored,
+    pin_masked_tokens_drop_out,
 ]

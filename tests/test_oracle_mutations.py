@@ -79,6 +79,10 @@ MUTATIONS = {
     # Hutchinson estimate
     "hutch_wrong_gram": ("O = G @ G.T", "O = G @ G.T + np.eye(G.shape[0])"),
     "hutch_first_column": ("for j in range(P.shape[1])))", "for j in range(1)))"),
+    # token mask
+    "mask_inverted": ("keep = (np.asarray(mask) != 0)[:, :, None]", "keep = (np.asarray(mask) == 0)[:, :, None]"),
+    "mask_zeroes_nothing": ("return [np.where(keep, g, 0.0) for g in Gout]", "return [g for g in Gout]"),
+    "token_mean_gradient": ("return A_i.T @ Gout_i", "return A_i.T @ Gout_i / A_i.shape[0]"),
     "hutch_transposed_sketch": ("return float(sum(P[:, j] @ O @ P[:, j] for j in range(P.shape[1])))",
                                 "return float(sum(P[:, j] @ O.T @ O @ P[:, j] for j in range(P.shape[1])))"),
 }
