@@ -63,6 +63,9 @@ def parse(argv=None):
     ap.add_argument("--workload", default="mlp4x1024", choices=sorted(WL.WORKLOADS))
     ap.add_argument("--mode", default="step", choices=["step", "sqnorms"],
                     help="step: the whole DP-GRAPE step; sqnorms: per-sample norm estimates only")
+    ap.add_argument("--mask-capacity", type=int, default=0,
+                    help="run masked steps (grape_step_masked) keeping at most this many loss "
+                         "tokens per sample; the workload's own token mask is passed in")
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -153,7 +156,7 @@ def phase_work(w, path: str):
     el = 4 if w.dtype == "f32" else 2
     ap_el = 4 if path == "simt" else 2
     dr_el = 4 if path == "simt" else 2
-    p_el = 4 if path == "simt" else 4          # tensor-core path writes P and P^T in bf16
+    p_el = 4 if path == "simt" else 2          # fp32 P on the CUDA cores, bf16 on the tensor path
     rows = w.B * w.T
     out = {}
     out["gen_P"] = {"bytes": sum(di * w.r * p_el for di, _ in w.layers), "flops": 0}
@@ -169,6 +172,9 @@ def phase_work(w, path: str):
     out["backproject"] = {"bytes": sum(8 * di * do + di * w.r * ap_el + w.r * do * dr_el
                                        for di, do in w.layers),
                           "flops": sum(2 * di * w.r * do for di, do in w.layers)}
+    # live-token compaction (--mask-capacity): scan the mask, read and write the kept rows
+    out["compact"] = {"bytes": w.B * w.T + sum(2 * rows * (di + do) * el for di, do in w.layers),
+                      "flops": 0}
     return out
 
 
@@ -317,7 +323,12 @@ def main(argv=None):
     w = WL.get(args.workload)
     path = {"auto": grape.GRAPE_PATH_AUTO, "simt": grape.GRAPE_PATH_SIMT,
             "tc": grape.GRAPE_PATH_TC}[args.path]
-    g = GrapeStep.for_workload(w, path=path)
+    masked = args.mask_capacity > 0
+    if masked and (args.mode != "step" or world > 1):
+        raise SystemExit("--mask-capacity runs the single-GPU step only")
+    g = GrapeStep.for_workload(w.replace(T=args.mask_capacity) if masked else w, path=path)
+    if masked:
+        g.enable_compaction(w.T)
     path_name = {grape.GRAPE_PATH_SIMT: "simt", grape.GRAPE_PATH_TC: "tc"}[g.path]
     Wd = [torch.from_numpy(x).to(dev) for x in WL.make_weights(w)]
 
@@ -329,14 +340,17 @@ def main(argv=None):
         x = WL.make_step_inputs(win, k, threads=16)
         conv = (lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)) \
             if w.dtype == "bf16" else torch.from_numpy
-        sets.append(([conv(a).to(dev) for a in x.A], [conv(a).to(dev) for a in x.Gout]))
+        sets.append(([conv(a).to(dev) for a in x.A], [conv(a).to(dev) for a in x.Gout],
+                     torch.from_numpy((x.mask != 0).astype(np.uint8)).to(dev)))
     set_bytes = w.input_bytes()
 
     sq_out = torch.empty(w.B, dtype=torch.float32, device=dev)
 
     def one(s):
-        A, G = sets[s % n_sets]
-        if args.mode == "sqnorms":
+        A, G, M = sets[s % n_sets]
+        if masked:
+            g.step_masked(A, G, Wd, M, s)
+        elif args.mode == "sqnorms":
             g.sqnorms(A, G, s, out=sq_out)     # per-sample estimates only (no exchange needed)
         elif world > 1:
             dp_step(g, A, G, Wd, s)
@@ -406,7 +420,10 @@ def main(argv=None):
     g.profile(False)
 
     pk = peaks()
-    work = phase_work(w, path_name)
+    w_run = w.replace(T=args.mask_capacity) if masked else w   # rows the GEMM phases see
+    work = phase_work(w_run, path_name)
+    if masked:
+        work["compact"]["bytes"] = w.B * w.T + (work["compact"]["bytes"] - w_run.B * w_run.T)
     per_phase = {}
     for name, (pms, calls) in phases.items():
         if calls == 0:
@@ -430,7 +447,12 @@ def main(argv=None):
         achieved = work[dom]["flops"] / avg_s / 1e12
         peak = 148 * 128 * 2 * pk["sm_max_mhz"] * 1e6 / 1e12
     traffic = traffic_for(dom, w.name, path_name, args.mode)
-    flops, byts = step_work(w) if args.mode == "step" else sqnorms_work(w)
+    if masked:
+        # the live-token lower bound: the method's work over the kept tokens only
+        kept = float(np.mean([m.float().sum(dim=1).mean().item() for _, _, m in sets]))
+        flops, byts = step_work(w.replace(T=max(1, int(round(kept)))))
+    else:
+        flops, byts = step_work(w) if args.mode == "step" else sqnorms_work(w)
     t_roof = max(flops / (pk["bf16_tflops"] * 1e12), byts / (pk["hbm_gbs"] * 1e9))
 
     # ---- end to end through the public API: host buffers, copies in the timed region ----
@@ -442,9 +464,21 @@ def main(argv=None):
         hostG = [torch.from_numpy(a.view(np.int16) if w.dtype == "bf16" else a).pin_memory()
                  for a in x.Gout]
         norms = torch.empty(w.B, dtype=torch.float32).pin_memory()
-        if args.mode == "sqnorms":
+        if masked:
+            dA, dG, dM = sets[0]
+            hostM = torch.from_numpy((x.mask != 0).astype(np.uint8)).pin_memory()
+
+            def e2e_one(s):
+                for d, h_ in zip(dA, hostA):
+                    d.view(torch.int16 if w.dtype == "bf16" else d.dtype).copy_(h_, non_blocking=True)
+                for d, h_ in zip(dG, hostG):
+                    d.view(torch.int16 if w.dtype == "bf16" else d.dtype).copy_(h_, non_blocking=True)
+                dM.copy_(hostM, non_blocking=True)
+                g.step_masked(dA, dG, Wd, dM, s)
+                g.norms()                          # synchronises and reads the B norms back
+        elif args.mode == "sqnorms":
             # public call with device buffers: copy the step's inputs in, estimate, copy out
-            dA, dG = sets[0]
+            dA, dG, _ = sets[0]
 
             def e2e_one(s):
                 for d, h_ in zip(dA, hostA):
@@ -470,9 +504,11 @@ def main(argv=None):
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             el = float(t.item())
         e2e = {"value": world * w.B * args.e2e_steps / el, "unit": "samples/s",
-               "h2d_bytes_per_step": set_bytes, "d2h_bytes_per_step": 4 * w.B,
+               "h2d_bytes_per_step": set_bytes + (w.B * w.T if masked else 0), "d2h_bytes_per_step": 4 * w.B,
                "steps": args.e2e_steps,
-               "note": ("grape_step_host: pinned host A/Gout copied in, per-sample norms copied out, "
+               "note": ("pinned host A/Gout and the token mask copied in, grape_step_masked, the B "
+                        "norms copied out, every step") if masked else
+                       ("grape_step_host: pinned host A/Gout copied in, per-sample norms copied out, "
                         "every step") if args.mode == "step" else
                        ("pinned host A/Gout copied in, grape_sqnorms, the B estimates copied out, "
                         "every step")}
@@ -494,6 +530,7 @@ def main(argv=None):
             "config": {"workload": w.name, "layers": layer_summary(w),
                        "r": w.r, "B_per_gpu": w.B, "global_batch": w.B * world, "T": w.T,
                        "path": path_name, "parallelism": f"dp{world}", "mode": args.mode,
+                       "mask_capacity": args.mask_capacity or None,
                        "l2": (f"inputs rotate over {n_sets} distinct sets of "
                               f"{set_bytes / 1e6:.0f} MB each (> 126 MB L2)")
                              if set_bytes > L2_BYTES else

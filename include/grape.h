@@ -125,6 +125,34 @@ GRAPE_API int grape_accumulate(grape_ctx* ctx, const void* const* A, const void*
 GRAPE_API int grape_S_ptr(grape_ctx* ctx, int32_t layer, float** S_dev);
 GRAPE_API int grape_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_total, void* stream);
 
+/* Live-token compaction for loss-masked inputs.  The pages are silent about
+ * masks; a masked token contributes nothing to a sample's gradient (the
+ * gradient of a linear layer is a sum over tokens), so dropping it before the
+ * projection is an exact rewrite of the step of "Metodologia: DP-GRAPE"
+ * (technical summary of "Memory-Efficient Differentially Private Training with
+ * Gradient Random Projection") that removes the masked tokens' share of the
+ * projection, norm and aggregation work.
+ *
+ * grape_enable_compaction: the context's T becomes the capacity (kept tokens per
+ *   sample); steps given to grape_step_masked read inputs of T_full >= T tokens
+ *   per sample.  Allocates B*T*(d_in + d_out) elements per layer of compact
+ *   buffers (input dtype) and B*T + B + 1 int32 of bookkeeping, zeroed; call once.
+ *   Errors: GRAPE_EINVAL (T_full < T, B > 65535, already enabled), GRAPE_ENOMEM.
+ * grape_step_masked: as grape_step, with A[l], Gout[l] of shape B x T_full x d and
+ *   mask_dev a device array of B x T_full bytes (row-major, nonzero = the token
+ *   carries loss and is kept; one mask for all layers).  Each sample's kept tokens,
+ *   in order, are gathered into T rows (zero padding after them) and the whole step
+ *   runs on those.  The result equals grape_step on inputs whose masked tokens'
+ *   Gout rows are zero.  A sample that keeps more than T tokens uses its first T
+ *   and makes the next synchronising call (grape_live_counts, grape_debug,
+ *   grape_step_host) return GRAPE_EINVAL.  Enqueued on `stream`.
+ * grape_live_counts: synchronises the device and copies the kept-token count of
+ *   each sample of the last masked step (at most T) to counts_host (B int32). */
+GRAPE_API int grape_enable_compaction(grape_ctx* ctx, int32_t T_full);
+GRAPE_API int grape_step_masked(grape_ctx* ctx, const void* const* A, const void* const* Gout,
+                                float* const* W, const uint8_t* mask_dev, int64_t step, void* stream);
+GRAPE_API int grape_live_counts(grape_ctx* ctx, int32_t* counts_host);
+
 /* Projection-refresh period K >= 1 (default 1).  P_l of step s is drawn with
  * the step field of its Philox counter set to floor(s / K) instead of s, so one
  * random subspace serves K consecutive steps (the refresh schedule is left
@@ -189,7 +217,8 @@ enum grape_phase {
   GRAPE_PHASE_AGGREGATE = 4,    /* S = sum_i c_i R_i */
   GRAPE_PHASE_ADAM = 5,         /* noise + projected Adam */
   GRAPE_PHASE_BACKPROJECT = 6,  /* W -= lr P dR */
-  GRAPE_N_PHASES = 7
+  GRAPE_PHASE_COMPACT = 7,      /* live-token scan and gather (grape_step_masked) */
+  GRAPE_N_PHASES = 8
 };
 GRAPE_API int grape_profile(grape_ctx* ctx, int32_t enable);
 GRAPE_API int grape_profile_read(grape_ctx* ctx, double* ms_out, int64_t* count_out);

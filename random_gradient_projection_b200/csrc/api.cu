@@ -11,6 +11,7 @@
 #include <vector>
 
 #include "../../include/grape.h"
+#include "compact.h"
 #include "kernels.h"
 #include "tc.h"
 
@@ -52,6 +53,14 @@ struct grape_ctx {
   // the P now in the scratch (-1: none), so a step with the same key skips generating it
   uint32_t refresh = 1;
   int64_t p_key = -1;
+  // live-token compaction (grape_enable_compaction): inputs of T_full tokens per sample,
+  // compacted to the context's T rows; one allocation holds every buffer below
+  int T_full = 0;
+  void* compact_buf = nullptr;
+  std::vector<void*> comp_A, comp_G;
+  int32_t* comp_idx = nullptr;
+  int32_t* comp_counts = nullptr;
+  int* comp_overflow = nullptr;
   double beta1 = 0.9, beta2 = 0.999;   // as given (bias corrections are formed in double)
   std::string err;
   // measurement
@@ -237,8 +246,19 @@ int run_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_total
   });
 }
 
-// After a device synchronisation: a tensor-core wait that gave up leaves a nonzero word.
+// After a device synchronisation: a sample that kept more live tokens than the compact
+// capacity, or a tensor-core wait that gave up, leaves a nonzero word.
 int check_device_error(grape_ctx* ctx) {
+  if (ctx->comp_overflow) {
+    int v = 0;
+    cudaError_t e = cudaMemcpy(&v, ctx->comp_overflow, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return ctx->cuda_fail(e, "read compaction flag");
+    if (v != 0) {
+      cudaMemset(ctx->comp_overflow, 0, sizeof(int));
+      return ctx->fail(GRAPE_EINVAL, "a sample kept more live tokens than the compaction capacity T = " +
+                                         std::to_string(ctx->sh.T) + " (only the first T were used)");
+    }
+  }
   if (ctx->path != GRAPE_PATH_TC) return GRAPE_OK;
   int* word = grape::tc_error_word(ctx->tc);
   if (!word) return GRAPE_OK;
@@ -493,6 +513,91 @@ int grape_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_tot
   return run_apply(ctx, W, step, batch_total, static_cast<cudaStream_t>(stream));
 }
 
+int grape_enable_compaction(grape_ctx* ctx, int32_t T_full) {
+  if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  if (T_full < ctx->sh.T) return ctx->fail(GRAPE_EINVAL, "T_full must be >= the context's T (the capacity)");
+  if (ctx->sh.B > 65535) return ctx->fail(GRAPE_EINVAL, "compaction supports B <= 65535");
+  if (ctx->compact_buf) return ctx->fail(GRAPE_EINVAL, "compaction is already enabled");
+  const size_t el = in_elsize(ctx->sh.dtype);
+  const size_t rows = static_cast<size_t>(ctx->sh.B) * ctx->sh.T;
+  Arena ar;
+  std::vector<size_t> oa, og;
+  for (const grape_layer& ly : ctx->layers) {
+    oa.push_back(ar.take(rows * ly.d_in * el));
+    og.push_back(ar.take(rows * ly.d_out * el));
+  }
+  const size_t o_idx = ar.take(rows * sizeof(int32_t));
+  const size_t o_cnt = ar.take(static_cast<size_t>(ctx->sh.B) * sizeof(int32_t));
+  const size_t o_flag = ar.take(sizeof(int));
+  void* buf = nullptr;
+  cudaError_t e = cudaMalloc(&buf, ar.off);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return ctx->fail(GRAPE_ENOMEM, "cudaMalloc of the compaction buffers failed");
+  }
+  e = cudaMemset(buf, 0, ar.off);
+  if (e != cudaSuccess) {
+    cudaFree(buf);
+    return ctx->cuda_fail(e, "cudaMemset");
+  }
+  char* base = static_cast<char*>(buf);
+  ctx->compact_buf = buf;
+  ctx->T_full = T_full;
+  for (size_t l = 0; l < oa.size(); ++l) {
+    ctx->comp_A.push_back(base + oa[l]);
+    ctx->comp_G.push_back(base + og[l]);
+  }
+  ctx->comp_idx = reinterpret_cast<int32_t*>(base + o_idx);
+  ctx->comp_counts = reinterpret_cast<int32_t*>(base + o_cnt);
+  ctx->comp_overflow = reinterpret_cast<int*>(base + o_flag);
+  return GRAPE_OK;
+}
+
+int grape_step_masked(grape_ctx* ctx, const void* const* A, const void* const* Gout, float* const* W,
+                      const uint8_t* mask_dev, int64_t step, void* stream) {
+  if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  if (!ctx->compact_buf) return ctx->fail(GRAPE_EINVAL, "call grape_enable_compaction first");
+  if (!mask_dev) return ctx->fail(GRAPE_EINVAL, "mask_dev must not be null");
+  int rc = check_step_index(ctx, step);
+  if (rc) return rc;
+  rc = validate_io(ctx, A, Gout, W, true, true);
+  if (rc) return rc;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const grape::StepShape& sh = ctx->sh;
+  rc = phase(ctx, GRAPE_PHASE_COMPACT, "compact live tokens", st, [&](int* n) {
+    *n = 2;
+    cudaError_t e = grape::compact_live_index(mask_dev, sh.B, ctx->T_full, sh.T, ctx->comp_idx,
+                                              ctx->comp_counts, ctx->comp_overflow, st);
+    if (e != cudaSuccess) return e;
+    grape::CompactTable tb{};
+    for (int l = 0; l < sh.L; ++l) {
+      tb.A[l] = A[l];
+      tb.G[l] = Gout[l];
+      tb.Ac[l] = ctx->comp_A[l];
+      tb.Gc[l] = ctx->comp_G[l];
+      tb.d_in[l] = ctx->layers[l].d_in;
+      tb.d_out[l] = ctx->layers[l].d_out;
+    }
+    return grape::compact_gather(tb, sh.L, sh.B, ctx->T_full, sh.T, static_cast<int>(in_elsize(sh.dtype)),
+                                 ctx->comp_idx, st);
+  });
+  if (rc) return rc;
+  rc = run_accumulate(ctx, ctx->comp_A.data(), ctx->comp_G.data(), step, st);
+  if (rc) return rc;
+  return run_apply(ctx, W, step, 0, st);
+}
+
+int grape_live_counts(grape_ctx* ctx, int32_t* counts_host) {
+  if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  if (!ctx->compact_buf) return ctx->fail(GRAPE_EINVAL, "compaction is not enabled");
+  if (!counts_host) return ctx->fail(GRAPE_EINVAL, "counts_host must not be null");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return ctx->cuda_fail(e, "cudaDeviceSynchronize");
+  e = cudaMemcpy(counts_host, ctx->comp_counts, sizeof(int32_t) * ctx->sh.B, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return ctx->cuda_fail(e, "cudaMemcpy");
+  return check_device_error(ctx);
+}
+
 int grape_set_refresh_period(grape_ctx* ctx, int32_t period) {
   if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
   if (period < 1) return ctx->fail(GRAPE_EINVAL, "refresh period must be >= 1");
@@ -656,6 +761,7 @@ void grape_destroy(grape_ctx* ctx) {
   for (void* p : ctx->stage_A) cudaFree(p);
   for (void* p : ctx->stage_G) cudaFree(p);
   if (ctx->arena) cudaFree(ctx->arena);
+  if (ctx->compact_buf) cudaFree(ctx->compact_buf);
   delete ctx;
 }
 

@@ -30,8 +30,9 @@ EXPORTS = (
     "grape_path_of", "grape_last_error", "grape_global_error", "grape_destroy",
     "grape_philox_words", "grape_gaussian", "grape_profile", "grape_profile_read",
     "grape_launch_count", "grape_layer_sqnorms_static", "grape_set_refresh_period", "grape_sqnorms",
+    "grape_enable_compaction", "grape_step_masked", "grape_live_counts",
 )
-PHASES = ("gen_P", "project", "norm", "clip", "aggregate", "adam", "backproject")
+PHASES = ("gen_P", "project", "norm", "clip", "aggregate", "adam", "backproject", "compact")   # GRAPE_N_PHASES
 
 
 class grape_layer(ctypes.Structure):
@@ -79,6 +80,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "grape_layer_sqnorms_static": ([vp, vp, i32, i32, i32, i32, i32, u64, u32, u32, vp, vp], i32),
         "grape_set_refresh_period": ([vp, i32], i32),
         "grape_sqnorms": ([vp, pp, pp, i64, vp, vp], i32),
+        "grape_enable_compaction": ([vp, i32], i32),
+        "grape_step_masked": ([vp, pp, pp, pp, vp, i64, vp], i32),
+        "grape_live_counts": ([vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -162,6 +166,21 @@ def grape_set_refresh_period(ctx: int, period: int):
 
 def grape_sqnorms(ctx: int, A, Gout, step: int, sqnorms_dev, stream=None):
     _check(lib().grape_sqnorms(ctx, _array(A), _array(Gout), step, _ptr(sqnorms_dev), _stream(stream)), ctx)
+
+
+def grape_enable_compaction(ctx: int, T_full: int):
+    _check(lib().grape_enable_compaction(ctx, T_full), ctx)
+
+
+def grape_step_masked(ctx: int, A, Gout, W, mask_dev, step: int, stream=None):
+    _check(lib().grape_step_masked(ctx, _array(A), _array(Gout), _array(W), _ptr(mask_dev), step,
+                                   _stream(stream)), ctx)
+
+
+def grape_live_counts(ctx: int, B: int) -> np.ndarray:
+    out = np.zeros(B, dtype=np.int32)
+    _check(lib().grape_live_counts(ctx, out.ctypes.data), ctx)
+    return out
 
 
 def grape_S_ptr(ctx: int, layer: int) -> int:
@@ -270,6 +289,17 @@ class GrapeStep:
         if getattr(w, "refresh", 1) != 1:
             g.set_refresh_period(w.refresh)
         return g
+
+    def enable_compaction(self, T_full: int):
+        """Inputs of T_full tokens per sample, compacted to this context's T kept tokens."""
+        grape_enable_compaction(self.ctx, T_full)
+
+    def step_masked(self, A, Gout, W, mask, step: int, stream=None):
+        """The step over the tokens ``mask`` (uint8 / bool device tensor, B x T_full) keeps."""
+        grape_step_masked(self.ctx, A, Gout, W, mask, step, stream)
+
+    def live_counts(self) -> np.ndarray:
+        return grape_live_counts(self.ctx, self.B)
 
     def set_refresh_period(self, period: int):
         grape_set_refresh_period(self.ctx, period)
