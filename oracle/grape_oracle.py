@@ -300,6 +300,24 @@ def sample_norms(A: Sequence[np.ndarray], Gout: Sequence[np.ndarray], step_index
 
 
 # --------------------------------------------------------------------------
+# Ghost norm of a projected per-sample gradient
+#
+# The technical summary of "Memory-Efficient Differentially Private Training with
+# Gradient Random Projection" places DP-GRAPE as orthogonal to Ghost Clipping; the
+# DP-SGD-RC summary gives Ghost Clipping's cost as O(B T^2 (p + d)) for a linear
+# layer.  Ghost clipping evaluates ||X^T Y||_F^2 as <X X^T, Y Y^T>_F from two T x T
+# Gram matrices, never forming X^T Y.  For DP-GRAPE, X = A_i P (T x r) and
+# Y = Gout_i (T x d_out).
+# --------------------------------------------------------------------------
+
+def ghost_sqnorm(AP_i: np.ndarray, Gout_i: np.ndarray) -> float:
+    """<(A_i P)(A_i P)^T, Gout_i Gout_i^T>_F, from the two T x T Gram matrices."""
+    X = AP_i @ AP_i.T
+    Y = Gout_i @ Gout_i.T
+    return float(np.sum(X * Y))
+
+
+# --------------------------------------------------------------------------
 # Loss-token masks
 #
 # The pages are silent about masking: a mask is a property of the workload

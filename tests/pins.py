@@ -365,6 +365,33 @@ def pin_refresh_period_two(O):
 
 
 # --------------------------------------------------------------------------
+# ghost norm
+# --------------------------------------------------------------------------
+
+def pin_ghost_norm_equals_projected_norm(O):
+    """<(AP)(AP)^T, G G^T>_F equals ||(AP)^T G||_F^2 computed with loops (the trace identity
+    tr(M^T M) for M = (AP)^T G, here written out element by element)."""
+    rng = np.random.default_rng(41)
+    A, G, P = rng.standard_normal((5, 6)), rng.standard_normal((5, 4)), rng.standard_normal((6, 3))
+    AP = A @ P
+    direct = 0.0
+    for j in range(3):
+        for n in range(4):
+            acc = sum(AP[t, j] * G[t, n] for t in range(5))
+            direct += acc * acc
+    assert math.isclose(O.ghost_sqnorm(AP, G), direct, rel_tol=1e-12)
+
+
+def pin_ghost_norm_with_identity_is_gradient_norm(O):
+    """With P = I the ghost norm is the textbook ghost-clipping norm of the full per-sample
+    gradient: <A A^T, G G^T>_F = ||A^T G||_F^2 of the materialised gradient."""
+    rng = np.random.default_rng(42)
+    A, G = rng.standard_normal((7, 5)), rng.standard_normal((7, 3))
+    full = float(np.sum(O.per_sample_gradient(A, G) ** 2))
+    assert math.isclose(O.ghost_sqnorm(A @ np.eye(5), G), full, rel_tol=1e-12)
+
+
+# --------------------------------------------------------------------------
 # token masks
 # --------------------------------------------------------------------------
 
@@ -450,5 +477,6 @@ ALL_PINS = [
     pin_adam_first_step, pin_no_privacy_reduction, pin_backprojection_unbiased,
     pin_projection_before_privatization, pin_refresh_fixed_subspace, pin_refresh_period_two,
     pin_hutchinson_identity_sketch, pin_hutchinson_unbiased, pin_hutchinson_factored,
-    pin_masked_tokens_drop_out,
+    pin_masked_tokens_drop_out, pin_ghost_norm_equals_projected_norm,
+    pin_ghost_norm_with_identity_is_gradient_norm,
 ]

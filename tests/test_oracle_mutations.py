@@ -79,6 +79,10 @@ MUTATIONS = {
     # Hutchinson estimate
     "hutch_wrong_gram": ("O = G @ G.T", "O = G @ G.T + np.eye(G.shape[0])"),
     "hutch_first_column": ("for j in range(P.shape[1])))", "for j in range(1)))"),
+    # ghost norm
+    "ghost_wrong_gram_side": ("X = AP_i @ AP_i.T", "X = AP_i.T @ AP_i"),
+    "ghost_half_gram": ("X = AP_i @ AP_i.T", "X = 0.5 * (AP_i @ AP_i.T)"),
+    "ghost_trace_only": ("return float(np.sum(X * Y))", "return float(np.trace(X) * np.trace(Y))"),
     # token mask
     "mask_inverted": ("keep = (np.asarray(mask) != 0)[:, :, None]", "keep = (np.asarray(mask) == 0)[:, :, None]"),
     "mask_zeroes_nothing": ("return [np.where(keep, g, 0.0) for g in Gout]", "return [g for g in Gout]"),
