@@ -63,6 +63,8 @@ def parse(argv=None):
     ap.add_argument("--workload", default="mlp4x1024", choices=sorted(WL.WORKLOADS))
     ap.add_argument("--mode", default="step", choices=["step", "sqnorms"],
                     help="step: the whole DP-GRAPE step; sqnorms: per-sample norm estimates only")
+    ap.add_argument("--norm", default="direct", choices=["direct", "ghost"],
+                    help="per-sample norms by R_i tiles (direct) or by the ghost Gram identity")
     ap.add_argument("--mask-capacity", type=int, default=0,
                     help="run masked steps (grape_step_masked) keeping at most this many loss "
                          "tokens per sample; the workload's own token mask is passed in")
@@ -329,6 +331,8 @@ def main(argv=None):
     g = GrapeStep.for_workload(w.replace(T=args.mask_capacity) if masked else w, path=path)
     if masked:
         g.enable_compaction(w.T)
+    if args.norm == "ghost":
+        g.set_norm_method(grape.GRAPE_NORM_GHOST)
     path_name = {grape.GRAPE_PATH_SIMT: "simt", grape.GRAPE_PATH_TC: "tc"}[g.path]
     Wd = [torch.from_numpy(x).to(dev) for x in WL.make_weights(w)]
 
@@ -530,7 +534,7 @@ def main(argv=None):
             "config": {"workload": w.name, "layers": layer_summary(w),
                        "r": w.r, "B_per_gpu": w.B, "global_batch": w.B * world, "T": w.T,
                        "path": path_name, "parallelism": f"dp{world}", "mode": args.mode,
-                       "mask_capacity": args.mask_capacity or None,
+                       "mask_capacity": args.mask_capacity or None, "norm": args.norm,
                        "l2": (f"inputs rotate over {n_sets} distinct sets of "
                               f"{set_bytes / 1e6:.0f} MB each (> 126 MB L2)")
                              if set_bytes > L2_BYTES else

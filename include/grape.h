@@ -153,6 +153,21 @@ GRAPE_API int grape_step_masked(grape_ctx* ctx, const void* const* A, const void
                                 float* const* W, const uint8_t* mask_dev, int64_t step, void* stream);
 GRAPE_API int grape_live_counts(grape_ctx* ctx, int32_t* counts_host);
 
+/* How the per-sample squared norms ||R_i||^2 = ||(A_i P)^T Gout_i||_F^2 are formed.
+ *  GRAPE_NORM_DIRECT  R_i tile by tile (r x 256 tiles, K = T), squares summed (default)
+ *  GRAPE_NORM_GHOST   the ghost identity <(A_i P)(A_i P)^T, Gout_i Gout_i^T>_F from two
+ *                     T x T Gram matrices per sample and layer, never forming R_i (Ghost
+ *                     Clipping, which the technical summary of "Memory-Efficient
+ *                     Differentially Private Training with Gradient Random Projection"
+ *                     calls orthogonal to DP-GRAPE; the DP-SGD-RC summary costs it at
+ *                     O(B T^2 (p + d)) per linear layer).  It costs 2 T^2 (r + d_out) flops
+ *                     per sample and layer against 2 T r d_out, so it pays for short T.
+ * Both give the same value up to rounding; the step, grape_sqnorms and clipping use it.
+ * Errors: GRAPE_EINVAL (unknown method); GRAPE_EUNSUPPORTED (ghost needs the
+ * tensor-core path and T <= 128). */
+enum grape_norm_method { GRAPE_NORM_DIRECT = 0, GRAPE_NORM_GHOST = 1 };
+GRAPE_API int grape_set_norm_method(grape_ctx* ctx, int32_t method);
+
 /* Projection-refresh period K >= 1 (default 1).  P_l of step s is drawn with
  * the step field of its Philox counter set to floor(s / K) instead of s, so one
  * random subspace serves K consecutive steps (the refresh schedule is left

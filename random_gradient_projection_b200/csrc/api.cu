@@ -53,6 +53,7 @@ struct grape_ctx {
   // the P now in the scratch (-1: none), so a step with the same key skips generating it
   uint32_t refresh = 1;
   int64_t p_key = -1;
+  int norm_method = GRAPE_NORM_DIRECT;
   // live-token compaction (grape_enable_compaction): inputs of T_full tokens per sample,
   // compacted to the context's T rows; one allocation holds every buffer below
   int T_full = 0;
@@ -177,6 +178,8 @@ int run_project_norm(grape_ctx* ctx, const grape::LayerIo* io, int64_t step, cud
                [&](int* n) { return grape::tc_project(sh, ws, io, tc, st, n, !gen); });
     if (rc) return rc;
     return phase(ctx, GRAPE_PHASE_NORM, "per-sample norms", st, [&](int* n) {
+      if (ctx->norm_method == GRAPE_NORM_GHOST)
+        return grape::tc_project_norm_ghost(sh, ws, io, tc, ctx->partials, st, n);
       return grape::tc_project_norm(sh, ws, io, tc, ctx->partials, st, n);
     });
   }
@@ -596,6 +599,17 @@ int grape_live_counts(grape_ctx* ctx, int32_t* counts_host) {
   e = cudaMemcpy(counts_host, ctx->comp_counts, sizeof(int32_t) * ctx->sh.B, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return ctx->cuda_fail(e, "cudaMemcpy");
   return check_device_error(ctx);
+}
+
+int grape_set_norm_method(grape_ctx* ctx, int32_t method) {
+  if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  if (method != GRAPE_NORM_DIRECT && method != GRAPE_NORM_GHOST)
+    return ctx->fail(GRAPE_EINVAL, "method must be GRAPE_NORM_DIRECT or GRAPE_NORM_GHOST");
+  if (method == GRAPE_NORM_GHOST &&
+      (ctx->path != GRAPE_PATH_TC || !grape::tc_ghost_supported(ctx->sh)))
+    return ctx->fail(GRAPE_EUNSUPPORTED, "the ghost norm runs on the tensor-core path with T <= 128");
+  ctx->norm_method = method;
+  return GRAPE_OK;
 }
 
 int grape_set_refresh_period(grape_ctx* ctx, int32_t period) {

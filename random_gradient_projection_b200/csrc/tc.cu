@@ -73,7 +73,7 @@ constexpr int kMaxGroup = 16;      // layers per launch
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr uint64_t kDrainLimitNs = 1000000000ull;   // after an abort: wait for loads in flight
 
-enum Mode : int { PROJECT = 0, NORM = 1, AGGREGATE = 2, BACKPROJ = 3 };
+enum Mode : int { PROJECT = 0, NORM = 1, AGGREGATE = 2, BACKPROJ = 3, GHOST = 4 };
 
 // error word bits
 constexpr int kErrTimeoutProducer = 1;
@@ -87,7 +87,9 @@ struct GroupLayer {
   int M, N;          // output extent
   int ldo;           // leading dimension of the output
   void* out;         // PROJECT: AP (bf16); AGGREGATE: S; BACKPROJ: W
-  int part_base;     // NORM: first partial slot of this layer
+  int part_base;     // NORM, GHOST: first partial slot of this layer
+  int slots;         // GHOST: partial slots of this layer per sample (the first gets the sum)
+  int kfirst;        // GHOST: k-blocks of Gout, loaded before the k-blocks of AP
 };
 
 struct GroupParams {
@@ -110,10 +112,10 @@ struct ModeTraits {
   static constexpr bool kB3d = (MODE == NORM);
 };
 
-template <int BN, int STAGES, int EXTRA = 0>
+template <int BN, int STAGES, int EXTRA = 0, int BCOLS = BN>
 struct Smem {
   static constexpr int kABytes = kBM * kBK * 2;
-  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kBBytes = BCOLS * kBK * 2;   // 0: one tile per stage serves as A and B
   static constexpr int kStage = kABytes + kBBytes;
   static constexpr int kBarOff = STAGES * kStage;
   // after the barriers, on a 1024-byte boundary (128-byte-swizzled TMA boxes live there)
@@ -131,6 +133,9 @@ template <int MODE>
 struct ModeExtra {
   static constexpr int kBytes = (MODE == BACKPROJ) ? 2 * kWTile : 0;
 };
+// GHOST stages hold a single 128-row tile, used as both operands of its Gram product.
+template <int MODE, int BN, int STAGES>
+using SmemOf = Smem<BN, STAGES, ModeExtra<MODE>::kBytes, MODE == GHOST ? 0 : BN>;
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
@@ -167,9 +172,13 @@ __device__ __forceinline__ TileCoord decode_tile(const GroupParams& p, int tile,
 template <int MODE, int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ GroupParams p) {
   using T = ModeTraits<MODE>;
-  using S = Smem<BN, STAGES, ModeExtra<MODE>::kBytes>;
-  constexpr uint32_t kTmemCols = 2 * BN;
-  constexpr uint32_t kIdesc = ptx::idesc_bf16(kBM, BN, T::kAMn, true);
+  using S = SmemOf<MODE, BN, STAGES>;
+  // GHOST keeps two accumulators per tile (Gout Gout^T and AP AP^T), both K-major products
+  constexpr uint32_t kAccCols = (MODE == GHOST) ? 2 * BN : BN;
+  constexpr uint32_t kTmemCols = 2 * kAccCols;
+  constexpr uint32_t kIdesc = (MODE == GHOST) ? ptx::idesc_bf16(kBM, BN, false, false)
+                                              : ptx::idesc_bf16(kBM, BN, T::kAMn, true);
+  static_assert(MODE != GHOST || BN == kBM, "a Gram tile is 128 x 128");
   static_assert(BN % 128 == 0, "each epilogue warp takes BN/2 columns in 64-column loads");
 
   extern __shared__ uint8_t smem_raw[];
@@ -312,7 +321,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             break;
           }
           ptx::mbar_arrive_expect_tx(&full[s], S::kStage);
-          if (MODE == PROJECT) {
+          if (MODE == GHOST) {
+            // rows 0..127 of the sample (past T: zeros); Gout first, then AP (after the wait)
+            const int kf = p.lay[c.g].kfirst;
+            uint8_t* st_ = smem + s * S::kStage;
+            if (kb < kf) {
+              ptx::tma_load_3d_hint(st_, &p.mapB[c.g], &full[s], kb * kBK, 0, c.s_t, polB);
+            } else {
+              ensure_wait();
+              ptx::tma_load_3d_hint(st_, &p.mapA[c.g], &full[s], (kb - kf) * kBK, 0, c.s_t, polA);
+            }
+          } else if (MODE == PROJECT) {
             load_a(c, kb, s);
             ensure_wait();
             load_b(c, kb, s);
@@ -352,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t d = tmem + b * BN;
+        const uint32_t d = tmem + b * kAccCols;
         for (int kb = c.kb0; kb < c.kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -364,14 +383,28 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
           ptx::tc_fence_after();
           const uint32_t a_base = ptx::smem_u32(smem + s * S::kStage);
           const uint32_t b_base = a_base + S::kABytes;
+          if (MODE == GHOST) {
+            // the stage's tile X (128 rows, 64 K-major columns) as both operands: D += X X^T,
+            // into the Gout Gram (first accumulator) or the AP Gram (second)
+            const int kf = p.lay[c.g].kfirst;
+            const bool second = kb >= kf;
+            const uint32_t dd = d + (second ? BN : 0);
+            const int kstart = second ? kf : c.kb0;
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k) {
-            // K-major: the next 16 elements are 32 bytes further along the swizzled row;
-            // M/N-major: the next 16 K-rows are 16 x 128 bytes further.
-            const uint64_t ad = T::kAMn ? ptx::desc_sw128(a_base + k * 2048, 8192, 1024)
-                                        : ptx::desc_sw128(a_base + k * 32, 16, 1024);
-            const uint64_t bd = ptx::desc_sw128(b_base + k * 2048, 8192, 1024);
-            ptx::umma_bf16(d, ad, bd, kIdesc, (kb > c.kb0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < kBK / 16; ++k) {
+              const uint64_t xd = ptx::desc_sw128(a_base + k * 32, 16, 1024);
+              ptx::umma_bf16(dd, xd, xd, kIdesc, (kb > kstart || k > 0) ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k) {
+              // K-major: the next 16 elements are 32 bytes further along the swizzled row;
+              // M/N-major: the next 16 K-rows are 16 x 128 bytes further.
+              const uint64_t ad = T::kAMn ? ptx::desc_sw128(a_base + k * 2048, 8192, 1024)
+                                          : ptx::desc_sw128(a_base + k * 32, 16, 1024);
+              const uint64_t bd = ptx::desc_sw128(b_base + k * 2048, 8192, 1024);
+              ptx::umma_bf16(d, ad, bd, kIdesc, (kb > c.kb0 || k > 0) ? 1u : 0u);
+            }
           }
           ptx::umma_commit(&empty[s]);
         }
@@ -398,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       const bool got = wait(&accfull[b], use & 1);
       if (!got) atomicOr(p.err, kErrTimeoutEpilogue);
       ptx::tc_fence_after();
-      const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * BN + h * kHalf;
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * kAccCols + h * kHalf;
       const int col0 = c.n_t * BN + h * kHalf;    // first output column of this warp
       const bool have = got && c.kb1 > c.kb0;
 
@@ -437,6 +470,34 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
 #pragma unroll
           for (int k = 0; k < kEpiWarps; ++k) tot += rb[k];
           p.partials[static_cast<size_t>(c.s_t) * p.part_stride + L.part_base + c.m_t * L.nt + c.n_t] = tot;
+        }
+      } else if (MODE == GHOST) {
+        // sum over this warp's 32 rows x 64 columns of (Gout Gram) * (AP Gram)
+        float ss = 0.0f;
+#pragma unroll 1
+        for (int cc = 0; cc < kHalf; cc += 32) {
+          float y[32], x[32];
+          ptx::tmem_ld32(tbase + cc, y);
+          ptx::tmem_ld32(tbase + BN + cc, x);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ss = fmaf(x[j], y[j], ss);
+        }
+        if (!have) ss = 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        float* rb = red + (tc & 1) * kEpiWarps;
+        if (lane == 0) rb[ew] = ss;
+        epi_bar();
+        if (ew == 0) {
+          // the layer's first slot holds the norm, its other slots zero (the clip sums them all)
+          float* slot = p.partials + static_cast<size_t>(c.s_t) * p.part_stride + L.part_base;
+          for (int k = lane; k < L.slots; k += 32) {
+            float tot = 0.0f;
+            if (k == 0)
+#pragma unroll
+              for (int w2 = 0; w2 < kEpiWarps; ++w2) tot += rb[w2];
+            slot[k] = tot;
+          }
         }
       } else if (MODE == AGGREGATE) {
         const int m = c.m_t * kBM + row;
@@ -824,13 +885,13 @@ bool map_2d_f32(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 [B][T][cols] as a 3-D map with a (64 x 64 x 1) box: rows past T read as zero.
-bool map_3d(CUtensorMap* m, const void* ptr, uint64_t B, uint64_t T, uint64_t cols) {
+// bf16 [B][T][cols] as a 3-D map with a (64 x box_rows x 1) box: rows past T read as zero.
+bool map_3d(CUtensorMap* m, const void* ptr, uint64_t B, uint64_t T, uint64_t cols, uint32_t box_rows = 64) {
   auto enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {cols, T, B};
   cuuint64_t strides[2] = {cols * 2, T * cols * 2};
-  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -875,6 +936,7 @@ constexpr int kStagesAgg = 4;          // 4 x 48 KB
 constexpr int kStagesBack = 3;         // 3 x 32 KB stages + 2 x 64 KB W tiles
 constexpr int kBnAggCluster = 128;     // cluster-split aggregation: 6 x 32 KB
 constexpr int kStagesAggCluster = 6;
+constexpr int kStagesGhost = 12;       // 12 x 16 KB: one 128-row tile per stage
 
 struct HostState {
   int L = 0, r = 0, B = 0, T = 0;
@@ -883,10 +945,11 @@ struct HostState {
   std::vector<CUtensorMap> mapP_mn;     // P16 as the MN-major B operand of PROJECT
   std::vector<CUtensorMap> mapP_k;      // P16 as the K-major A operand of BACKPROJ
   std::vector<CUtensorMap> mapAP3;      // AP as [B][T][r] (NORM A operand)
+  std::vector<CUtensorMap> mapAP3k;     // AP as [B][T][r], 128-row boxes (GHOST, T <= 128)
   std::vector<CUtensorMap> mapAP2;      // AP as [B*T][r] (AGGREGATE A operand)
   std::vector<CUtensorMap> mapDR;       // dR as [r][d_out] (BACKPROJ B operand)
   // per-step maps, cached by pointer
-  std::vector<MapCache> cacheA, cacheG3, cacheG2, cacheW;
+  std::vector<MapCache> cacheA, cacheG3, cacheG2, cacheW, cacheG3k;
   int* err = nullptr;
   int bn_project = 128;
   GroupParams gp;   // host staging of one launch's kernel parameters
@@ -935,7 +998,7 @@ int sm_count() {
 // would run its surplus CTAs as a second wave behind the first.
 template <int MODE, int BN, int STAGES>
 cudaError_t launch_group(GroupParams& gp, int tiles, cudaStream_t st, bool pdl = true) {
-  using S = Smem<BN, STAGES, ModeExtra<MODE>::kBytes>;
+  using S = SmemOf<MODE, BN, STAGES>;
   static int per_sm = 0;
   if (per_sm == 0) {
     cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<MODE, BN, STAGES>,
@@ -1033,10 +1096,12 @@ cudaError_t tc_init(const StepShape& sh, const LayerWs* ws, void* scratch, size_
   hs->mapP_mn.resize(sh.L);
   hs->mapP_k.resize(sh.L);
   hs->mapAP3.resize(sh.L);
+  hs->mapAP3k.resize(sh.L);
   hs->mapAP2.resize(sh.L);
   hs->mapDR.resize(sh.L);
   hs->cacheA.resize(sh.L);
   hs->cacheG3.resize(sh.L);
+  hs->cacheG3k.resize(sh.L);
   hs->cacheG2.resize(sh.L);
   hs->cacheW.resize(sh.L);
   const uint64_t rows = static_cast<uint64_t>(sh.B) * sh.T;
@@ -1046,6 +1111,7 @@ cudaError_t tc_init(const StepShape& sh, const LayerWs* ws, void* scratch, size_
     bool ok = map_2d(&hs->mapP_mn[l], ws[l].P16, ws[l].d_in, sh.r, 64, 64) &&
               map_2d(&hs->mapP_k[l], ws[l].P16, ws[l].d_in, sh.r, 64, kBM) &&
               map_3d(&hs->mapAP3[l], ws[l].AP, sh.B, sh.T, sh.r) &&
+              (sh.T > kBM || map_3d(&hs->mapAP3k[l], ws[l].AP, sh.B, sh.T, sh.r, kBM)) &&
               map_2d(&hs->mapAP2[l], ws[l].AP, rows, sh.r, 64, 64) &&
               map_2d(&hs->mapDR[l], ws[l].dR, sh.r, ws[l].d_out, 64, 64);
     if (!ok) {
@@ -1147,6 +1213,41 @@ cudaError_t tc_project_norm(const StepShape& sh, const LayerWs* ws, const LayerI
     return true;
   };
   return run_mode<NORM, kBnWide, kStagesNorm>(hs, sh.L, st, launches, fill, gp);
+}
+
+bool tc_ghost_supported(const StepShape& sh) { return sh.T <= kBM; }
+
+// Per-sample squared norms by the ghost identity ||(A_i P)^T Gout_i||^2 =
+// <(A_i P)(A_i P)^T, Gout_i Gout_i^T>_F: one 128 x 128 Gram tile pair per (sample, layer).
+cudaError_t tc_project_norm_ghost(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
+                                  const TcWorkspace& tc, float* partials, cudaStream_t st, int* launches) {
+  if (sh.T > kBM) return cudaErrorInvalidValue;
+  HostState& hs = *static_cast<HostState*>(tc.host_state);
+  GroupParams& gp = hs.gp;
+  std::memset(&gp, 0, sizeof(gp));
+  gp.err = hs.err;
+  gp.partials = partials;
+  gp.part_stride = sh.part_stride;
+  auto fill = [&](int g, int l, int* tiles) {
+    gp.mapA[g] = hs.mapAP3k[l];
+    if (!hs.cacheG3k[l].get(io[l].G, &gp.mapB[g], [&](CUtensorMap* m) {
+          return map_3d(m, io[l].G, sh.B, sh.T, ws[l].d_out, kBM);
+        }))
+      return false;
+    GroupLayer& L = gp.lay[g];
+    L.mt = 1;
+    L.nt = 1;
+    L.ns = sh.B;
+    L.kfirst = cdiv(ws[l].d_out, kBK);
+    L.kblocks = L.kfirst + cdiv(sh.r, kBK);
+    L.M = sh.T;
+    L.N = sh.T;
+    L.part_base = ws[l].part_base;
+    L.slots = tc_partials_per_sample(sh.r, ws[l].d_out);
+    *tiles = sh.B;
+    return true;
+  };
+  return run_mode<GHOST, kBM, kStagesGhost>(hs, sh.L, st, launches, fill, gp);
 }
 
 cudaError_t tc_clip_scale(const StepShape& sh, const LayerWs* ws, const TcWorkspace&,

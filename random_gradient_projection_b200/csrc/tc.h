@@ -32,6 +32,11 @@ cudaError_t tc_generate_P(const StepShape& sh, const LayerWs* ws, const TcWorksp
 // so the projection is the step's first kernel and is launched as an ordinary launch.
 cudaError_t tc_project(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                        const TcWorkspace& tc, cudaStream_t st, int* launches, bool first_in_step);
+// The same partials by the ghost identity (two T x T Gram matrices per sample and layer);
+// needs T <= 128 (tc_ghost_supported).
+bool tc_ghost_supported(const StepShape& sh);
+cudaError_t tc_project_norm_ghost(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
+                                  const TcWorkspace& tc, float* partials, cudaStream_t st, int* launches);
 cudaError_t tc_project_norm(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                             const TcWorkspace& tc, float* partials, cudaStream_t st, int* launches);
 cudaError_t tc_clip_scale(const StepShape& sh, const LayerWs* ws, const TcWorkspace& tc,

@@ -30,8 +30,9 @@ EXPORTS = (
     "grape_path_of", "grape_last_error", "grape_global_error", "grape_destroy",
     "grape_philox_words", "grape_gaussian", "grape_profile", "grape_profile_read",
     "grape_launch_count", "grape_layer_sqnorms_static", "grape_set_refresh_period", "grape_sqnorms",
-    "grape_enable_compaction", "grape_step_masked", "grape_live_counts",
+    "grape_enable_compaction", "grape_step_masked", "grape_live_counts", "grape_set_norm_method",
 )
+GRAPE_NORM_DIRECT, GRAPE_NORM_GHOST = 0, 1
 PHASES = ("gen_P", "project", "norm", "clip", "aggregate", "adam", "backproject", "compact")   # GRAPE_N_PHASES
 
 
@@ -83,6 +84,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "grape_enable_compaction": ([vp, i32], i32),
         "grape_step_masked": ([vp, pp, pp, pp, vp, i64, vp], i32),
         "grape_live_counts": ([vp, vp], i32),
+        "grape_set_norm_method": ([vp, i32], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -166,6 +168,10 @@ def grape_set_refresh_period(ctx: int, period: int):
 
 def grape_sqnorms(ctx: int, A, Gout, step: int, sqnorms_dev, stream=None):
     _check(lib().grape_sqnorms(ctx, _array(A), _array(Gout), step, _ptr(sqnorms_dev), _stream(stream)), ctx)
+
+
+def grape_set_norm_method(ctx: int, method: int):
+    _check(lib().grape_set_norm_method(ctx, method), ctx)
 
 
 def grape_enable_compaction(ctx: int, T_full: int):
@@ -289,6 +295,10 @@ class GrapeStep:
         if getattr(w, "refresh", 1) != 1:
             g.set_refresh_period(w.refresh)
         return g
+
+    def set_norm_method(self, method: int):
+        """GRAPE_NORM_DIRECT (default) or GRAPE_NORM_GHOST (tensor-core path, T <= 128)."""
+        grape_set_norm_method(self.ctx, method)
 
     def enable_compaction(self, T_full: int):
         """Inputs of T_full tokens per sample, compacted to this context's T kept tokens."""
