@@ -63,6 +63,9 @@ def parse(argv=None):
     ap.add_argument("--workload", default="mlp4x1024", choices=sorted(WL.WORKLOADS))
     ap.add_argument("--mode", default="step", choices=["step", "sqnorms"],
                     help="step: the whole DP-GRAPE step; sqnorms: per-sample norm estimates only")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every kernel of grape_step from the host instead of replaying a "
+                         "CUDA graph of the step (grape_set_graph)")
     ap.add_argument("--norm", default="direct", choices=["direct", "ghost"],
                     help="per-sample norms by R_i tiles (direct) or by the ghost Gram identity")
     ap.add_argument("--mask-capacity", type=int, default=0,
@@ -333,6 +336,8 @@ def main(argv=None):
         g.enable_compaction(w.T)
     if args.norm == "ghost":
         g.set_norm_method(grape.GRAPE_NORM_GHOST)
+    if not args.no_graph:
+        g.set_graph(True)      # grape_step replays one CUDA graph per input set
     path_name = {grape.GRAPE_PATH_SIMT: "simt", grape.GRAPE_PATH_TC: "tc"}[g.path]
     Wd = [torch.from_numpy(x).to(dev) for x in WL.make_weights(w)]
 
@@ -535,6 +540,7 @@ def main(argv=None):
                        "r": w.r, "B_per_gpu": w.B, "global_batch": w.B * world, "T": w.T,
                        "path": path_name, "parallelism": f"dp{world}", "mode": args.mode,
                        "mask_capacity": args.mask_capacity or None, "norm": args.norm,
+                       "cuda_graph": (not args.no_graph) and args.mode == "step" and not masked and world == 1,
                        "l2": (f"inputs rotate over {n_sets} distinct sets of "
                               f"{set_bytes / 1e6:.0f} MB each (> 126 MB L2)")
                              if set_bytes > L2_BYTES else

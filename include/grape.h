@@ -153,6 +153,19 @@ GRAPE_API int grape_step_masked(grape_ctx* ctx, const void* const* A, const void
                                 float* const* W, const uint8_t* mask_dev, int64_t step, void* stream);
 GRAPE_API int grape_live_counts(grape_ctx* ctx, int32_t* counts_host);
 
+/* CUDA-graph replay of grape_step (enable != 0; default off).  The step's launches
+ * are captured once per set of A, Gout and W pointers (the first grape_step with a
+ * set runs as ordinary launches, the second captures it on a library stream), with
+ * their programmatic dependencies, and replayed on the caller's stream (NULL
+ * included); each replay rewrites the arguments that change with the step (P's
+ * Philox key, Adam's step and bias corrections), so a replay computes exactly what
+ * the ordinary launches compute, with one host call instead of one per kernel.  P is
+ * regenerated on every replay (a refresh period then costs one P generation per step).
+ * At most 8 pointer sets are kept (least recently used dropped).  Profiling
+ * (grape_profile) runs the ordinary launches.  Disabling frees every graph.  Only
+ * grape_step replays; the other entry points always launch directly. */
+GRAPE_API int grape_set_graph(grape_ctx* ctx, int32_t enable);
+
 /* How the per-sample squared norms ||R_i||^2 = ||(A_i P)^T Gout_i||_F^2 are formed.
  *  GRAPE_NORM_DIRECT  R_i tile by tile (r x 256 tiles, K = T), squares summed (default)
  *  GRAPE_NORM_GHOST   the ghost identity <(A_i P)(A_i P)^T, Gout_i Gout_i^T>_F from two

@@ -54,6 +54,28 @@ struct grape_ctx {
   uint32_t refresh = 1;
   int64_t p_key = -1;
   int norm_method = GRAPE_NORM_DIRECT;
+  // CUDA-graph replay of grape_step (grape_set_graph): one graph per set of A, Gout, W
+  // pointers; the first step with a set runs as ordinary launches, the second captures
+  struct StepGraph {
+    std::vector<const void*> A, G;
+    std::vector<float*> W;
+    bool captured = false;
+    cudaGraph_t graph = nullptr;
+    cudaGraphExec_t exec = nullptr;
+    cudaGraphNode_t gen_p = nullptr, adam = nullptr;
+    uint64_t launches = 0, used = 0;
+  };
+  bool graph_on = false;
+  std::vector<StepGraph> graphs;
+  uint64_t graph_tick = 0;
+  cudaStream_t capture_stream = nullptr;
+
+  void drop_graph(StepGraph& g) {
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+    if (g.graph) cudaGraphDestroy(g.graph);
+    g.exec = nullptr;
+    g.graph = nullptr;
+  }
   // live-token compaction (grape_enable_compaction): inputs of T_full tokens per sample,
   // compacted to the context's T rows; one allocation holds every buffer below
   int T_full = 0;
@@ -224,7 +246,7 @@ int run_accumulate(grape_ctx* ctx, const void* const* A, const void* const* G, i
   return GRAPE_OK;
 }
 
-int run_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_total, cudaStream_t st) {
+grape::UpdateScalars update_scalars(const grape_ctx* ctx, int64_t step, int64_t batch_total) {
   const int64_t bt = batch_total > 0 ? batch_total : ctx->sh.B;
   const double t = static_cast<double>(step) + 1.0;
   grape::UpdateScalars u{};
@@ -232,6 +254,11 @@ int run_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_total
   u.inv_batch = static_cast<float>(1.0 / static_cast<double>(bt));
   u.inv_bc1 = static_cast<float>(1.0 / (1.0 - std::pow(ctx->beta1, t)));
   u.inv_bc2 = static_cast<float>(1.0 / (1.0 - std::pow(ctx->beta2, t)));
+  return u;
+}
+
+int run_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_total, cudaStream_t st) {
+  const grape::UpdateScalars u = update_scalars(ctx, step, batch_total);
   std::vector<grape::LayerIo> io(ctx->sh.L);
   for (int l = 0; l < ctx->sh.L; ++l) io[l] = grape::LayerIo{nullptr, nullptr, W[l]};
   const bool tc = ctx->path == GRAPE_PATH_TC;
@@ -247,6 +274,104 @@ int run_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_total
     *n = 1;
     return grape::simt_backproject(sh, ws, io.data(), sh.lr, st);
   });
+}
+
+// grape_step through a CUDA graph (see StepGraph).  Capture records the same launches as
+// run_accumulate + run_apply, including their programmatic (PDL) dependencies, on a
+// library stream; every replay rewrites the two step-dependent kernels' arguments (P's
+// Philox key; the step and bias corrections of noise + Adam) and launches the graph on
+// the caller's stream.  P is generated on every replay, so one graph serves any step.
+int step_graph(grape_ctx* ctx, const void* const* A, const void* const* G, float* const* W, int64_t step,
+               cudaStream_t st) {
+  const int L = ctx->sh.L;
+  grape_ctx::StepGraph* hit = nullptr;
+  for (auto& g : ctx->graphs) {
+    bool same = true;
+    for (int l = 0; l < L && same; ++l) same = g.A[l] == A[l] && g.G[l] == G[l] && g.W[l] == W[l];
+    if (same) {
+      hit = &g;
+      break;
+    }
+  }
+  if (!hit) {   // first sight of this pointer set: ordinary launches, remembered for capture
+    if (ctx->graphs.size() >= 8) {
+      size_t lru = 0;
+      for (size_t k = 1; k < ctx->graphs.size(); ++k)
+        if (ctx->graphs[k].used < ctx->graphs[lru].used) lru = k;
+      ctx->drop_graph(ctx->graphs[lru]);
+      ctx->graphs.erase(ctx->graphs.begin() + static_cast<long>(lru));
+    }
+    grape_ctx::StepGraph g;
+    g.A.assign(A, A + L);
+    g.G.assign(G, G + L);
+    g.W.assign(W, W + L);
+    g.used = ++ctx->graph_tick;
+    ctx->graphs.push_back(g);
+    int rc = run_accumulate(ctx, A, G, step, st);
+    return rc ? rc : run_apply(ctx, W, step, 0, st);
+  }
+  hit->used = ++ctx->graph_tick;
+  if (!hit->captured) {
+    if (!ctx->capture_stream) {
+      cudaError_t e = cudaStreamCreateWithFlags(&ctx->capture_stream, cudaStreamNonBlocking);
+      if (e != cudaSuccess) return ctx->cuda_fail(e, "cudaStreamCreate");
+    }
+    const int64_t saved_key = ctx->p_key;
+    const uint64_t l0 = ctx->launches;
+    ctx->p_key = -1;   // the graph always contains the generation of P
+    cudaError_t e = cudaStreamBeginCapture(ctx->capture_stream, cudaStreamCaptureModeThreadLocal);
+    if (e != cudaSuccess) return ctx->cuda_fail(e, "cudaStreamBeginCapture");
+    int rc = run_accumulate(ctx, A, G, step, ctx->capture_stream);
+    if (!rc) rc = run_apply(ctx, W, step, 0, ctx->capture_stream);
+    cudaGraph_t graph = nullptr;
+    e = cudaStreamEndCapture(ctx->capture_stream, &graph);
+    hit->launches = ctx->launches - l0;
+    ctx->launches = l0;           // nothing ran yet
+    ctx->p_key = saved_key;       // nor was P generated
+    if (rc || e != cudaSuccess) {
+      if (graph) cudaGraphDestroy(graph);
+      cudaGetLastError();
+      return rc ? rc : ctx->cuda_fail(e, "cudaStreamEndCapture");
+    }
+    e = cudaGraphInstantiate(&hit->exec, graph, 0);
+    if (e != cudaSuccess) {
+      cudaGraphDestroy(graph);
+      return ctx->cuda_fail(e, "cudaGraphInstantiate");
+    }
+    hit->graph = graph;
+    size_t n = 0;
+    cudaGraphGetNodes(graph, nullptr, &n);
+    std::vector<cudaGraphNode_t> nodes(n);
+    cudaGraphGetNodes(graph, nodes.data(), &n);
+    const void* gen_fn = ctx->path == GRAPE_PATH_TC ? grape::tc_gen_P_func() : grape::simt_generate_P_func();
+    for (cudaGraphNode_t nd : nodes) {
+      cudaGraphNodeType ty;
+      if (cudaGraphNodeGetType(nd, &ty) != cudaSuccess || ty != cudaGraphNodeTypeKernel) continue;
+      cudaKernelNodeParams kp{};
+      if (cudaGraphKernelNodeGetParams(nd, &kp) != cudaSuccess) continue;
+      if (kp.func == gen_fn) hit->gen_p = nd;
+      if (kp.func == grape::noise_adam_func()) hit->adam = nd;
+    }
+    if (!hit->gen_p || !hit->adam) {
+      ctx->drop_graph(*hit);
+      return ctx->fail(GRAPE_ECUDA, "captured step graph lacks its P-generation or Adam node");
+    }
+    hit->captured = true;
+  }
+  const uint32_t key = static_cast<uint32_t>(step) / ctx->refresh;
+  const grape::StepShape& sh = ctx->sh;
+  cudaError_t e = ctx->path == GRAPE_PATH_TC
+                      ? grape::tc_generate_P_set_node(hit->exec, hit->gen_p, sh, ctx->ws.data(), key)
+                      : grape::simt_generate_P_set_node(hit->exec, hit->gen_p, sh, ctx->ws.data(), key);
+  if (e == cudaSuccess)
+    e = grape::noise_adam_set_node(hit->exec, hit->adam, sh, ctx->ws.data(), update_scalars(ctx, step, 0),
+                                   ctx->path == GRAPE_PATH_TC);
+  if (e == cudaSuccess) e = cudaGraphLaunch(hit->exec, st);
+  if (e != cudaSuccess) return ctx->cuda_fail(e, "graph replay");
+  ctx->launches += hit->launches;
+  ctx->p_key = key;
+  ctx->last_step = step;
+  return GRAPE_OK;
 }
 
 // After a device synchronisation: a sample that kept more live tokens than the compact
@@ -438,6 +563,7 @@ int grape_step(grape_ctx* ctx, const void* const* A, const void* const* Gout, fl
   rc = validate_io(ctx, A, Gout, W, true, true);
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (ctx->graph_on && !ctx->prof_on) return step_graph(ctx, A, Gout, W, step, st);
   rc = run_accumulate(ctx, A, Gout, step, st);
   if (rc) return rc;
   return run_apply(ctx, W, step, 0, st);
@@ -601,6 +727,16 @@ int grape_live_counts(grape_ctx* ctx, int32_t* counts_host) {
   return check_device_error(ctx);
 }
 
+int grape_set_graph(grape_ctx* ctx, int32_t enable) {
+  if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  if (!enable) {
+    for (auto& g : ctx->graphs) ctx->drop_graph(g);
+    ctx->graphs.clear();
+  }
+  ctx->graph_on = enable != 0;
+  return GRAPE_OK;
+}
+
 int grape_set_norm_method(grape_ctx* ctx, int32_t method) {
   if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
   if (method != GRAPE_NORM_DIRECT && method != GRAPE_NORM_GHOST)
@@ -608,6 +744,10 @@ int grape_set_norm_method(grape_ctx* ctx, int32_t method) {
   if (method == GRAPE_NORM_GHOST &&
       (ctx->path != GRAPE_PATH_TC || !grape::tc_ghost_supported(ctx->sh)))
     return ctx->fail(GRAPE_EUNSUPPORTED, "the ghost norm runs on the tensor-core path with T <= 128");
+  if (method != ctx->norm_method) {   // captured graphs hold the other norm kernel
+    for (auto& g : ctx->graphs) ctx->drop_graph(g);
+    ctx->graphs.clear();
+  }
   ctx->norm_method = method;
   return GRAPE_OK;
 }
@@ -776,6 +916,8 @@ void grape_destroy(grape_ctx* ctx) {
   for (void* p : ctx->stage_G) cudaFree(p);
   if (ctx->arena) cudaFree(ctx->arena);
   if (ctx->compact_buf) cudaFree(ctx->compact_buf);
+  for (auto& g : ctx->graphs) ctx->drop_graph(g);
+  if (ctx->capture_stream) cudaStreamDestroy(ctx->capture_stream);
   delete ctx;
 }
 

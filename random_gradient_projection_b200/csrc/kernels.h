@@ -56,6 +56,14 @@ cudaError_t simt_project_ap(const StepShape& sh, const LayerWs* ws, const LayerI
                             cudaStream_t st);
 cudaError_t simt_project_norm(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                               float* partials, cudaStream_t st);
+// CUDA-graph replay: the kernels whose arguments change every step, and the rewrite of
+// those arguments in an instantiated graph (node = the node of the captured graph).
+const void* noise_adam_func();
+const void* simt_generate_P_func();
+cudaError_t noise_adam_set_node(cudaGraphExec_t exec, cudaGraphNode_t node, const StepShape& sh,
+                                const LayerWs* ws, const UpdateScalars& u, bool dR_bf16);
+cudaError_t simt_generate_P_set_node(cudaGraphExec_t exec, cudaGraphNode_t node, const StepShape& sh,
+                                     const LayerWs* ws, uint32_t key);
 // Per-sample squared norms: each sample's partial slots summed in a fixed order (no clip).
 cudaError_t sum_partials(const StepShape& sh, const float* partials, float* sqnorms, cudaStream_t st);
 cudaError_t finalize_clip(const StepShape& sh, const float* partials, float* norms, float* clip,

@@ -452,6 +452,39 @@ cudaError_t simt_backproject(const StepShape& sh, const LayerWs* ws, const Layer
   return cudaGetLastError();
 }
 
+// ---- CUDA-graph replay: the step-dependent arguments of captured nodes ----------------
+const void* noise_adam_func() { return reinterpret_cast<const void*>(noise_adam_kernel); }
+const void* simt_generate_P_func() { return reinterpret_cast<const void*>(generate_P_kernel); }
+
+cudaError_t noise_adam_set_node(cudaGraphExec_t exec, cudaGraphNode_t node, const StepShape& sh,
+                                const LayerWs* ws, const UpdateScalars& u, bool dR_bf16) {
+  cudaKernelNodeParams p{};
+  cudaError_t e = cudaGraphKernelNodeGetParams(node, &p);
+  if (e != cudaSuccess) return e;
+  StepShape a0 = sh;
+  LayerTable a1 = make_table(sh, ws, nullptr);
+  UpdateScalars a2 = u;
+  int a3 = dR_bf16 ? 1 : 0;
+  void* args[] = {&a0, &a1, &a2, &a3};
+  p.kernelParams = args;
+  p.extra = nullptr;
+  return cudaGraphExecKernelNodeSetParams(exec, node, &p);
+}
+
+cudaError_t simt_generate_P_set_node(cudaGraphExec_t exec, cudaGraphNode_t node, const StepShape& sh,
+                                     const LayerWs* ws, uint32_t key) {
+  cudaKernelNodeParams p{};
+  cudaError_t e = cudaGraphKernelNodeGetParams(node, &p);
+  if (e != cudaSuccess) return e;
+  StepShape a0 = sh;
+  LayerTable a1 = make_table(sh, ws, nullptr);
+  uint32_t a2 = key;
+  void* args[] = {&a0, &a1, &a2};
+  p.kernelParams = args;
+  p.extra = nullptr;
+  return cudaGraphExecKernelNodeSetParams(exec, node, &p);
+}
+
 cudaError_t launch_philox_words(uint64_t seed, uint32_t layer, uint32_t step, uint32_t stream_id,
                                 int64_t n_blocks, uint32_t* out, cudaStream_t st) {
   const int grid = cdiv(n_blocks, 256) < 1184 ? cdiv(n_blocks, 256) : 1184;

@@ -1157,6 +1157,27 @@ cudaError_t tc_generate_P(const StepShape& sh, const LayerWs* ws, const TcWorksp
   return cudaGetLastError();
 }
 
+const void* tc_gen_P_func() { return reinterpret_cast<const void*>(gen_P_bf16_kernel); }
+
+cudaError_t tc_generate_P_set_node(cudaGraphExec_t exec, cudaGraphNode_t node, const StepShape& sh,
+                                   const LayerWs* ws, uint32_t key) {
+  cudaKernelNodeParams p{};
+  cudaError_t e = cudaGraphKernelNodeGetParams(node, &p);
+  if (e != cudaSuccess) return e;
+  PTable a0{};
+  for (int l = 0; l < sh.L; ++l) {
+    a0.P16[l] = ws[l].P16;
+    a0.d_in[l] = ws[l].d_in;
+  }
+  uint64_t a1 = sh.seed;
+  uint32_t a2 = key;
+  int a3 = sh.r;
+  void* args[] = {&a0, &a1, &a2, &a3};
+  p.kernelParams = args;
+  p.extra = nullptr;
+  return cudaGraphExecKernelNodeSetParams(exec, node, &p);
+}
+
 cudaError_t tc_project(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                        const TcWorkspace& tc, cudaStream_t st, int* launches, bool first_in_step) {
   HostState& hs = *static_cast<HostState*>(tc.host_state);

@@ -25,6 +25,10 @@ void tc_release(TcWorkspace* tc);
 int* tc_error_word(const TcWorkspace& tc);
 // The phases of the tensor-core path; each enqueues on `st`, adds the number of
 // kernels it launched to *launches and returns the first CUDA error.
+// CUDA-graph replay: the P-generation kernel and the rewrite of its key in a graph.
+const void* tc_gen_P_func();
+cudaError_t tc_generate_P_set_node(cudaGraphExec_t exec, cudaGraphNode_t node, const StepShape& sh,
+                                   const LayerWs* ws, uint32_t key);
 // `key` is the step field of P's Philox counter (the step, or step / refresh period).
 cudaError_t tc_generate_P(const StepShape& sh, const LayerWs* ws, const TcWorkspace& tc,
                           uint32_t key, cudaStream_t st, int* launches);

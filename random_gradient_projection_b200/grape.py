@@ -31,6 +31,7 @@ EXPORTS = (
     "grape_philox_words", "grape_gaussian", "grape_profile", "grape_profile_read",
     "grape_launch_count", "grape_layer_sqnorms_static", "grape_set_refresh_period", "grape_sqnorms",
     "grape_enable_compaction", "grape_step_masked", "grape_live_counts", "grape_set_norm_method",
+    "grape_set_graph",
 )
 GRAPE_NORM_DIRECT, GRAPE_NORM_GHOST = 0, 1
 PHASES = ("gen_P", "project", "norm", "clip", "aggregate", "adam", "backproject", "compact")   # GRAPE_N_PHASES
@@ -85,6 +86,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "grape_step_masked": ([vp, pp, pp, pp, vp, i64, vp], i32),
         "grape_live_counts": ([vp, vp], i32),
         "grape_set_norm_method": ([vp, i32], i32),
+        "grape_set_graph": ([vp, i32], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -168,6 +170,10 @@ def grape_set_refresh_period(ctx: int, period: int):
 
 def grape_sqnorms(ctx: int, A, Gout, step: int, sqnorms_dev, stream=None):
     _check(lib().grape_sqnorms(ctx, _array(A), _array(Gout), step, _ptr(sqnorms_dev), _stream(stream)), ctx)
+
+
+def grape_set_graph(ctx: int, enable: bool):
+    _check(lib().grape_set_graph(ctx, 1 if enable else 0), ctx)
 
 
 def grape_set_norm_method(ctx: int, method: int):
@@ -295,6 +301,10 @@ class GrapeStep:
         if getattr(w, "refresh", 1) != 1:
             g.set_refresh_period(w.refresh)
         return g
+
+    def set_graph(self, enable: bool = True):
+        """Replay grape_step through CUDA graphs (one per set of A, Gout, W pointers)."""
+        grape_set_graph(self.ctx, enable)
 
     def set_norm_method(self, method: int):
         """GRAPE_NORM_DIRECT (default) or GRAPE_NORM_GHOST (tensor-core path, T <= 128)."""
