@@ -238,7 +238,8 @@ def oracle_samples_per_s(w, target_s: float, max_steps: int = 1000, sub_batch=No
     h = O.Hyper.of(w)
     st = O.State.init(WL.make_weights(w), w.r)
     done, spent, s = 0, 0.0, 0
-    while spent < target_s and s < max_steps:
+    # a target of 0 s means: exactly max_steps calls (the reference arm's warm-up)
+    while (spent < target_s or target_s <= 0) and s < max_steps:
         x = WL.make_step_inputs(w, s, samples=list(range(nb)), threads=8)
         A = [x.as_f64(a) for a in x.A]
         G = [x.as_f64(g) for g in x.Gout]
@@ -250,7 +251,7 @@ def oracle_samples_per_s(w, target_s: float, max_steps: int = 1000, sub_batch=No
         spent += time.perf_counter() - t0
         done += nb
         s += 1
-    return done / spent, done, spent, threads
+    return (done / spent if spent > 0 else 0.0), done, spent, threads
 
 
 def run_reference(args, rank: int, world: int):

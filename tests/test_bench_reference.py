@@ -1,0 +1,35 @@
+"""bench.py's reference arm (the fp64 oracle on the host cores): the JSON line the driver
+reads, on CPU.  Rank 0 prints one line; other ranks exit 0 without work."""
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _run(args, env_extra=None):
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", *args],
+                         cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    return [l for l in out.stdout.splitlines() if l.startswith("{")]
+
+
+def test_reference_arm_prints_the_contract_line():
+    lines = _run(["--workload", "tiny_f32", "--steps", "2", "--warmup", "1"])
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "samples/s"
+    assert d["steps"] == 2 and d["warmup"] == 1 and d["higher_is_better"] is True
+    for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"):
+        assert k in d["e2e"]
+    for k in ("value", "unit", "cores", "kind", "sample"):
+        assert k in d["cpu_baseline"]
+    assert d["config"]["workload"] == "tiny_f32"
+
+
+def test_reference_arm_other_ranks_do_no_work():
+    assert _run(["--workload", "tiny_f32", "--steps", "1", "--warmup", "1"],
+                {"RANK": "1", "WORLD_SIZE": "2"}) == []
