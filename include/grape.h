@@ -153,6 +153,19 @@ GRAPE_API int grape_step_masked(grape_ctx* ctx, const void* const* A, const void
                                 float* const* W, const uint8_t* mask_dev, int64_t step, void* stream);
 GRAPE_API int grape_live_counts(grape_ctx* ctx, int32_t* counts_host);
 
+/* Self-test of the bounded waits every tensor-core kernel relies on; it faults and
+ * hangs nothing.  One CTA waits on two mbarriers that nothing ever arrives on.  Warp 0
+ * waits at most short_ns and must give up by itself, raising the CTA's abort flag.
+ * Warp 1 waits at most long_ns and must give up early on that flag.  This is the
+ * mechanism that turns a lost TMA load or MMA completion in a step into GRAPE_ETIMEOUT
+ * with the context still usable.  *bits_out (may be NULL) receives 1 when warp 0 gave
+ * up at its limit, plus 2 when warp 1 left on the abort flag (4 instead of 2 if it ran
+ * to its own limit): 3 is the expected result.  Returns GRAPE_ETIMEOUT when warp 0 gave
+ * up (the expected outcome) and GRAPE_OK otherwise.  Synchronises the current device.
+ * Errors: GRAPE_EINVAL (need 0 <= short_ns <= 1e9 and short_ns <= long_ns <= 1e10),
+ * GRAPE_ENOMEM, GRAPE_ECUDA. */
+GRAPE_API int grape_selftest_wait_timeout(int64_t short_ns, int64_t long_ns, int32_t* bits_out);
+
 /* CUDA-graph replay of grape_step (enable != 0; default off).  The step's launches
  * are captured once per set of A, Gout and W pointers (the first grape_step with a
  * set runs as ordinary launches, the second captures it on a library stream), with

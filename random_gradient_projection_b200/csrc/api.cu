@@ -941,6 +941,25 @@ int grape_gaussian(uint64_t seed, uint32_t layer, uint32_t step, uint32_t stream
   return e == cudaSuccess ? GRAPE_OK : set_global(GRAPE_ECUDA, cudaGetErrorString(e));
 }
 
+int grape_selftest_wait_timeout(int64_t short_ns, int64_t long_ns, int32_t* bits_out) {
+  if (short_ns < 0 || short_ns > 1000000000ll || long_ns < short_ns || long_ns > 10000000000ll)
+    return set_global(GRAPE_EINVAL, "need 0 <= short_ns <= 1e9 and short_ns <= long_ns <= 1e10");
+  int* bits = nullptr;
+  cudaError_t e = cudaMalloc(&bits, sizeof(int));
+  if (e != cudaSuccess) return set_global(GRAPE_ENOMEM, cudaGetErrorString(e));
+  e = cudaMemset(bits, 0, sizeof(int));
+  if (e == cudaSuccess)
+    e = grape::tc_selftest_wait(static_cast<uint64_t>(short_ns), static_cast<uint64_t>(long_ns), bits, nullptr);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  int v = 0;
+  if (e == cudaSuccess) e = cudaMemcpy(&v, bits, sizeof(int), cudaMemcpyDeviceToHost);
+  cudaFree(bits);
+  if (e != cudaSuccess) return set_global(GRAPE_ECUDA, cudaGetErrorString(e));
+  if (bits_out) *bits_out = v;
+  if (v & 1) return set_global(GRAPE_ETIMEOUT, "a bounded device wait gave up (self-test)");
+  return GRAPE_OK;
+}
+
 int grape_layer_sqnorms_static(const void* A, const void* Gout, int32_t d_in, int32_t d_out,
                                int32_t r, int32_t B, int32_t T, uint64_t seed, uint32_t layer,
                                uint32_t step, float* sqnorms_out, void* stream) {

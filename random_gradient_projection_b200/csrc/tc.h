@@ -25,6 +25,10 @@ void tc_release(TcWorkspace* tc);
 int* tc_error_word(const TcWorkspace& tc);
 // The phases of the tensor-core path; each enqueues on `st`, adds the number of
 // kernels it launched to *launches and returns the first CUDA error.
+// Self-test of the bounded mbarrier waits (see grape_selftest_wait_timeout): ORs into
+// *bits_dev 1 (warp 0 gave up at its limit), 2 (warp 1 left on the abort flag) or 4
+// (warp 1 ran to its own limit).
+cudaError_t tc_selftest_wait(uint64_t short_ns, uint64_t long_ns, int* bits_dev, cudaStream_t st);
 // CUDA-graph replay: the P-generation kernel and the rewrite of its key in a graph.
 const void* tc_gen_P_func();
 cudaError_t tc_generate_P_set_node(cudaGraphExec_t exec, cudaGraphNode_t node, const StepShape& sh,

@@ -31,7 +31,7 @@ EXPORTS = (
     "grape_philox_words", "grape_gaussian", "grape_profile", "grape_profile_read",
     "grape_launch_count", "grape_layer_sqnorms_static", "grape_set_refresh_period", "grape_sqnorms",
     "grape_enable_compaction", "grape_step_masked", "grape_live_counts", "grape_set_norm_method",
-    "grape_set_graph",
+    "grape_set_graph", "grape_selftest_wait_timeout",
 )
 GRAPE_NORM_DIRECT, GRAPE_NORM_GHOST = 0, 1
 PHASES = ("gen_P", "project", "norm", "clip", "aggregate", "adam", "backproject", "compact")   # GRAPE_N_PHASES
@@ -87,6 +87,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "grape_live_counts": ([vp, vp], i32),
         "grape_set_norm_method": ([vp, i32], i32),
         "grape_set_graph": ([vp, i32], i32),
+        "grape_selftest_wait_timeout": ([i64, i64, ctypes.POINTER(i32)], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -170,6 +171,13 @@ def grape_set_refresh_period(ctx: int, period: int):
 
 def grape_sqnorms(ctx: int, A, Gout, step: int, sqnorms_dev, stream=None):
     _check(lib().grape_sqnorms(ctx, _array(A), _array(Gout), step, _ptr(sqnorms_dev), _stream(stream)), ctx)
+
+
+def grape_selftest_wait_timeout(short_ns: int, long_ns: int):
+    """(status code, bits) of the bounded-wait self-test; GRAPE_ETIMEOUT with bits 3 is correct."""
+    bits = ctypes.c_int32(0)
+    rc = lib().grape_selftest_wait_timeout(short_ns, long_ns, ctypes.byref(bits))
+    return rc, bits.value
 
 
 def grape_set_graph(ctx: int, enable: bool):

@@ -75,3 +75,10 @@ def test_refresh_and_sqnorms_validate_the_handle(lib):
     assert lib.grape_set_refresh_period(None, 2) == 1          # GRAPE_EINVAL
     assert b"ctx" in lib.grape_global_error()
     assert lib.grape_sqnorms(None, None, None, 0, None, None) == 1
+
+
+def test_selftest_validates_its_limits(lib):
+    """Bad limits are refused on the host, before any device work."""
+    assert lib.grape_selftest_wait_timeout(-1, 10, None) == 1          # GRAPE_EINVAL
+    assert lib.grape_selftest_wait_timeout(10, 5, None) == 1
+    assert lib.grape_selftest_wait_timeout(2_000_000_000, 3_000_000_000, None) == 1
