@@ -202,9 +202,15 @@ def step_work(w):
 
 
 def kernel_source_sha(path: str) -> str:
+    """Hash of the kernel source's code: comments and blank lines stripped, so that a
+    comment edit does not orphan counters taken from unchanged code."""
+    import re
     name = "tc.cu" if path == "tc" else "simt.cu"
-    src = os.path.join(ROOT, "random_gradient_projection_b200", "csrc", name)
-    return hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    src = open(os.path.join(ROOT, "random_gradient_projection_b200", "csrc", name)).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    code = "\n".join(l.rstrip() for l in src.splitlines() if l.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def traffic_for(kernel: str, workload: str, path: str, mode: str = "step"):

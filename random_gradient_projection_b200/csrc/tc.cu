@@ -957,10 +957,10 @@ struct HostState {
 
 int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
-// Launch as a programmatic dependent of the previous kernel in the stream (the kernel
-// itself waits with griddepcontrol.wait before it reads that kernel's outputs).
-// A programmatic dependent launch when `pdl`, else an ordinary one (the first kernel of a
-// step is ordinary: it waits for all earlier work, which the early loads rely on).
+// A programmatic dependent launch of `kernel` after the previous kernel in the stream when
+// `pdl` (the kernel itself waits with griddepcontrol.wait before it reads that kernel's
+// outputs), else an ordinary one: the first kernel of a step is ordinary, so it waits for
+// all earlier work, which the early loads of the later kernels rely on.
 template <class Kern, class... Args>
 cudaError_t launch_maybe_pdl(bool pdl, Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                              Args... args) {
