@@ -123,6 +123,11 @@ GRAPE_API int grape_step_host(grape_ctx* ctx, const void* const* A_host, const v
 GRAPE_API int grape_accumulate(grape_ctx* ctx, const void* const* A, const void* const* Gout, int64_t step,
                      void* stream);
 GRAPE_API int grape_S_ptr(grape_ctx* ctx, int32_t layer, float** S_dev);
+/* All S_l at once: they lie back to back in layer order (layer l at element offset
+ * sum_{k<l} r * d_out_k, each r x d_out row-major, no padding), so one all-reduce of
+ * *count fp32 elements from *S_dev sums every layer over the ranks.  Errors:
+ * GRAPE_EINVAL for NULL arguments. */
+GRAPE_API int grape_S_all(grape_ctx* ctx, float** S_dev, int64_t* count);
 GRAPE_API int grape_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_total, void* stream);
 
 /* Live-token compaction for loss-masked inputs.  The pages are silent about

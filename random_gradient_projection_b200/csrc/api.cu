@@ -49,6 +49,7 @@ struct grape_ctx {
   // staging for grape_step_host (allocated on first use)
   std::vector<void*> stage_A, stage_G;
   int64_t last_step = -1;
+  int64_t S_count = 0;   // elements of all S_l together (they are contiguous)
   // projection refresh: P of step s is drawn with key s / refresh; p_key is the key of
   // the P now in the scratch (-1: none), so a step with the same key skips generating it
   uint32_t refresh = 1;
@@ -479,13 +480,21 @@ int grape_create(const grape_layer* layers, int32_t n_layers, int32_t r, double 
   std::vector<Offs> offs(n_layers);
   int part = 0;
   ctx->ws.resize(n_layers);
+  // every S_l back to back in one block (layer order, no padding), so a data-parallel
+  // caller can sum them over ranks with a single all-reduce (grape_S_all)
+  size_t s_total = 0;
+  for (int l = 0; l < n_layers; ++l) s_total += static_cast<size_t>(r) * layers[l].d_out;
+  const size_t off_s_all = ar.take(s_total * 4);
+  ctx->S_count = static_cast<int64_t>(s_total);
+  size_t s_at = off_s_all;
   for (int l = 0; l < n_layers; ++l) {
     const size_t di = layers[l].d_in, dout = layers[l].d_out;
     Offs& o = offs[l];
     o.P32 = tc ? SIZE_MAX : ar.take(di * r * 4);
     o.P16 = tc ? ar.take(di * r * 2) : SIZE_MAX;
     o.AP = ar.take(static_cast<size_t>(B) * T * r * ap_el);
-    o.S = ar.take(r * dout * 4);
+    o.S = s_at;
+    s_at += r * dout * 4;
     o.m = ar.take(r * dout * 4);
     o.v = ar.take(r * dout * 4);
     o.dR = ar.take(r * dout * (tc ? 2 : 4));
@@ -629,6 +638,13 @@ int grape_S_ptr(grape_ctx* ctx, int32_t layer, float** S_dev) {
   if (!ctx || !S_dev) return set_global(GRAPE_EINVAL, "ctx and S_dev must not be null");
   if (layer < 0 || layer >= ctx->sh.L) return ctx->fail(GRAPE_EINVAL, "layer out of range");
   *S_dev = ctx->ws[layer].S;
+  return GRAPE_OK;
+}
+
+int grape_S_all(grape_ctx* ctx, float** S_dev, int64_t* count) {
+  if (!ctx || !S_dev || !count) return set_global(GRAPE_EINVAL, "ctx, S_dev and count must not be null");
+  *S_dev = ctx->ws[0].S;
+  *count = ctx->S_count;
   return GRAPE_OK;
 }
 

@@ -17,6 +17,10 @@ def dp_step(g, A, Gout, W, step: int, group=None, stream=None):
     world = dist.get_world_size(group)
     g.accumulate(A, Gout, step, stream)
     if world > 1:
-        for l in range(len(g.layers)):
-            dist.all_reduce(g.S_tensor(l), op=dist.ReduceOp.SUM, group=group)
+        if hasattr(g, "S_all_tensor"):
+            # every S_l lies back to back: one all-reduce for the whole step
+            dist.all_reduce(g.S_all_tensor(), op=dist.ReduceOp.SUM, group=group)
+        else:
+            for l in range(len(g.layers)):
+                dist.all_reduce(g.S_tensor(l), op=dist.ReduceOp.SUM, group=group)
     g.apply(W, step, g.B * world, stream)

@@ -31,7 +31,7 @@ EXPORTS = (
     "grape_philox_words", "grape_gaussian", "grape_profile", "grape_profile_read",
     "grape_launch_count", "grape_layer_sqnorms_static", "grape_set_refresh_period", "grape_sqnorms",
     "grape_enable_compaction", "grape_step_masked", "grape_live_counts", "grape_set_norm_method",
-    "grape_set_graph", "grape_selftest_wait_timeout",
+    "grape_set_graph", "grape_selftest_wait_timeout", "grape_S_all",
 )
 GRAPE_NORM_DIRECT, GRAPE_NORM_GHOST = 0, 1
 PHASES = ("gen_P", "project", "norm", "clip", "aggregate", "adam", "backproject", "compact")   # GRAPE_N_PHASES
@@ -88,6 +88,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "grape_set_norm_method": ([vp, i32], i32),
         "grape_set_graph": ([vp, i32], i32),
         "grape_selftest_wait_timeout": ([i64, i64, ctypes.POINTER(i32)], i32),
+        "grape_S_all": ([vp, ctypes.POINTER(vp), ctypes.POINTER(i64)], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -201,6 +202,13 @@ def grape_live_counts(ctx: int, B: int) -> np.ndarray:
     out = np.zeros(B, dtype=np.int32)
     _check(lib().grape_live_counts(ctx, out.ctypes.data), ctx)
     return out
+
+
+def grape_S_all(ctx: int):
+    """(device address, element count) of all S_l, back to back in layer order."""
+    ptr, n = ctypes.c_void_p(), ctypes.c_int64()
+    _check(lib().grape_S_all(ctx, ctypes.byref(ptr), ctypes.byref(n)), ctx)
+    return ptr.value, n.value
 
 
 def grape_S_ptr(ctx: int, layer: int) -> int:
@@ -391,6 +399,13 @@ class GrapeStep:
         import torch
         ptr = grape_S_ptr(self.ctx, layer)
         return torch.as_tensor(_DeviceArray(ptr, (self.r, self.layers[layer][1])), device="cuda")
+
+    def S_all_tensor(self):
+        """Every S_l as one flat torch tensor sharing the library's memory (layer order):
+        one all-reduce sums all layers over the ranks."""
+        import torch
+        ptr, n = grape_S_all(self.ctx)
+        return torch.as_tensor(_DeviceArray(ptr, (n,)), device="cuda")
 
     def get_state(self, layer: int, m, v, stream=None):
         grape_get_state(self.ctx, layer, m, v, stream)

@@ -1,7 +1,7 @@
 """Data-parallel orchestration on two gloo ranks (CPU, no GPU).
 
 dp_step (random_gradient_projection_b200/data_parallel.py) runs, on every rank,
-accumulate -> all-reduce of every S_l -> apply(batch_total = B * world).  Here each
+accumulate -> one all-reduce of all S_l (back to back) -> apply(batch_total = B * world).  Here each
 rank drives a stand-in context that computes its shard with the fp64 oracle, so the
 test checks the orchestration itself: which tensors are reduced, in which order, and
 the global batch used for the average.  Two ranks of 3 samples each must reproduce the
@@ -42,11 +42,19 @@ class OracleShard:
         norms = [np.sqrt(sum(np.sum(R[i][l] ** 2) for l in range(len(Ps)))) for i in range(self.B)]
         c = [O.clip_factor(n, self.h.C) for n in norms]
         self.P = Ps
-        self.S = [torch.from_numpy(sum(c[i] * R[i][l] for i in range(self.B)).copy())
-                  for l in range(len(Ps))]
+        # like the library: every S_l a view into one flat buffer, in layer order
+        parts = [sum(c[i] * R[i][l] for i in range(self.B)) for l in range(len(Ps))]
+        self.S_flat = torch.from_numpy(np.concatenate([p.reshape(-1) for p in parts]))
+        self.S, at = [], 0
+        for p_ in parts:
+            self.S.append(self.S_flat[at:at + p_.size].view(p_.shape))
+            at += p_.size
 
     def S_tensor(self, l):
         return self.S[l]
+
+    def S_all_tensor(self):
+        return self.S_flat
 
     def apply(self, Wt, step, batch_total, stream=None):
         t = step + 1

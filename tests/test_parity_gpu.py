@@ -268,3 +268,23 @@ def test_allocation_failure_is_reported(monkeypatch):
     with pytest.raises(GrapeError) as e:
         GrapeStep.for_workload(W.get("tiny_f32"))
     assert e.value.code == grape.GRAPE_ENOMEM
+
+
+@pytest.mark.parametrize("path", [SIMT, TC])
+def test_S_all_is_every_layer_back_to_back(path):
+    w = W.scaled(W.get("mlp4x1024"), layers=((1024, 1024), (1024, 512 * 2), (768, 2304)), B=2, T=32)
+    if path == SIMT:
+        w = w.replace(layers=((24, 16), (16, 12), (12, 20)), r=8, dtype="f32")
+    g = GrapeStep.for_workload(w, path=path)
+    Ws = [torch.from_numpy(x).cuda() for x in W.make_weights(w)]
+    x = W.make_step_inputs(w, 0, threads=8)
+    g.accumulate([to_device(a, w.dtype) for a in x.A], [to_device(a, w.dtype) for a in x.Gout], 0)
+    torch.cuda.synchronize()
+    flat = g.S_all_tensor().cpu().numpy()
+    at = 0
+    for l, (_, do) in enumerate(w.layers):
+        n = w.r * do
+        assert np.array_equal(flat[at:at + n].reshape(w.r, do), g.S(l)), l
+        at += n
+    assert at == flat.size
+    g.close()
