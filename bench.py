@@ -504,6 +504,18 @@ def main(argv=None):
                 g.sqnorms(dA, dG, s, out=sq_out)
                 norms.copy_(sq_out, non_blocking=True)
                 torch.cuda.current_stream().synchronize()
+        elif world > 1:
+            # the data-parallel step: this rank's inputs copied in, dp_step (with its
+            # all-reduce), the norms read back
+            dA, dG, _ = sets[0]
+
+            def e2e_one(s):
+                for d, h_ in zip(dA, hostA):
+                    d.view(torch.int16 if w.dtype == "bf16" else d.dtype).copy_(h_, non_blocking=True)
+                for d, h_ in zip(dG, hostG):
+                    d.view(torch.int16 if w.dtype == "bf16" else d.dtype).copy_(h_, non_blocking=True)
+                dp_step(g, dA, dG, Wd, s)
+                g.norms()                          # synchronises and reads the B norms back
         else:
             def e2e_one(s):
                 g.step_host(hostA, hostG, Wd, s, norms)   # synchronises its stream
@@ -524,6 +536,9 @@ def main(argv=None):
                "steps": args.e2e_steps,
                "note": ("pinned host A/Gout and the token mask copied in, grape_step_masked, the B "
                         "norms copied out, every step") if masked else
+                       ("pinned host A/Gout copied in on every rank, dp_step (accumulate, one "
+                        "all-reduce of S, apply), the B norms copied out, every step")
+                       if world > 1 and args.mode == "step" else
                        ("grape_step_host: pinned host A/Gout copied in, per-sample norms copied out, "
                         "every step") if args.mode == "step" else
                        ("pinned host A/Gout copied in, grape_sqnorms, the B estimates copied out, "
