@@ -201,12 +201,16 @@ def step_work(w):
     return flops, byts
 
 
+KERNEL_SOURCES = {"tc": ("tc.cu", "tc_ptx.cuh", "philox.cuh"), "simt": ("simt.cu", "philox.cuh")}
+
+
 def kernel_source_sha(path: str) -> str:
-    """Hash of the kernel source's code: comments and blank lines stripped, so that a
-    comment edit does not orphan counters taken from unchanged code."""
+    """Hash of the kernel sources' code (the path's .cu file and the device headers it
+    includes): comments and blank lines stripped, so that a comment edit does not orphan
+    counters taken from unchanged code."""
     import re
-    name = "tc.cu" if path == "tc" else "simt.cu"
-    src = open(os.path.join(ROOT, "random_gradient_projection_b200", "csrc", name)).read()
+    csrc = os.path.join(ROOT, "random_gradient_projection_b200", "csrc")
+    src = "\n".join(open(os.path.join(csrc, n)).read() for n in KERNEL_SOURCES[path])
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     src = re.sub(r"//[^\n]*", "", src)
     code = "\n".join(l.rstrip() for l in src.splitlines() if l.strip())

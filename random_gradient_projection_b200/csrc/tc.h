@@ -23,8 +23,6 @@ cudaError_t tc_init(const StepShape& sh, const LayerWs* ws, void* scratch, size_
 void tc_release(TcWorkspace* tc);
 // Device word where the tensor-core kernels record bounded waits that gave up (0 = none).
 int* tc_error_word(const TcWorkspace& tc);
-// The phases of the tensor-core path; each enqueues on `st`, adds the number of
-// kernels it launched to *launches and returns the first CUDA error.
 // Self-test of the bounded mbarrier waits (see grape_selftest_wait_timeout): ORs into
 // *bits_dev 1 (warp 0 gave up at its limit), 2 (warp 1 left on the abort flag) or 4
 // (warp 1 ran to its own limit).
@@ -33,6 +31,8 @@ cudaError_t tc_selftest_wait(uint64_t short_ns, uint64_t long_ns, int* bits_dev,
 const void* tc_gen_P_func();
 cudaError_t tc_generate_P_set_node(cudaGraphExec_t exec, cudaGraphNode_t node, const StepShape& sh,
                                    const LayerWs* ws, uint32_t key);
+// The phases of the tensor-core path; each enqueues on `st`, adds the number of
+// kernels it launched to *launches and returns the first CUDA error.
 // `key` is the step field of P's Philox counter (the step, or step / refresh period).
 cudaError_t tc_generate_P(const StepShape& sh, const LayerWs* ws, const TcWorkspace& tc,
                           uint32_t key, cudaStream_t st, int* launches);
