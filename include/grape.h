@@ -128,6 +128,10 @@ GRAPE_API int grape_S_ptr(grape_ctx* ctx, int32_t layer, float** S_dev);
  * *count fp32 elements from *S_dev sums every layer over the ranks.  Errors:
  * GRAPE_EINVAL for NULL arguments. */
 GRAPE_API int grape_S_all(grape_ctx* ctx, float** S_dev, int64_t* count);
+/* grape_apply(step) back-projects with the P of step's key (step / refresh period),
+ * which must be the P the last grape_accumulate used and still the one in the scratch:
+ * GRAPE_EINVAL when no accumulation ran, when the last one drew another key, or when
+ * a later call (grape_sqnorms of another key, grape_set_refresh_period) replaced P. */
 GRAPE_API int grape_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_total, void* stream);
 
 /* Live-token compaction for loss-masked inputs.  The pages are silent about

@@ -591,15 +591,18 @@ int grape_step_host(grape_ctx* ctx, const void* const* A_host, const void* const
   const size_t el = in_elsize(ctx->sh.dtype);
   const size_t rows = static_cast<size_t>(ctx->sh.B) * ctx->sh.T;
   if (ctx->stage_A.empty()) {
-    ctx->stage_A.assign(ctx->sh.L, nullptr);
-    ctx->stage_G.assign(ctx->sh.L, nullptr);
+    std::vector<void*> sa(ctx->sh.L, nullptr), sg(ctx->sh.L, nullptr);
     for (int l = 0; l < ctx->sh.L; ++l) {
-      if (cudaMalloc(&ctx->stage_A[l], rows * ctx->layers[l].d_in * el) != cudaSuccess ||
-          cudaMalloc(&ctx->stage_G[l], rows * ctx->layers[l].d_out * el) != cudaSuccess) {
+      if (cudaMalloc(&sa[l], rows * ctx->layers[l].d_in * el) != cudaSuccess ||
+          cudaMalloc(&sg[l], rows * ctx->layers[l].d_out * el) != cudaSuccess) {
         cudaGetLastError();
+        for (void* p : sa) cudaFree(p);   // cudaFree(nullptr) is a no-op
+        for (void* p : sg) cudaFree(p);
         return ctx->fail(GRAPE_ENOMEM, "staging allocation for grape_step_host failed");
       }
     }
+    ctx->stage_A = sa;   // kept only when every layer's staging exists
+    ctx->stage_G = sg;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   for (int l = 0; l < ctx->sh.L; ++l) {
@@ -655,6 +658,14 @@ int grape_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_tot
   if (batch_total < 0) return ctx->fail(GRAPE_EINVAL, "batch_total must be >= 0");
   rc = validate_io(ctx, nullptr, nullptr, W, false, true);
   if (rc) return rc;
+  // S lies in the span of the P its aggregation used, so the back-projection must use
+  // that P: the last accumulation drew it with this step's key, and no later call
+  // (grape_sqnorms, a refresh-period change) has replaced it in the scratch since.
+  const int64_t key = static_cast<uint32_t>(step) / ctx->refresh;
+  if (ctx->last_step < 0 || static_cast<uint32_t>(ctx->last_step) / ctx->refresh != key || ctx->p_key != key)
+    return ctx->fail(GRAPE_EINVAL, "grape_apply(step " + std::to_string(step) +
+                                       ") needs a grape_accumulate of a step with the same projection"
+                                       " (key step / refresh period) as the last call that drew P");
   return run_apply(ctx, W, step, batch_total, static_cast<cudaStream_t>(stream));
 }
 

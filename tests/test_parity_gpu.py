@@ -180,6 +180,36 @@ def test_accumulate_apply_equals_step(path):
 
 
 @pytest.mark.parametrize("path", [SIMT, TC], ids=["simt", "tc"])
+def test_apply_needs_the_accumulated_projection(path):
+    """apply(s) back-projects with the P the aggregation of S used: it is refused before
+    any accumulation, for a step of another key, and after sqnorms replaced P; W is left
+    untouched by a refused call, and a step of the same refresh key is accepted."""
+    w = W.scaled(W.get("mlp4x1024"), n_layers=2, B=3, T=32)
+    g = GrapeStep.for_workload(w, path=path)
+    Wd = [torch.from_numpy(x).cuda() for x in W.make_weights(w)]
+    before = [x.clone() for x in Wd]
+    A, G = _inputs(w, 0)
+    with pytest.raises(GrapeError) as e:
+        g.apply(Wd, 0)
+    assert e.value.code == grape.GRAPE_EINVAL
+    g.accumulate(A, G, 0)
+    with pytest.raises(GrapeError):
+        g.apply(Wd, 1)
+    g.sqnorms(A, G, 1)                       # draws P of step 1 into the scratch
+    with pytest.raises(GrapeError):
+        g.apply(Wd, 0)
+    torch.cuda.synchronize()
+    assert all(torch.equal(a, b) for a, b in zip(Wd, before))
+    g.accumulate(A, G, 0)
+    g.apply(Wd, 0)                           # the matching pair runs
+    g.set_refresh_period(2)
+    g.accumulate(A, G, 2)
+    g.apply(Wd, 3)                           # 2 // 2 == 3 // 2: the same P
+    torch.cuda.synchronize()
+    g.close()
+
+
+@pytest.mark.parametrize("path", [SIMT, TC], ids=["simt", "tc"])
 def test_step_host_equals_step(path):
     w = W.scaled(W.get("mlp4x1024"), n_layers=2, B=3, T=32)
     W0 = W.make_weights(w)
