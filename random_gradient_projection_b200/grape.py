@@ -289,6 +289,28 @@ def grape_gaussian(seed: int, layer: int, step: int, stream_id: int, n: int, out
                                 _stream(stream)))
 
 
+# ---- buffer checks of the context owner below ---------------------------------
+
+def _need(x, nbytes: int, el: int, what: str, cuda: Optional[bool]):
+    """Refuse a torch tensor or numpy array that cannot serve as `nbytes` contiguous bytes
+    of `el`-byte elements from its start, or that lies on the wrong side of the host /
+    device split (cuda None: either side).  The kernels read and write whole buffers
+    from plain addresses, so a short or strided buffer would be accessed out of bounds.
+    Raw integer addresses pass unchecked."""
+    if x is None or isinstance(x, int):
+        return
+    if isinstance(x, np.ndarray):
+        ok = (x.flags.c_contiguous and x.itemsize == el and x.nbytes >= nbytes and cuda is not True)
+    else:
+        ok = (x.is_contiguous() and x.element_size() == el and x.numel() * el >= nbytes
+              and (cuda is None or x.is_cuda == cuda))
+    if not ok:
+        where = {True: "a CUDA", False: "a host", None: "a"}[cuda]
+        raise ValueError(f"{what}: need {where} contiguous buffer of at least {nbytes} bytes of "
+                         f"{el}-byte elements, got {getattr(x, 'shape', None)} "
+                         f"{getattr(x, 'dtype', type(x).__name__)}")
+
+
 # ---- a context owner for torch tensors ---------------------------------------
 
 class _DeviceArray:
@@ -307,8 +329,24 @@ class GrapeStep:
         self.layers = [tuple(int(x) for x in l) for l in layers]
         self.r, self.B, self.T = int(r), int(B), int(T)
         self.dtype = GRAPE_BF16 if dtype in ("bf16", GRAPE_BF16) else GRAPE_F32
+        self.T_full = 0   # tokens per sample of masked inputs (enable_compaction)
         self.ctx = grape_create(self.layers, self.r, C, sigma, seed, lr, beta1, beta2, eps, B, T,
                                 self.dtype, path)
+
+    def _inputs(self, A, Gout, T=None, cuda=True):
+        el = 2 if self.dtype == GRAPE_BF16 else 4
+        rows = self.B * (T or self.T)
+        if len(A) != len(self.layers) or len(Gout) != len(self.layers):
+            raise ValueError(f"need {len(self.layers)} A and Gout buffers")
+        for l, (d_in, d_out) in enumerate(self.layers):
+            _need(A[l], rows * d_in * el, el, f"A[{l}]", cuda)
+            _need(Gout[l], rows * d_out * el, el, f"Gout[{l}]", cuda)
+
+    def _weights(self, W):
+        if len(W) != len(self.layers):
+            raise ValueError(f"need {len(self.layers)} W buffers")
+        for l, (d_in, d_out) in enumerate(self.layers):
+            _need(W[l], d_in * d_out * 4, 4, f"W[{l}]", True)
 
     @classmethod
     def for_workload(cls, w, path=GRAPE_PATH_AUTO, B=None):
@@ -329,9 +367,13 @@ class GrapeStep:
     def enable_compaction(self, T_full: int):
         """Inputs of T_full tokens per sample, compacted to this context's T kept tokens."""
         grape_enable_compaction(self.ctx, T_full)
+        self.T_full = int(T_full)
 
     def step_masked(self, A, Gout, W, mask, step: int, stream=None):
         """The step over the tokens ``mask`` (uint8 / bool device tensor, B x T_full) keeps."""
+        self._inputs(A, Gout, self.T_full)
+        self._weights(W)
+        _need(mask, self.B * self.T_full, 1, "mask", True)
         grape_step_masked(self.ctx, A, Gout, W, mask, step, stream)
 
     def live_counts(self) -> np.ndarray:
@@ -346,6 +388,8 @@ class GrapeStep:
         if out is None:
             import torch
             out = torch.empty(self.B, dtype=torch.float32, device=A[0].device)
+        self._inputs(A, Gout)
+        _need(out, self.B * 4, 4, "out", True)
         grape_sqnorms(self.ctx, A, Gout, step, out, stream)
         return out
 
@@ -383,15 +427,22 @@ class GrapeStep:
         return grape_launch_count(self.ctx)
 
     def step(self, A, Gout, W, step: int, stream=None):
+        self._inputs(A, Gout)
+        self._weights(W)
         grape_step(self.ctx, A, Gout, W, step, stream)
 
     def step_host(self, A_host, Gout_host, W, step: int, norms_host=None, stream=None):
+        self._inputs(A_host, Gout_host, cuda=False)
+        self._weights(W)
+        _need(norms_host, self.B * 4, 4, "norms_host", False)
         grape_step_host(self.ctx, A_host, Gout_host, W, step, norms_host, stream)
 
     def accumulate(self, A, Gout, step: int, stream=None):
+        self._inputs(A, Gout)
         grape_accumulate(self.ctx, A, Gout, step, stream)
 
     def apply(self, W, step: int, batch_total: int = 0, stream=None):
+        self._weights(W)
         grape_apply(self.ctx, W, step, batch_total, stream)
 
     def S_tensor(self, layer: int):
@@ -408,9 +459,17 @@ class GrapeStep:
         return torch.as_tensor(_DeviceArray(ptr, (n,)), device="cuda")
 
     def get_state(self, layer: int, m, v, stream=None):
+        if 0 <= layer < len(self.layers):   # the library refuses other layers
+            n = self.r * self.layers[layer][1] * 4
+            _need(m, n, 4, "m", True)
+            _need(v, n, 4, "v", True)
         grape_get_state(self.ctx, layer, m, v, stream)
 
     def set_state(self, layer: int, m, v, stream=None):
+        if 0 <= layer < len(self.layers):   # the library refuses other layers
+            n = self.r * self.layers[layer][1] * 4
+            _need(m, n, 4, "m", True)
+            _need(v, n, 4, "v", True)
         grape_set_state(self.ctx, layer, m, v, stream)
 
     # intermediates of the last step (host copies)
