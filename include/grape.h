@@ -208,7 +208,7 @@ GRAPE_API int grape_set_norm_method(grape_ctx* ctx, int32_t method);
  * random subspace serves K consecutive steps (the refresh schedule is left
  * open by design choice 1 of "Metodologia: DP-GRAPE" in the technical summary
  * of "Memory-Efficient Differentially Private Training with Gradient Random
- * Projection": P is "regenerated from a seed").  The noise is still drawn per
+ * Projection", which has P rebuilt from a seed).  The noise is still drawn per
  * step, and m and v carry over a refresh unchanged.  A step whose key equals
  * that of the P already in the library's scratch does not regenerate it.
  * Setting the period makes the next step draw P afresh.  The scratch is shared

@@ -16,10 +16,10 @@ pages of the same paper):
 1. random Gaussian projection matrices, one per layer, regenerated from a
    seed instead of stored (design choice 1 of "Metodología");
 2. the *raw* per-sample gradients are projected first, then clipped and
-   noised in the projected space (design choice 2, "projection before
-   privatization");
+   noised in the projected space (design choice 2: projection comes before
+   privatization);
 3. Adam's first and second moments live in the projected space
-   (design choice 3, "projected optimizer states");
+   (design choice 3: the optimizer states are kept projected);
 4. the loop: per-layer projection of per-sample gradients, then
    aggregation, clipping and noise, then a projected Adam update of the
    parameters (closing paragraph of "Metodología").
@@ -82,8 +82,9 @@ def philox4x32_10(counter: np.ndarray, key: Sequence[int]) -> np.ndarray:
     return np.stack(c, axis=1).astype(np.uint32)
 
 
-# Streams of the method's randomness (reading: the pages only say "regenerated
-# from a seed"; the key and counter layout below are this library's choice).
+# Streams of the method's randomness (reading: the pages say only that P is rebuilt
+# from a seed rather than stored; the key and counter layout below are this
+# library's choice).
 STREAM_PROJECTION = 0
 STREAM_NOISE = 1
 
@@ -132,8 +133,8 @@ def projection_matrix(seed: int, layer: int, step: int, d_in: int, r: int) -> np
 
     Reading: the pages give no scale for the Gaussian matrix; 1/sqrt(r) makes
     E[P P^T] = I, so P P^T G is an unbiased estimate of G.  P is re-drawn at
-    every step from (seed, layer, step) (reading of "regenerated on the fly
-    from a seed").
+    every step from (seed, layer, step) (reading of design choice 1, which has P
+    rebuilt from a seed whenever it is needed).
     """
     return gaussian_stream(seed, layer, step, STREAM_PROJECTION, d_in * r).reshape(d_in, r) / np.sqrt(r)
 
@@ -196,8 +197,8 @@ class Hyper:
     def projection_key(self, step: int) -> int:
         """Step field of P's Philox counter at step s.
 
-        Reading: "regenerated on the fly from a seed" (design choice 1 of
-        "Metodología") leaves the refresh schedule open.  K = 1 re-draws P every
+        Reading: design choice 1 of "Metodología" has P rebuilt from a seed and
+        leaves the refresh schedule open.  K = 1 re-draws P every
         step; K > 1 keeps one random subspace for K consecutive steps (as GaLore
         keeps its SVD subspace between refreshes), with m and v carried across
         refreshes unchanged.  The noise is drawn per step whatever K is.

@@ -7,8 +7,8 @@
 // constants between rounds.
 //
 // Stream layout of the method's randomness (this library's reading of
-// "regenerated on the fly from a seed", Metodologia design choice 1 of the
-// DP-GRAPE technical summary): key = (seed lo, seed hi), counter =
+// Metodologia design choice 1 of the DP-GRAPE technical summary, which has P
+// rebuilt from a seed instead of stored): key = (seed lo, seed hi), counter =
 // (q, layer, step, stream), stream 0 = projection matrix, 1 = noise.  Element
 // e of a stream uses block q = e / 4: words (x0, x1) give elements 4q, 4q+1
 // (cosine, sine) and words (x2, x3) give 4q+2, 4q+3.
