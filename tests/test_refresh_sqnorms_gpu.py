@@ -80,6 +80,9 @@ SQN = {
     "vit_qkv_down_B3_T197": (W.scaled(W.get("vit_b"), layers=((768, 2304), (3072, 768)), B=3), TC, 2e-2),
     "r512_T130": (W.scaled(W.get("llm7b_slice"), layers=((512, 1024),), r=512, B=2, T=130), TC, 2e-2),
     "mlp_K2_step3": (W.scaled(W.get("mlp4x1024"), n_layers=2, B=3, T=64, refresh=2), TC, 2e-2),
+    # the DP-SGD-RC page's sketch width k = 32, on odd fp32 shapes (CUDA-core path)
+    "f32_k32_T100": (W.scaled(W.get("tiny_f32"), layers=((256, 192), (96, 130)), r=32, B=5, T=100),
+                     SIMT, 1e-5),
 }
 
 
