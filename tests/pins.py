@@ -362,6 +362,38 @@ def pin_refresh_period_two(O):
     P = [O.step(st, A, G, s, h)["P"][0] for s in range(3)]
     assert np.array_equal(P[0], P[1]) and not np.allclose(P[1], P[2])
     assert not np.allclose(O.noise_matrix(h.seed, 0, 0, 2, 4), O.noise_matrix(h.seed, 0, 1, 2, 4))
+    # the noise the step itself adds, recovered from a first Adam step (m = (1 - beta1) g,
+    # g = (S + sigma C xi) / B): stream 1 keyed on the step, not on the refresh key, so
+    # the two steps of one period draw different noise
+    B = A[0].shape[0]
+    xi = []
+    for s in (0, 1):
+        st = O.State.init(W0, h.r)
+        out = O.step(st, A, G, s, h)
+        for l in range(len(W0)):
+            got = (B * st.m[l] / (1.0 - h.beta1) - out["S"][l]) / (h.sigma * h.C)
+            assert np.allclose(got, O.noise_matrix(h.seed, l, s, h.r, W0[l].shape[1]), rtol=1e-9, atol=1e-9)
+        xi.append(got)
+    assert not np.allclose(xi[0], xi[1])
+
+
+def pin_spot_check_norms_match_the_step(O):
+    """The full-size parity tests recompute a few samples' norms with ``sample_norms`` and
+    compare ``grape_sqnorms`` with ``hutchinson_sample_sqnorms``.  On a subset of samples,
+    under a refresh period (step 3, K = 2, so the key differs from the step), the first
+    must equal the norms the step computes, and the second, with k = r sketch columns
+    drawn as DP-GRAPE draws P, their squares (sum_j p_j^T G G^T p_j = ||P^T G||_F^2)."""
+    A, G, W0 = _tiny_problem(41, B=5)
+    h = O.Hyper(r=3, C=0.5, sigma=0.7, seed=12, refresh=2)
+    out = O.step(O.State.init(W0, h.r), A, G, 3, h)
+    pick = [0, 2, 4]
+    sub_A = [a[pick] for a in A]
+    sub_G = [g[pick] for g in G]
+    d_in = [w.shape[0] for w in W0]
+    n = O.sample_norms(sub_A, sub_G, 3, h, d_in)
+    assert np.allclose(n, out["norms"][pick], rtol=1e-12, atol=0)
+    sq = O.hutchinson_sample_sqnorms(sub_A, sub_G, 3, h, d_in)
+    assert np.allclose(sq, out["norms"][pick] ** 2, rtol=1e-10, atol=0)
 
 
 # --------------------------------------------------------------------------
@@ -476,6 +508,7 @@ ALL_PINS = [
     pin_identity_projection_is_dp_adam, pin_clipping_bound, pin_sigma_zero,
     pin_adam_first_step, pin_no_privacy_reduction, pin_backprojection_unbiased,
     pin_projection_before_privatization, pin_refresh_fixed_subspace, pin_refresh_period_two,
+    pin_spot_check_norms_match_the_step,
     pin_hutchinson_identity_sketch, pin_hutchinson_unbiased, pin_hutchinson_factored,
     pin_masked_tokens_drop_out, pin_ghost_norm_equals_projected_norm,
     pin_ghost_norm_with_identity_is_gradient_norm,

@@ -89,6 +89,45 @@ MUTATIONS = {
     "token_mean_gradient": ("return A_i.T @ Gout_i", "return A_i.T @ Gout_i / A_i.shape[0]"),
     "hutch_transposed_sketch": ("return float(sum(P[:, j] @ O @ P[:, j] for j in range(P.shape[1])))",
                                 "return float(sum(P[:, j] @ O.T @ O @ P[:, j] for j in range(P.shape[1])))"),
+    # generator details
+    "key_words_swapped": ("return philox4x32_10(ctr, (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF))",
+                          "return philox4x32_10(ctr, ((seed >> 32) & 0xFFFFFFFF, seed & 0xFFFFFFFF))"),
+    "philox_hi_lo_swapped": ("hi0, lo0 = p0 >> np.uint64(32), p0 & _MASK32",
+                             "lo0, hi0 = p0 >> np.uint64(32), p0 & _MASK32"),
+    "weyl_before_first_round": ("        if rnd > 0:\n", "        if True:\n"),
+    "bm_u2_offset": ("u2 = xb.astype(np.float64) * 2.0 ** -32",
+                     "u2 = (xb.astype(np.float64) + 1.0) * 2.0 ** -32"),
+    "bm_log2": ("rho = np.sqrt(-2.0 * np.log(u1))", "rho = np.sqrt(-2.0 * np.log2(u1))"),
+    # the step
+    "noise_not_averaged": ("g = (S_l + h.sigma * h.C * xi) / div", "g = S_l / div + h.sigma * h.C * xi"),
+    "clip_on_sqnorm": ("c = np.array([clip_factor(n, h.C) for n in norms])",
+                       "c = np.array([clip_factor(n * n, h.C) for n in norms])"),
+    "noise_keyed_by_refresh": ("xi = noise_matrix(h.seed, l, step_index,",
+                               "xi = noise_matrix(h.seed, l, h.projection_key(step_index),"),
+    "noise_layer_zero": ("xi = noise_matrix(h.seed, l, step_index,", "xi = noise_matrix(h.seed, 0, step_index,"),
+    "P_layer_zero": ("return lambda layer, step, d_in, r: projection_matrix(h.seed, layer,",
+                     "return lambda layer, step, d_in, r: projection_matrix(h.seed, 0,"),
+    "adam_no_sqrt": ("return m, v, m_hat / (np.sqrt(v_hat) + eps)", "return m, v, m_hat / (v_hat + eps)"),
+    "hutch_divided_by_k": ("return float(sum(P[:, j] @ O @ P[:, j] for j in range(P.shape[1])))",
+                           "return float(sum(P[:, j] @ O @ P[:, j] for j in range(P.shape[1]))) / P.shape[1]"),
+    # the spot-check functions of the full-size tests
+    "sample_norms_no_sqrt": (
+        "            tot[j] += float(np.sum(project(P, per_sample_gradient(A[l][j], Gout[l][j])) ** 2))\n"
+        "    return np.sqrt(tot)",
+        "            tot[j] += float(np.sum(project(P, per_sample_gradient(A[l][j], Gout[l][j])) ** 2))\n"
+        "    return tot"),
+    "sample_norms_ignore_refresh": (
+        "        P = projection_matrix(h.seed, l, h.projection_key(step_index), d_in[l], h.r)\n"
+        "        for j in range(n):\n            tot[j] += float(",
+        "        P = projection_matrix(h.seed, l, step_index, d_in[l], h.r)\n"
+        "        for j in range(n):\n            tot[j] += float("),
+    "hutch_samples_ignore_refresh": (
+        "            tot[j] += hutchinson_sqnorm(A[l][j], Gout[l][j], P)",
+        "            tot[j] += hutchinson_sqnorm(A[l][j], Gout[l][j], "
+        "projection_matrix(h.seed, l, step_index, d_in[l], h.r))"),
+    "hutch_samples_first_layer": (
+        "            tot[j] += hutchinson_sqnorm(A[l][j], Gout[l][j], P)",
+        "            tot[j] += hutchinson_sqnorm(A[0][j], Gout[0][j], P) if l == 0 else 0.0"),
 }
 
 # cheap pins first: a mutation stops at the first pin that fails
