@@ -10,11 +10,17 @@ stay identical.
 from __future__ import annotations
 
 
-def dp_step(g, A, Gout, W, step: int, group=None, stream=None):
+def dp_step(g, A, Gout, W, step: int, group=None, stream=None, batch_total=None):
     """One step of context ``g`` (a GrapeStep or an object with the same methods)
-    inside ``torch.distributed`` process group ``group``."""
+    inside ``torch.distributed`` process group ``group``.
+
+    ``batch_total`` is the global batch the noisy sum is averaged over.  By default
+    every rank holds ``g.B`` samples (B x world); ranks whose shards differ in size
+    pass the sum of their shard sizes, the same number on every rank."""
     import torch.distributed as dist
     world = dist.get_world_size(group)
+    if batch_total is None:
+        batch_total = g.B * world
     g.accumulate(A, Gout, step, stream)
     if world > 1:
         if hasattr(g, "S_all_tensor"):
@@ -23,4 +29,4 @@ def dp_step(g, A, Gout, W, step: int, group=None, stream=None):
         else:
             for l in range(len(g.layers)):
                 dist.all_reduce(g.S_tensor(l), op=dist.ReduceOp.SUM, group=group)
-    g.apply(W, step, g.B * world, stream)
+    g.apply(W, step, batch_total, stream)

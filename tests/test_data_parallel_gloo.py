@@ -66,22 +66,32 @@ class OracleShard:
             Wt[l] -= torch.from_numpy(self.h.lr * (self.P[l] @ d))
 
 
-def _rank(rank, world, port, out):
+class PerLayerShard(OracleShard):
+    """The same shard without the flat S buffer: dp_step reduces S_l layer by layer."""
+
+    def __getattribute__(self, name):
+        if name == "S_all_tensor":
+            raise AttributeError(name)
+        return super().__getattribute__(name)
+
+
+def _rank(rank, world, port, out, shards=None, per_layer=False):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     from random_gradient_projection_b200.data_parallel import dp_step
     w = _workload()
-    per = w.B // world
-    rows = range(rank * per, (rank + 1) * per)
+    sizes = shards or [w.B // world] * world
+    start = sum(sizes[:rank])
+    rows = range(start, start + sizes[rank])
     W0 = W.make_weights(w)
-    g = OracleShard(w, rows, W0)
+    g = (PerLayerShard if per_layer else OracleShard)(w, rows, W0)
     Wt = [torch.from_numpy(x.astype(np.float64)) for x in W0]
     for s in range(w.steps):
         x = W.make_step_inputs(w, s, samples=list(rows))
         A = [x.as_f64(a) for a in x.A]
         G = [x.as_f64(gg) for gg in x.Gout]
-        dp_step(g, A, G, Wt, s)
+        dp_step(g, A, G, Wt, s, batch_total=sum(sizes) if shards else None)
     out[rank] = [t.numpy().copy() for t in Wt]
     dist.barrier()
     dist.destroy_process_group()
@@ -97,4 +107,22 @@ def test_two_rank_dp_step_equals_full_batch_oracle():
     ref = O.run(w, w.steps)["state"]
     for l in range(w.n_layers):
         assert np.array_equal(out[0][l], out[1][l])          # replicas identical
+        assert np.allclose(out[0][l], ref.W[l], rtol=0, atol=1e-13), l
+
+
+@pytest.mark.parametrize("per_layer", [False, True], ids=["one_allreduce", "per_layer"])
+def test_three_uneven_ranks_equal_full_batch_oracle(per_layer):
+    """Shards of 3, 2 and 1 samples with batch_total = 6, reduced either as one flat
+    buffer or layer by layer: every replica equals the single-process oracle step."""
+    world, shards = 3, [3, 2, 1]
+    port = 30500 + os.getpid() % 1000 + (7 if per_layer else 0)
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_rank, args=(world, port, out, shards, per_layer), nprocs=world,
+                       start_method="spawn", join=True)
+    w = _workload()
+    ref = O.run(w, w.steps)["state"]
+    for l in range(w.n_layers):
+        for r in range(1, world):
+            assert np.array_equal(out[0][l], out[r][l])
         assert np.allclose(out[0][l], ref.W[l], rtol=0, atol=1e-13), l
