@@ -72,6 +72,11 @@ CASES = {
     "no_noise_bf16": (W.scaled(W.get("mlp4x1024"), n_layers=2, B=4, T=64, sigma=0.0), 2),
     "T1_bf16_tc": (W.Workload("T1_tc", ((256, 256),), r=128, B=5, T=1, dtype="bf16", C=1.0,
                               sigma=0.5, steps=2), 2),
+    # tensor-core path with d_in off the 64-wide k-block and the 128-row back-projection
+    # tile (d_in % 8 == 0 is all it needs): a ragged last k-block in the projection and a
+    # ragged last M tile of W, both at the edge of their TMA boxes
+    "ragged_d_in_tc": (W.Workload("ragged_din", ((520, 256), (136, 512)), r=128, B=3, T=40,
+                                  dtype="bf16", C=1.0, sigma=0.8, steps=2), 2),
 }
 
 
