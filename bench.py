@@ -12,8 +12,9 @@ and rotate over several distinct per-step sets whose total is far larger than
 the 126 MB L2, each set alone already larger than L2.
 
 Prints one JSON line (rank 0).  With N > 1 (launched by torch.distributed.run)
-every rank runs its own B samples (weak scaling); the per-layer S is
-all-reduced over NCCL between aggregation and Adam.
+every rank runs its own B samples (weak scaling); every layer's S, back to back in
+one buffer, is summed over the ranks by a single NCCL all-reduce between the
+aggregation and Adam.
 """
 from __future__ import annotations
 
