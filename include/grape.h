@@ -27,7 +27,9 @@
  *
  * Conventions
  *  - Every device pointer is a CUDA device address on the context's device;
- *    host pointers are ordinary (preferably pinned) host memory.
+ *    host pointers are ordinary (preferably pinned) host memory.  A context is
+ *    bound to the device current at grape_create: every call that launches,
+ *    copies or synchronises returns GRAPE_EINVAL when another device is current.
  *  - Matrices are row-major.  A_l is B x T x d_in, Gout_l is B x T x d_out
  *    (samples contiguous, each sample's T token rows contiguous), in the
  *    context's input dtype (fp32, or bf16 as raw 16-bit patterns).  W_l is

@@ -149,7 +149,22 @@ int validate_io(grape_ctx* ctx, const void* const* A, const void* const* G, floa
   return GRAPE_OK;
 }
 
+// The context's buffers live on the device it was created on: a call made while another
+// device is current would launch there with this device's pointers.
+int check_device(grape_ctx* ctx) {
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) {
+    cudaGetLastError();
+    return ctx->fail(GRAPE_ECUDA, "cudaGetDevice failed");
+  }
+  if (cur != ctx->device)
+    return ctx->fail(GRAPE_EINVAL, "the context was created on device " + std::to_string(ctx->device) +
+                                       " but device " + std::to_string(cur) + " is current");
+  return GRAPE_OK;
+}
+
 int check_step_index(grape_ctx* ctx, int64_t step) {
+  if (int rc = check_device(ctx)) return rc;
   if (step < 0 || step > 0xFFFFFFFFll)
     return ctx->fail(GRAPE_EINVAL, "step must be in [0, 2^32)");
   return GRAPE_OK;
@@ -671,6 +686,7 @@ int grape_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_tot
 
 int grape_enable_compaction(grape_ctx* ctx, int32_t T_full) {
   if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  if (int rc = check_device(ctx)) return rc;
   if (T_full < ctx->sh.T) return ctx->fail(GRAPE_EINVAL, "T_full must be >= the context's T (the capacity)");
   if (ctx->sh.B > 65535) return ctx->fail(GRAPE_EINVAL, "compaction supports B <= 65535");
   if (ctx->compact_buf) return ctx->fail(GRAPE_EINVAL, "compaction is already enabled");
@@ -745,6 +761,7 @@ int grape_step_masked(grape_ctx* ctx, const void* const* A, const void* const* G
 
 int grape_live_counts(grape_ctx* ctx, int32_t* counts_host) {
   if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  if (int rc = check_device(ctx)) return rc;
   if (!ctx->compact_buf) return ctx->fail(GRAPE_EINVAL, "compaction is not enabled");
   if (!counts_host) return ctx->fail(GRAPE_EINVAL, "counts_host must not be null");
   cudaError_t e = cudaDeviceSynchronize();
@@ -809,6 +826,7 @@ int grape_sqnorms(grape_ctx* ctx, const void* const* A, const void* const* Gout,
 
 int grape_get_state(grape_ctx* ctx, int32_t layer, float* m_dev, float* v_dev, void* stream) {
   if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  if (int rc = check_device(ctx)) return rc;
   if (layer < 0 || layer >= ctx->sh.L) return ctx->fail(GRAPE_EINVAL, "layer out of range");
   if (!m_dev || !v_dev) return ctx->fail(GRAPE_EINVAL, "m_dev and v_dev must not be null");
   const size_t bytes = static_cast<size_t>(ctx->sh.r) * ctx->layers[layer].d_out * 4;
@@ -821,6 +839,7 @@ int grape_get_state(grape_ctx* ctx, int32_t layer, float* m_dev, float* v_dev, v
 int grape_set_state(grape_ctx* ctx, int32_t layer, const float* m_dev, const float* v_dev,
                     void* stream) {
   if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  if (int rc = check_device(ctx)) return rc;
   if (layer < 0 || layer >= ctx->sh.L) return ctx->fail(GRAPE_EINVAL, "layer out of range");
   if (!m_dev || !v_dev) return ctx->fail(GRAPE_EINVAL, "m_dev and v_dev must not be null");
   const size_t bytes = static_cast<size_t>(ctx->sh.r) * ctx->layers[layer].d_out * 4;
@@ -832,6 +851,7 @@ int grape_set_state(grape_ctx* ctx, int32_t layer, const float* m_dev, const flo
 
 int grape_debug(grape_ctx* ctx, int32_t what, int32_t layer, void* host_out) {
   if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  if (int rc = check_device(ctx)) return rc;
   if (!host_out) return ctx->fail(GRAPE_EINVAL, "host_out must not be null");
   const bool per_layer = what >= GRAPE_DBG_S;
   if (what < GRAPE_DBG_NORMS || what > GRAPE_DBG_V) return ctx->fail(GRAPE_EINVAL, "unknown debug item");
@@ -882,6 +902,7 @@ int grape_debug(grape_ctx* ctx, int32_t what, int32_t layer, void* host_out) {
 
 int grape_profile(grape_ctx* ctx, int32_t enable) {
   if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  if (int rc = check_device(ctx)) return rc;
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return ctx->cuda_fail(e, "synchronize");
   ctx->marks.clear();
@@ -892,6 +913,7 @@ int grape_profile(grape_ctx* ctx, int32_t enable) {
 
 int grape_profile_read(grape_ctx* ctx, double* ms_out, int64_t* count_out) {
   if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  if (int rc = check_device(ctx)) return rc;
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return ctx->cuda_fail(e, "synchronize");
   double ms[GRAPE_N_PHASES] = {};
