@@ -50,7 +50,7 @@ def build(force: bool = False, verbose: bool = False, extra=None) -> str:
         return LIB
     cmd = [nvcc(), *ARCH, "-lineinfo", "-O3", "-std=c++17", "--shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "-cudart", "static", "-I", os.path.join(ROOT, "include"),
-           "-Xptxas", "-warn-spills", *(extra or []), *sources(), "-o", LIB + ".tmp"]
+           "-Xptxas", "-warn-spills", *(extra or []), *sources(), "-ldl", "-o", LIB + ".tmp"]
     if verbose:
         print(" ".join(cmd))
     res = subprocess.run(cmd, capture_output=True, text=True)

@@ -2,6 +2,7 @@
 // phases (see include/grape.h for the contract of every entry point).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cmath>
 #include <cstdint>
@@ -25,6 +26,16 @@ int set_global(int code, const std::string& msg) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// An NVTX range over a scope: each public call and each phase of the step shows up by
+// name in a timeline or under `ncu --nvtx`.  Without an attached tool the push and pop
+// return at once.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Test hook: GRAPE_FAULT_ALLOC=n makes the n-th device allocation of a context fail.
 int fault_alloc_index() {
@@ -174,6 +185,7 @@ int check_step_index(grape_ctx* ctx, int64_t step) {
 // with two events on the step's stream.
 template <class F>
 int phase(grape_ctx* ctx, int id, const char* what, cudaStream_t st, F&& launch) {
+  const NvtxRange range(what);
   cudaEvent_t a = nullptr;
   if (ctx->prof_on) {
     a = ctx->next_event();
@@ -587,7 +599,11 @@ int grape_step(grape_ctx* ctx, const void* const* A, const void* const* Gout, fl
   rc = validate_io(ctx, A, Gout, W, true, true);
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (ctx->graph_on && !ctx->prof_on) return step_graph(ctx, A, Gout, W, step, st);
+  if (ctx->graph_on && !ctx->prof_on) {
+    const NvtxRange range("grape_step (graph replay)");
+    return step_graph(ctx, A, Gout, W, step, st);
+  }
+  const NvtxRange range("grape_step");
   rc = run_accumulate(ctx, A, Gout, step, st);
   if (rc) return rc;
   return run_apply(ctx, W, step, 0, st);
@@ -603,6 +619,7 @@ int grape_step_host(grape_ctx* ctx, const void* const* A_host, const void* const
     if (!A_host[l] || !Gout_host[l]) return ctx->fail(GRAPE_EINVAL, "null host input pointer");
   rc = validate_io(ctx, nullptr, nullptr, W, false, true);
   if (rc) return rc;
+  const NvtxRange range("grape_step_host");
   const size_t el = in_elsize(ctx->sh.dtype);
   const size_t rows = static_cast<size_t>(ctx->sh.B) * ctx->sh.T;
   if (ctx->stage_A.empty()) {
@@ -649,6 +666,7 @@ int grape_accumulate(grape_ctx* ctx, const void* const* A, const void* const* Go
   if (rc) return rc;
   rc = validate_io(ctx, A, Gout, nullptr, true, false);
   if (rc) return rc;
+  const NvtxRange range("grape_accumulate");
   return run_accumulate(ctx, A, Gout, step, static_cast<cudaStream_t>(stream));
 }
 
@@ -681,6 +699,7 @@ int grape_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_tot
     return ctx->fail(GRAPE_EINVAL, "grape_apply(step " + std::to_string(step) +
                                        ") needs a grape_accumulate of a step with the same projection"
                                        " (key step / refresh period) as the last call that drew P");
+  const NvtxRange range("grape_apply");
   return run_apply(ctx, W, step, batch_total, static_cast<cudaStream_t>(stream));
 }
 
@@ -736,6 +755,7 @@ int grape_step_masked(grape_ctx* ctx, const void* const* A, const void* const* G
   if (rc) return rc;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const grape::StepShape& sh = ctx->sh;
+  const NvtxRange range("grape_step_masked");
   rc = phase(ctx, GRAPE_PHASE_COMPACT, "compact live tokens", st, [&](int* n) {
     *n = 2;
     cudaError_t e = grape::compact_live_index(mask_dev, sh.B, ctx->T_full, sh.T, ctx->comp_idx,
@@ -814,6 +834,7 @@ int grape_sqnorms(grape_ctx* ctx, const void* const* A, const void* const* Gout,
   if (!sqnorms_dev || (reinterpret_cast<uintptr_t>(sqnorms_dev) & 3u) != 0)
     return ctx->fail(GRAPE_EINVAL, "sqnorms_dev must be a non-null, 4-byte aligned device pointer");
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const NvtxRange range("grape_sqnorms");
   std::vector<grape::LayerIo> io(ctx->sh.L);
   for (int l = 0; l < ctx->sh.L; ++l) io[l] = grape::LayerIo{A[l], Gout[l], nullptr};
   rc = run_project_norm(ctx, io.data(), step, st);
