@@ -50,6 +50,11 @@ def test_every_declared_symbol_is_exported(lib):
     (dict(layers=[(64, 32)], r=8, beta1=1.0), "adam"),
     (dict(layers=[(64, 32)], r=8, dtype=7), "in_dtype"),
     (dict(layers=[(64, 32)] * 65, r=8), "n_layers"),
+    (dict(layers=[(64, 32)], r=8, B=1 << 16, T=1 << 14), "B*T too large"),
+    (dict(layers=[(64, 0)], r=8), "d_in and d_out"),
+    (dict(layers=[(64, 32)], r=0), "r must be >= 1"),
+    (dict(layers=[(64, 32)], r=8, eps=0.0), "adam"),
+    (dict(layers=[(64, 32)], r=8, path=3), "path"),
 ])
 def test_create_validates_before_touching_the_device(lib, kw, msg):
     from random_gradient_projection_b200 import grape
