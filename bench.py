@@ -323,6 +323,10 @@ def main(argv=None):
     if args.impl == "reference":
         run_reference(args, rank, world)
         return 0
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} needs {args.gpus} ranks, one per GPU, but {world} "
+                         f"{'was' if world == 1 else 'were'} launched: run it under "
+                         f"`python -m torch.distributed.run --nproc-per-node {args.gpus} ...`")
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
     import torch

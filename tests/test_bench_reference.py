@@ -33,3 +33,14 @@ def test_reference_arm_prints_the_contract_line():
 def test_reference_arm_other_ranks_do_no_work():
     assert _run(["--workload", "tiny_f32", "--steps", "1", "--warmup", "1"],
                 {"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def test_our_arm_refuses_a_gpu_count_it_was_not_launched_with():
+    """--gpus N without N ranks would time one GPU and report it as N: it stops first,
+    before any device work (this runs on a machine without a GPU)."""
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--steps", "1",
+                          "--warmup", "3"], cwd=ROOT,
+                         capture_output=True, text=True, env=env, timeout=300)
+    assert out.returncode != 0
+    assert "needs 2 ranks" in out.stderr
