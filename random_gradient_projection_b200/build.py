@@ -19,6 +19,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libgrape.so")
+# bounds-checked variant (-DGRAPE_CHECKED): every TMA box start is checked in the kernels
+LIB_CHECKED = os.path.join(HERE, "libgrape_checked.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -38,19 +40,22 @@ def headers():
                   glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in sources() + headers() + [__file__])
 
 
-def build(force: bool = False, verbose: bool = False, extra=None) -> str:
-    if not force and up_to_date():
-        return LIB
+def build(force: bool = False, verbose: bool = False, extra=None, checked: bool = False) -> str:
+    """Build libgrape.so, or with ``checked`` the bounds-checked libgrape_checked.so."""
+    lib = LIB_CHECKED if checked else LIB
+    if not force and up_to_date(lib):
+        return lib
+    flags = ["-DGRAPE_CHECKED"] if checked else []
     cmd = [nvcc(), *ARCH, "-lineinfo", "-O3", "-std=c++17", "--shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "-cudart", "static", "-I", os.path.join(ROOT, "include"),
-           "-Xptxas", "-warn-spills", *(extra or []), *sources(), "-ldl", "-o", LIB + ".tmp"]
+           "-Xptxas", "-warn-spills", *flags, *(extra or []), *sources(), "-ldl", "-o", lib + ".tmp"]
     if verbose:
         print(" ".join(cmd))
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -58,8 +63,8 @@ def build(force: bool = False, verbose: bool = False, extra=None) -> str:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose and (res.stdout or res.stderr):
         print(res.stdout + res.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 def main(argv=None):
@@ -67,9 +72,11 @@ def main(argv=None):
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-v", action="store_true", help="print registers / spills per kernel")
+    ap.add_argument("--checked", action="store_true",
+                    help="build the bounds-checked libgrape_checked.so (GRAPE_LIB=checked loads it)")
     a = ap.parse_args(argv)
     extra = ["-Xptxas", "-v"] if a.ptxas_v else None
-    print(build(force=a.force or a.ptxas_v, verbose=a.verbose or a.ptxas_v, extra=extra))
+    print(build(force=a.force or a.ptxas_v, verbose=a.verbose or a.ptxas_v, extra=extra, checked=a.checked))
 
 
 if __name__ == "__main__":

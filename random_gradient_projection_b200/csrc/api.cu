@@ -423,6 +423,11 @@ int check_device_error(grape_ctx* ctx) {
   if (e != cudaSuccess) return ctx->cuda_fail(e, "read error word");
   if (v != 0) {
     cudaMemset(word, 0, sizeof(int));
+#ifdef GRAPE_CHECKED
+    if (v & grape::kTcErrBounds)
+      return ctx->fail(GRAPE_ECUDA, "checked build: a TMA box started outside its tensor or off the "
+                                    "16-byte rule, and its copy was skipped (code " + std::to_string(v) + ")");
+#endif
     return ctx->fail(GRAPE_ETIMEOUT, "a tensor-core kernel gave up waiting (code " +
                                          std::to_string(v) + ")");
   }

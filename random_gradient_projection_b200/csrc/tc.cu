@@ -104,7 +104,36 @@ struct GroupParams {
   float lr;          // BACKPROJ
   int cluster;       // AGGREGATE on a cluster: CTAs per output tile (K split)
   int* err;
+#ifdef GRAPE_CHECKED
+  int extA[kMaxGroup][3];   // x, y, z extents of the tensors behind mapA, mapB, mapW
+  int extB[kMaxGroup][3];
+  int extW[kMaxGroup][3];
+#endif
 };
+
+// Bounds-checked build (GRAPE_CHECKED): before each TMA copy, GRAPE_BOX checks that
+// the box starts inside its tensor and that x times the element size is a multiple of
+// 16 bytes.  A violation sets kTcErrBounds in the error word and skips the copy; its
+// stage then never completes, and the bounded waits end the kernel.  In the default
+// build GRAPE_BOX and GRAPE_EXT expand to nothing.
+#ifdef GRAPE_CHECKED
+__device__ __forceinline__ bool box_ok(int* err, const int (&ext)[3], int el, int x, int y, int z) {
+  const bool ok = x >= 0 && y >= 0 && z >= 0 && x < ext[0] && y < ext[1] && z < ext[2] &&
+                  (x * el) % 16 == 0;
+  if (!ok) atomicOr(err, kTcErrBounds);
+  return ok;
+}
+inline void set_ext(int (&e)[3], int64_t x, int64_t y, int64_t z) {
+  e[0] = static_cast<int>(x);
+  e[1] = static_cast<int>(y);
+  e[2] = static_cast<int>(z);
+}
+#define GRAPE_BOX(err, ext, el, x, y, z) if (!box_ok(err, ext, el, x, y, z)) {} else
+#define GRAPE_EXT(e, x, y, z) set_ext(e, x, y, z);
+#else
+#define GRAPE_BOX(err, ext, el, x, y, z)
+#define GRAPE_EXT(e, x, y, z)
+#endif
 
 template <int MODE>
 struct ModeTraits {
@@ -246,14 +275,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         const CUtensorMap* mapA = &p.mapA[c.g];
         const int kk = kb * kBK;
         if (MODE == PROJECT || MODE == BACKPROJ) {
+          GRAPE_BOX(p.err, p.extA[c.g], 2, kk, c.m_t * kBM, 0)
           ptx::tma_load_2d_hint(sa, mapA, &full[s], kk, c.m_t * kBM, MODE == BACKPROJ ? polB : polA);
         } else if (MODE == NORM) {
 #pragma unroll
           for (int q = 0; q < kBM / 64; ++q)
+            GRAPE_BOX(p.err, p.extA[c.g], 2, c.m_t * kBM + 64 * q, kk, c.s_t)
             ptx::tma_load_3d_hint(sa + q * 8192, mapA, &full[s], c.m_t * kBM + 64 * q, kk, c.s_t, polA);
         } else {
 #pragma unroll
           for (int q = 0; q < kBM / 64; ++q)
+            GRAPE_BOX(p.err, p.extA[c.g], 2, c.m_t * kBM + 64 * q, kk, 0)
             ptx::tma_load_2d_hint(sa + q * 8192, mapA, &full[s], c.m_t * kBM + 64 * q, kk, polA);
         }
       };
@@ -264,8 +296,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
 #pragma unroll
         for (int q = 0; q < BN / 64; ++q) {
           if (T::kB3d)
+            GRAPE_BOX(p.err, p.extB[c.g], 2, c.n_t * BN + 64 * q, kk, c.s_t)
             ptx::tma_load_3d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kk, c.s_t, polB);
           else
+            GRAPE_BOX(p.err, p.extB[c.g], 2, c.n_t * BN + 64 * q, kk, 0)
             ptx::tma_load_2d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kk, polB);
         }
       };
@@ -274,6 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         ptx::mbar_arrive_expect_tx(&wfull[wb], kWTile);
 #pragma unroll
         for (int q = 0; q < kBnBack / 32; ++q)
+          GRAPE_BOX(p.err, p.extW[c.g], 4, c.n_t * kBnBack + 32 * q, c.m_t * kBM, 0)
           ptx::tma_load_2d_hint(wbuf + q * kWBox, &p.mapW[c.g], &wfull[wb], c.n_t * kBnBack + 32 * q,
                                 c.m_t * kBM, polA);
       };
@@ -326,9 +361,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             const int kf = p.lay[c.g].kfirst;
             uint8_t* st_ = smem + s * S::kStage;
             if (kb < kf) {
+              GRAPE_BOX(p.err, p.extB[c.g], 2, kb * kBK, 0, c.s_t)
               ptx::tma_load_3d_hint(st_, &p.mapB[c.g], &full[s], kb * kBK, 0, c.s_t, polB);
             } else {
               ensure_wait();
+              GRAPE_BOX(p.err, p.extA[c.g], 2, (kb - kf) * kBK, 0, c.s_t)
               ptx::tma_load_3d_hint(st_, &p.mapA[c.g], &full[s], (kb - kf) * kBK, 0, c.s_t, polA);
             }
           } else if (MODE == PROJECT) {
@@ -555,6 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
           if (have && wgot) {
 #pragma unroll
             for (int q2 = 0; q2 < kBnBack / 32; ++q2)
+              GRAPE_BOX(p.err, p.extW[c.g], 4, c.n_t * kBnBack + 32 * q2, c.m_t * kBM, 0)
               ptx::tma_store_2d(&p.mapW[c.g], wbuf + q2 * kWBox, c.n_t * kBnBack + 32 * q2, c.m_t * kBM);
             ptx::bulk_commit_group();
             ptx::bulk_wait_group_read0();
@@ -663,6 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
         ptx::mbar_arrive_expect_tx(&full[s], S::kStage);
 #pragma unroll
         for (int q = 0; q < BN / 64; ++q)
+          GRAPE_BOX(p.err, p.extB[c.g], 2, c.n_t * BN + 64 * q, kb * kBK, 0)
           ptx::tma_load_2d_hint(sb + q * 8192, mapB, &full[s], c.n_t * BN + 64 * q, kb * kBK, pol);
         if (!waited) {
           ptx::griddep_wait();
@@ -670,6 +709,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
         }
 #pragma unroll
         for (int q = 0; q < kBM / 64; ++q)
+          GRAPE_BOX(p.err, p.extA[c.g], 2, c.m_t * kBM + 64 * q, kb * kBK, 0)
           ptx::tma_load_2d_hint(sa + q * 8192, mapA, &full[s], c.m_t * kBM + 64 * q, kb * kBK, pol);
         issued_end = it + 1;
       }
@@ -1191,6 +1231,8 @@ cudaError_t tc_project(const StepShape& sh, const LayerWs* ws, const LayerIo* io
         }))
       return false;
     gp.mapB[g] = hs.mapP_mn[l];
+    GRAPE_EXT(gp.extA[g], ws[l].d_in, rows, 1)
+    GRAPE_EXT(gp.extB[g], sh.r, ws[l].d_in, 1)
     GroupLayer& L = gp.lay[g];
     L.mt = cdiv(rows, kBM);
     L.nt = sh.r / hs.bn_project;
@@ -1222,6 +1264,8 @@ cudaError_t tc_project_norm(const StepShape& sh, const LayerWs* ws, const LayerI
           return map_3d(m, io[l].G, sh.B, sh.T, ws[l].d_out);
         }))
       return false;
+    GRAPE_EXT(gp.extA[g], sh.r, sh.T, sh.B)
+    GRAPE_EXT(gp.extB[g], ws[l].d_out, sh.T, sh.B)
     GroupLayer& L = gp.lay[g];
     L.mt = cdiv(sh.r, kBM);
     L.nt = cdiv(ws[l].d_out, kBnWide);
@@ -1255,6 +1299,8 @@ cudaError_t tc_project_norm_ghost(const StepShape& sh, const LayerWs* ws, const 
           return map_3d(m, io[l].G, sh.B, sh.T, ws[l].d_out, kBM);
         }))
       return false;
+    GRAPE_EXT(gp.extA[g], sh.r, sh.T, sh.B)
+    GRAPE_EXT(gp.extB[g], ws[l].d_out, sh.T, sh.B)
     GroupLayer& L = gp.lay[g];
     L.mt = 1;
     L.nt = 1;
@@ -1381,6 +1427,8 @@ cudaError_t tc_aggregate(const StepShape& sh, const LayerWs* ws, const LayerIo* 
             return map_2d(m, io[l].G, rows, ws[l].d_out, 64, 64);
           }))
         return cudaErrorInvalidValue;
+      GRAPE_EXT(gp.extA[g], sh.r, rows, 1)
+      GRAPE_EXT(gp.extB[g], ws[l].d_out, rows, 1)
       GroupLayer& L = gp.lay[g];
       L.tiles_begin = tiles;
       L.mt = cdiv(sh.r, kBM);
@@ -1411,6 +1459,9 @@ cudaError_t tc_backproject(const StepShape& sh, const LayerWs* ws, const LayerIo
   auto fill = [&](int g, int l, int* tiles) {
     gp.mapA[g] = hs.mapP_k[l];
     gp.mapB[g] = hs.mapDR[l];
+    GRAPE_EXT(gp.extA[g], sh.r, ws[l].d_in, 1)
+    GRAPE_EXT(gp.extB[g], ws[l].d_out, sh.r, 1)
+    GRAPE_EXT(gp.extW[g], ws[l].d_out, ws[l].d_in, 1)
     if (!hs.cacheW[l].get(io[l].W, &gp.mapW[g], [&](CUtensorMap* m) {
           return map_2d_f32(m, io[l].W, ws[l].d_in, ws[l].d_out);
         }))
@@ -1529,6 +1580,8 @@ cudaError_t tc_layer_sqnorms_static(const void* A, const void* G, int d_in, int 
   // AP = A P
   if (!map_2d(&gp.mapA[0], A, rows, d_in, 64, kBM) || !map_2d(&gp.mapB[0], P16, d_in, r, 64, 64))
     return cudaErrorInvalidValue;
+  GRAPE_EXT(gp.extA[0], d_in, rows, 1)
+  GRAPE_EXT(gp.extB[0], r, d_in, 1)
   GroupLayer& L = gp.lay[0];
   L.tiles_begin = 0;
   L.mt = cdiv(rows, kBM);
@@ -1550,6 +1603,8 @@ cudaError_t tc_layer_sqnorms_static(const void* A, const void* G, int d_in, int 
   gp.part_stride = slots;
   if (!map_3d(&gp.mapA[0], AP, B, T, r) || !map_3d(&gp.mapB[0], G, B, T, d_out))
     return cudaErrorInvalidValue;
+  GRAPE_EXT(gp.extA[0], r, T, B)
+  GRAPE_EXT(gp.extB[0], d_out, T, B)
   L = GroupLayer{};
   L.mt = cdiv(r, kBM);
   L.nt = cdiv(d_out, kBnWide);

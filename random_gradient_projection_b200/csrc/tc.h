@@ -8,6 +8,12 @@
 
 namespace grape {
 
+#ifdef GRAPE_CHECKED
+// Bounds-checked build: the error-word bit of a TMA box that would start outside its
+// tensor or off the 16-byte rule (the copy is skipped).
+constexpr int kTcErrBounds = 8;
+#endif
+
 struct TcWorkspace {
   void* base = nullptr;       // library scratch inside the context arena
   size_t bytes = 0;

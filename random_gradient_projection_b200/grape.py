@@ -14,7 +14,9 @@ from typing import Optional, Sequence
 import numpy as np
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libgrape.so")
+# GRAPE_LIB=checked loads the bounds-checked build (libgrape_checked.so) instead
+LIB_PATH = os.path.join(HERE, "libgrape_checked.so" if os.environ.get("GRAPE_LIB") == "checked"
+                        else "libgrape.so")
 
 GRAPE_OK, GRAPE_EINVAL, GRAPE_ENOMEM, GRAPE_ECUDA, GRAPE_ETIMEOUT, GRAPE_EUNSUPPORTED = range(6)
 GRAPE_MAX_LAYERS = 64
