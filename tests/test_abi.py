@@ -87,3 +87,30 @@ def test_selftest_validates_its_limits(lib):
     assert lib.grape_selftest_wait_timeout(-1, 10, None) == 1          # GRAPE_EINVAL
     assert lib.grape_selftest_wait_timeout(10, 5, None) == 1
     assert lib.grape_selftest_wait_timeout(2_000_000_000, 3_000_000_000, None) == 1
+
+
+def _header_constants():
+    """Every GRAPE_* integer the header defines, by #define or in an enum."""
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    vals = {k: int(v) for k, v in re.findall(r"#define\s+(GRAPE_[A-Z0-9_]+)\s+(\d+)\b", src)}
+    for body in re.findall(r"enum\s+\w+\s*\{(.*?)\}", src, flags=re.S):
+        vals.update({k: int(v) for k, v in re.findall(r"(GRAPE_[A-Z0-9_]+)\s*=\s*(\d+)", body)})
+    return vals
+
+
+def test_binding_constants_equal_the_header():
+    """grape.py restates the header's codes, paths, dtypes, debug items, norm methods and
+    phase order; a drift would mislabel results without any error."""
+    from random_gradient_projection_b200 import grape
+    hdr = _header_constants()
+    named = [k for k in hdr if hasattr(grape, k)]
+    assert len(named) >= 20, named
+    for k in named:
+        assert getattr(grape, k) == hdr[k], k
+    phases = sorted((v, k) for k, v in hdr.items() if k.startswith("GRAPE_PHASE_"))
+    assert len(grape.PHASES) == hdr["GRAPE_N_PHASES"] == len(phases)
+    short = {"GEN_P": "gen_P", "BACKPROJECT": "backproject"}
+    for (v, k), name in zip(phases, grape.PHASES):
+        tail = k[len("GRAPE_PHASE_"):]
+        assert short.get(tail, tail.lower()) == name, (k, name)
