@@ -74,10 +74,13 @@ def test_graph_replay_is_bitwise_the_ordinary_step(case):
     assert all(c == full for c in graph["counts"][2 * len(sets):])
 
 
-def test_graph_on_a_side_stream_matches_oracle():
+@pytest.mark.parametrize("size", ["reduced", "bench"])
+def test_graph_on_a_side_stream_matches_oracle(size):
     """Two persistent input buffers, refilled with each step's inputs: the pointers repeat
-    (steps 0-1 ordinary, 2-3 captured, 4-5 replayed) while the contents follow the oracle."""
-    w = W.scaled(W.get("mlp4x1024"), n_layers=2, B=4)
+    (steps 0-1 ordinary, 2-3 captured, 4-5 replayed) while the contents follow the oracle.
+    ``bench`` is the benchmarked workload at full size (4 x 1024^2, B = 64, T = 128) in the
+    launch configuration bench.py times: CUDA-graph replay."""
+    w = W.get("mlp4x1024") if size == "bench" else W.scaled(W.get("mlp4x1024"), n_layers=2, B=4)
     steps = 6
     bufs = _inputs(w, 2)
     side = torch.cuda.Stream()
