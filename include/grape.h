@@ -278,6 +278,15 @@ GRAPE_API int grape_launch_count(const grape_ctx* ctx, uint64_t* launches);
 
 /* Bytes of device memory the context holds (moments + workspace). */
 GRAPE_API int grape_device_bytes(const grape_ctx* ctx, uint64_t* bytes);
+/* The bytes grape_create would allocate for these arguments, computed on the host with no
+ * device call: the Adam moments m and v (8 r d_out per layer), every S_l (4 r d_out), dR,
+ * the projection scratch P (d_in r) and AP (B T r) per layer, and the per-sample norm
+ * buffers, each block rounded up to 256 bytes.  grape_enable_compaction and the staging of
+ * grape_step_host allocate separately.  Errors: as grape_create's argument checks
+ * (GRAPE_EINVAL; GRAPE_EUNSUPPORTED for the tensor-core path with fp32 inputs).  It does
+ * not check that the device supports the tensor-core path. */
+GRAPE_API int grape_context_bytes(const grape_layer* layers, int32_t n_layers, int32_t r, int32_t B, int32_t T,
+                                  int32_t in_dtype, int32_t path, uint64_t* bytes);
 
 /* Which kernel family the context runs (enum grape_path, never AUTO). */
 GRAPE_API int grape_path_of(const grape_ctx* ctx, int32_t* path);

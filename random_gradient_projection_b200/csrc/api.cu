@@ -983,6 +983,66 @@ const char* grape_last_error(const grape_ctx* ctx) { return ctx ? ctx->err.c_str
 
 const char* grape_global_error(void) { return g_global_error.c_str(); }
 
+int grape_context_bytes(const grape_layer* layers, int32_t n_layers, int32_t r, int32_t B, int32_t T,
+                        int32_t in_dtype, int32_t path, uint64_t* bytes) {
+  if (!bytes || !layers) return set_global(GRAPE_EINVAL, "layers and bytes must not be null");
+  if (n_layers < 1 || n_layers > GRAPE_MAX_LAYERS)
+    return set_global(GRAPE_EINVAL, "n_layers must be in [1, " + std::to_string(GRAPE_MAX_LAYERS) + "]");
+  if (B < 1 || T < 1) return set_global(GRAPE_EINVAL, "B and T must be >= 1");
+  if (r < 1) return set_global(GRAPE_EINVAL, "r must be >= 1");
+  if (in_dtype != GRAPE_F32 && in_dtype != GRAPE_BF16)
+    return set_global(GRAPE_EINVAL, "in_dtype must be GRAPE_F32 or GRAPE_BF16");
+  if (path < GRAPE_PATH_AUTO || path > GRAPE_PATH_TC)
+    return set_global(GRAPE_EINVAL, "path must be a grape_path value");
+  for (int l = 0; l < n_layers; ++l) {
+    if (layers[l].d_in < 1 || layers[l].d_out < 1)
+      return set_global(GRAPE_EINVAL, "layer " + std::to_string(l) + ": d_in and d_out must be >= 1");
+    if (r > layers[l].d_in)
+      return set_global(GRAPE_EINVAL, "layer " + std::to_string(l) + ": r must be <= d_in");
+  }
+  if (static_cast<int64_t>(B) * T > (int64_t{1} << 31) / 4) return set_global(GRAPE_EINVAL, "B*T too large");
+  const int resolved = path == GRAPE_PATH_AUTO ? (in_dtype == GRAPE_BF16 ? GRAPE_PATH_TC : GRAPE_PATH_SIMT) : path;
+  if (resolved == GRAPE_PATH_TC && in_dtype != GRAPE_BF16)
+    return set_global(GRAPE_EUNSUPPORTED, "the tensor-core path takes bf16 inputs");
+  // the arena of grape_create, block by block in its order
+  const bool tc = resolved == GRAPE_PATH_TC;
+  Arena ar;
+  size_t s_total = 0;
+  for (int l = 0; l < n_layers; ++l) s_total += static_cast<size_t>(r) * layers[l].d_out;
+  ar.take(s_total * 4);                                         // every S_l
+  int part = 0;
+  std::vector<grape::LayerWs> ws(n_layers);
+  for (int l = 0; l < n_layers; ++l) {
+    const size_t di = layers[l].d_in, dout = layers[l].d_out;
+    ar.take(di * r * (tc ? 2 : 4));                             // P (bf16 or fp32)
+    ar.take(static_cast<size_t>(B) * T * r * (tc ? 2 : 4));     // AP
+    ar.take(r * dout * 4);                                      // m
+    ar.take(r * dout * 4);                                      // v
+    ar.take(r * dout * (tc ? 2 : 4));                           // dR
+    ws[l].d_in = layers[l].d_in;
+    ws[l].d_out = layers[l].d_out;
+    ws[l].part_base = part;
+    ws[l].part_count = tc ? grape::tc_partials_per_sample(r, layers[l].d_out)
+                          : grape::simt_partials_per_sample(r, layers[l].d_out);
+    part += ws[l].part_count;
+  }
+  ar.take(static_cast<size_t>(B) * part * 4);                   // norm partials
+  ar.take(static_cast<size_t>(B) * 4);                          // norms
+  ar.take(static_cast<size_t>(B) * 4);                          // clip factors
+  if (tc) {
+    grape::StepShape sh{};
+    sh.L = n_layers;
+    sh.r = r;
+    sh.B = B;
+    sh.T = T;
+    sh.dtype = in_dtype;
+    sh.part_stride = part;
+    ar.take(grape::tc_workspace_bytes(sh, ws.data()));
+  }
+  *bytes = ar.off;
+  return GRAPE_OK;
+}
+
 void grape_destroy(grape_ctx* ctx) {
   if (!ctx) return;
   grape::tc_release(&ctx->tc);

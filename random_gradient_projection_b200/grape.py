@@ -33,7 +33,7 @@ EXPORTS = (
     "grape_philox_words", "grape_gaussian", "grape_profile", "grape_profile_read",
     "grape_launch_count", "grape_layer_sqnorms_static", "grape_set_refresh_period", "grape_sqnorms",
     "grape_enable_compaction", "grape_step_masked", "grape_live_counts", "grape_set_norm_method",
-    "grape_set_graph", "grape_selftest_wait_timeout", "grape_S_all",
+    "grape_set_graph", "grape_selftest_wait_timeout", "grape_S_all", "grape_context_bytes",
 )
 GRAPE_NORM_DIRECT, GRAPE_NORM_GHOST = 0, 1
 PHASES = ("gen_P", "project", "norm", "clip", "aggregate", "adam", "backproject", "compact")   # GRAPE_N_PHASES
@@ -72,6 +72,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "grape_set_state": ([vp, i32, vp, vp, vp], i32),
         "grape_debug": ([vp, i32, i32, vp], i32),
         "grape_device_bytes": ([vp, ctypes.POINTER(u64)], i32),
+        "grape_context_bytes": ([ctypes.POINTER(grape_layer), i32, i32, i32, i32, i32, i32,
+                                 ctypes.POINTER(u64)], i32),
         "grape_path_of": ([vp, ctypes.POINTER(i32)], i32),
         "grape_last_error": ([vp], ctypes.c_char_p),
         "grape_global_error": ([], ctypes.c_char_p),
@@ -235,6 +237,15 @@ def grape_debug(ctx: int, what: int, layer: int, shape) -> np.ndarray:
     out = np.empty(shape, dtype=np.float32)
     _check(lib().grape_debug(ctx, what, layer, out.ctypes.data), ctx)
     return out
+
+
+def grape_context_bytes(layers: Sequence[Sequence[int]], r: int, B: int, T: int, dtype: int,
+                        path: int = GRAPE_PATH_AUTO) -> int:
+    """Bytes grape_create would allocate for these arguments (host only, no device call)."""
+    arr = (grape_layer * len(layers))(*[grape_layer(int(a), int(b)) for a, b in layers])
+    out = ctypes.c_uint64()
+    _check(lib().grape_context_bytes(arr, len(layers), r, B, T, dtype, path, ctypes.byref(out)))
+    return out.value
 
 
 def grape_device_bytes(ctx: int) -> int:

@@ -114,3 +114,45 @@ def test_binding_constants_equal_the_header():
     for (v, k), name in zip(phases, grape.PHASES):
         tail = k[len("GRAPE_PHASE_"):]
         assert short.get(tail, tail.lower()) == name, (k, name)
+
+
+def test_context_bytes_is_the_documented_arena(lib):
+    """grape_context_bytes needs no device.  For the bench workload (4 x 1024^2, r = 128,
+    B = 64, T = 128, bf16, tensor-core path), block by block, each rounded up to 256 B:
+    every S_l 4 r sum(d_out) = 2 MiB; per layer P 2 d_in r = 256 KiB, AP 2 B T r = 2 MiB,
+    m and v 4 r d_out = 512 KiB each, dR 2 r d_out = 256 KiB; then the norm partials
+    (B x 16 slots x 4 B), norms, clip factors and the 256-byte error word."""
+    from random_gradient_projection_b200 import grape
+    layers = [(1024, 1024)] * 4
+    KiB, MiB = 1024, 1 << 20
+    per_layer = 256 * KiB + 2 * MiB + 2 * 512 * KiB + 256 * KiB
+    expect = 2 * MiB + 4 * per_layer + 64 * 16 * 4 + 256 + 256 + 256
+    assert grape.grape_context_bytes(layers, 128, 64, 128, grape.GRAPE_BF16) == expect == 16_782_080
+    # the fp32 CUDA-core path: fp32 P, AP and dR, one 64 x 64 partial slot per layer here
+    tiny = grape.grape_context_bytes([(64, 32)], 8, 4, 16, grape.GRAPE_F32)
+    assert tiny == 1024 + 2048 + 2048 + 1024 + 1024 + 1024 + 3 * 256
+
+
+def test_context_bytes_grows_with_r_times_d_out_not_d_in_times_d_out(lib):
+    """Optimizer state is O(r x layers): doubling d_in changes only P (d_in r), never the
+    moments; the moments alone are 8 r d_out per layer."""
+    from random_gradient_projection_b200 import grape
+    a = grape.grape_context_bytes([(1024, 1024)], 128, 8, 64, grape.GRAPE_BF16)
+    b = grape.grape_context_bytes([(2048, 1024)], 128, 8, 64, grape.GRAPE_BF16)
+    assert b - a == 1024 * 128 * 2                       # P grows by d_in r bf16, nothing else
+    c = grape.grape_context_bytes([(1024, 2048)], 128, 8, 64, grape.GRAPE_BF16)
+    assert c - a >= 8 * 128 * 1024                       # m and v grow with d_out
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(layers=[(64, 32)], r=80), 1),
+    (dict(layers=[(64, 32)], r=8, dtype=0, path=2), 5),
+    (dict(layers=[], r=8), 1),
+])
+def test_context_bytes_validates_like_create(lib, kw, code):
+    from random_gradient_projection_b200 import grape
+    args = dict(layers=[(64, 32)], r=8, B=4, T=16, dtype=grape.GRAPE_BF16, path=0)
+    args.update(kw)
+    with pytest.raises(grape.GrapeError) as e:
+        grape.grape_context_bytes(**args)
+    assert e.value.code == code
