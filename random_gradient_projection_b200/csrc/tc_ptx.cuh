@@ -76,7 +76,7 @@ __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parit
   }
 }
 
-// ---- TMA (no multicast) ---------------------------------------------------------
+// ---- TMA: tiled loads into this CTA's own shared memory, and tiled stores ----------
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");
 }
