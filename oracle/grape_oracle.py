@@ -281,7 +281,9 @@ def step(state: State, A: Sequence[np.ndarray], Gout: Sequence[np.ndarray], step
         state.W[l] = state.W[l] - h.lr * (Ps[l] @ d)
         S.append(S_l)
         dR.append(d)
-    return {"P": Ps, "R": R, "norms": norms, "clip": c, "S": S, "dR": dR}
+    # the moments after this step (copies: the state is updated again by later steps)
+    return {"P": Ps, "R": R, "norms": norms, "clip": c, "S": S, "dR": dR,
+            "m": [m.copy() for m in state.m], "v": [v.copy() for v in state.v]}
 
 
 def sample_norms(A: Sequence[np.ndarray], Gout: Sequence[np.ndarray], step_index: int,

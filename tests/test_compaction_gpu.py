@@ -14,7 +14,7 @@ import pytest
 
 import oracle.grape_oracle as O
 import workloads as W
-from harness import compare, rel_fro, to_device
+from harness import compare, rel_fro, snapshot, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -42,10 +42,7 @@ def _run(w, T_cap, steps, path, mask_fn=None):
         g.step_masked(A, G, Wd, torch.from_numpy(mask.astype(np.uint8)).cuda(), s)
         torch.cuda.synchronize()
         counts.append(g.live_counts())
-        lib_trace.append({"norms": g.norms(), "clip": g.clip(),
-                          "S": [g.S(l) for l in range(w.n_layers)],
-                          "m": [g.m(l) for l in range(w.n_layers)],
-                          "v": [g.v(l) for l in range(w.n_layers)]})
+        lib_trace.append(snapshot(g, w.n_layers))
         Gm = O.apply_token_mask([x.as_f64(a) for a in x.Gout], mask)
         orc_trace.append(O.step(st, [x.as_f64(a) for a in x.A], Gm, s, h))
         assert np.array_equal(counts[-1], np.minimum(mask.sum(axis=1), T_cap))

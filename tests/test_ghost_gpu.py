@@ -6,7 +6,7 @@ import pytest
 
 import oracle.grape_oracle as O
 import workloads as W
-from harness import compare, rel_fro, to_device
+from harness import compare, rel_fro, snapshot, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -36,8 +36,7 @@ def _run(w, steps, method):
         G = [to_device(a, w.dtype) for a in x.Gout]
         g.step(A, G, Ws, s)
         torch.cuda.synchronize()
-        trace.append({"norms": g.norms(), "clip": g.clip(), "S": [g.S(l) for l in range(w.n_layers)],
-                      "m": [g.m(l) for l in range(w.n_layers)], "v": [g.v(l) for l in range(w.n_layers)]})
+        trace.append(snapshot(g, w.n_layers))
     out = {"trace": trace, "W": [t.cpu().numpy() for t in Ws]}
     g.close()
     return out

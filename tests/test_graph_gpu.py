@@ -10,7 +10,7 @@ import pytest
 
 import oracle.grape_oracle as O
 import workloads as W
-from harness import compare, to_device
+from harness import compare, snapshot, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -98,8 +98,7 @@ def test_graph_on_a_side_stream_matches_oracle(size):
         torch.cuda.synchronize()
         g.step(A, G, Ws, s, side)
         side.synchronize()
-        trace.append({"norms": g.norms(), "clip": g.clip(), "S": [g.S(l) for l in range(w.n_layers)],
-                      "m": [g.m(l) for l in range(w.n_layers)], "v": [g.v(l) for l in range(w.n_layers)]})
+        trace.append(snapshot(g, w.n_layers))
     lib = {"trace": trace, "W": [x.cpu().numpy() for x in Ws]}
     g.close()
     res = O.run(w, steps)
