@@ -321,6 +321,10 @@ GRAPE_API int grape_gaussian(uint64_t seed, uint32_t layer, uint32_t step, uint3
  *
  *  A, Gout        device pointers, bf16, B x T x d_in and B x T x d_out
  *  r              projection width; P = z(seed, layer, step, stream 0, .)/sqrt(r)
+ *  layer, step    the layer and step fields of P's Philox counter.  `step` is the
+ *                 projection KEY, not necessarily the training step: a context with
+ *                 a refresh period K (grape_set_refresh_period) draws the P of
+ *                 training step s with key s / K, so pass s / K to get its norms
  *  sqnorms_out    device pointer, B floats (written; NaN if a device-side wait
  *                 gave up)
  *  stream         cudaStream_t (NULL = default stream); nothing is synchronised
@@ -330,10 +334,16 @@ GRAPE_API int grape_gaussian(uint64_t seed, uint32_t layer, uint32_t step, uint3
  * are rejected with GRAPE_EINVAL before anything is launched.
  * All calls share that one array (every GPU that loads the library holds its
  * 8 MiB until the process exits), so calls whose work overlaps on the GPU, on
- * different streams or host threads, race on it; serialise them.  The first
- * call on a device looks the array's address up on that device (it must be the
- * current device); make that first call before any stream capture.  Errors are
- * reported through grape_global_error(). */
+ * different streams or host threads, race on it; serialise them.  The array
+ * keeps the last call's contents; each call clears the one word that must start
+ * at zero (its error word) and rewrites the rest.  The first call on a device
+ * looks the array's address up on that device (it must be the current device)
+ * and keeps it for the life of the process; make that first call before any
+ * stream capture.  A cudaDeviceReset invalidates the kept address: do not call
+ * this entry point on a device after resetting it.  Several devices may each use
+ * it from one process (each has its own array and address).  Errors are reported
+ * through grape_global_error(): GRAPE_EINVAL (arguments, size), GRAPE_EUNSUPPORTED
+ * (not an sm_100a device, or no tensor-map encoder in the driver), GRAPE_ECUDA. */
 GRAPE_API int grape_layer_sqnorms_static(const void* A, const void* Gout, int32_t d_in, int32_t d_out,
                                          int32_t r, int32_t B, int32_t T, uint64_t seed,
                                          uint32_t layer, uint32_t step, float* sqnorms_out,

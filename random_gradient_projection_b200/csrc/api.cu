@@ -1111,6 +1111,8 @@ int grape_layer_sqnorms_static(const void* A, const void* Gout, int32_t d_in, in
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
   cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
   if (major != 10 || minor != 0) return set_global(GRAPE_EUNSUPPORTED, "needs an sm_100a device (B200)");
+  if (!grape::tc_tensor_maps_available())
+    return set_global(GRAPE_EUNSUPPORTED, "cuTensorMapEncodeTiled is not available from the driver");
   const size_t need = grape::tc_static_scratch_needed(d_in, d_out, r, B, T);
   if (need > grape::tc_static_scratch_bytes())
     return set_global(GRAPE_EINVAL, "problem needs " + std::to_string(need) + " bytes of scratch; the static scratch holds " +

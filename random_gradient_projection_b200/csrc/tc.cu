@@ -42,7 +42,9 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
 #include <vector>
 
 #include "philox.cuh"
@@ -1022,15 +1024,53 @@ cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStre
   return launch_maybe_pdl(true, kernel, grid, block, smem, st, args...);
 }
 
+// Launch configuration that belongs to a device: its SM count, and per kernel the
+// opt-in to more than 48 KB of dynamic shared memory (cudaFuncSetAttribute acts on the
+// current device only) with the residency that follows from it.  Each entry is taken
+// once per (device, kernel, key) under one lock, so host threads driving several GPUs
+// launch every kernel with its attribute set on the device it runs on.
+std::mutex g_launch_cfg_mu;
+std::map<std::tuple<int, const void*, int>, int> g_launch_cfg;   // (device, kernel, key) -> value
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    dev = 0;
+  }
+  return dev;
+}
+
 int sm_count() {
-  static int n = 0;
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lock(g_launch_cfg_mu);
+  int& n = g_launch_cfg[std::make_tuple(dev, static_cast<const void*>(nullptr), 0)];
   if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     if (n <= 0) n = 148;
   }
   return n;
+}
+
+// Sets `kernel`'s dynamic shared memory to `smem` bytes on the current device (once per
+// device) and returns in *per_sm how many of its CTAs of `threads` threads an SM holds.
+cudaError_t configure_kernel(const void* kernel, int smem, int threads, int* per_sm) {
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lock(g_launch_cfg_mu);
+  int& n = g_launch_cfg[std::make_tuple(dev, kernel, 1)];
+  if (n == 0) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    int got = 0;
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&got, kernel, threads, smem);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return e;
+    }
+    if (got < 1) return cudaErrorInvalidConfiguration;   // does not fit on an SM
+    n = got;
+  }
+  *per_sm = n;
+  return cudaSuccess;
 }
 
 // Persistent launch: as many CTAs as the runtime keeps resident at once (one per SM
@@ -1039,19 +1079,10 @@ int sm_count() {
 template <int MODE, int BN, int STAGES>
 cudaError_t launch_group(GroupParams& gp, int tiles, cudaStream_t st, bool pdl = true) {
   using S = SmemOf<MODE, BN, STAGES>;
-  static int per_sm = 0;
-  if (per_sm == 0) {
-    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<MODE, BN, STAGES>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
-    if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tc_gemm_kernel<MODE, BN, STAGES>, kThreads,
-                                                        S::kBytes);
-    if (e != cudaSuccess) {
-      per_sm = 0;
-      return e;
-    }
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;   // does not fit on an SM
-  }
+  int per_sm = 0;
+  cudaError_t e = configure_kernel(reinterpret_cast<const void*>(tc_gemm_kernel<MODE, BN, STAGES>), S::kBytes,
+                                   kThreads, &per_sm);
+  if (e != cudaSuccess) return e;
   gp.total_tiles = tiles;
   if (tiles <= 0) return cudaSuccess;
   int grid = sm_count() * per_sm;
@@ -1330,14 +1361,18 @@ cudaError_t tc_clip_scale(const StepShape& sh, const LayerWs* ws, const TcWorksp
 namespace {
 
 // How many clusters of `cs` CTAs of the aggregation kernel the device holds at once.
+// (cached per device and cluster size, 0 when the size cannot run)
 template <int BN, int STAGES>
 int clusters_resident(int cs) {
-  static int cached[9] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
   if (cs < 1 || cs > 8) return 0;
-  if (cached[cs] < 0) {
-    using S = Smem<BN, STAGES>;
-    cudaFuncSetAttribute(tc_agg_cluster_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         S::kBytes);
+  using S = Smem<BN, STAGES>;
+  const void* kern = reinterpret_cast<const void*>(tc_agg_cluster_kernel<BN, STAGES>);
+  int per_sm = 0;
+  if (configure_kernel(kern, S::kBytes, kThreads, &per_sm) != cudaSuccess) return 0;
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lock(g_launch_cfg_mu);
+  int& cached = g_launch_cfg[std::make_tuple(dev, kern, 100 + cs)];   // stored as count + 1
+  if (cached == 0) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(cs);
     cfg.blockDim = dim3(kThreads);
@@ -1352,21 +1387,18 @@ int clusters_resident(int cs) {
     int n = 0;
     const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, tc_agg_cluster_kernel<BN, STAGES>, &cfg);
     if (e != cudaSuccess) cudaGetLastError();
-    cached[cs] = (e == cudaSuccess) ? n : 0;
+    cached = 1 + ((e == cudaSuccess) ? n : 0);
   }
-  return cached[cs];
+  return cached - 1;
 }
 
 template <int BN, int STAGES>
 cudaError_t launch_agg_cluster(GroupParams& gp, int tiles, int cs, cudaStream_t st) {
   using S = Smem<BN, STAGES>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(tc_agg_cluster_kernel<BN, STAGES>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  int per_sm = 0;
+  cudaError_t e = configure_kernel(reinterpret_cast<const void*>(tc_agg_cluster_kernel<BN, STAGES>),
+                                   S::kBytes, kThreads, &per_sm);
+  if (e != cudaSuccess) return e;
   gp.total_tiles = tiles;
   gp.cluster = cs;
   cudaLaunchConfig_t cfg{};
@@ -1525,6 +1557,8 @@ __global__ void sum_slots_static_kernel(const float* partials, int slots, int B,
 }  // namespace
 
 size_t tc_static_scratch_bytes() { return kStaticScratchBytes; }
+
+bool tc_tensor_maps_available() { return encode_fn() != nullptr; }
 
 size_t tc_static_scratch_needed(int d_in, int d_out, int r, int B, int T) {
   const size_t slots = static_cast<size_t>(cdiv(r, kBM)) * cdiv(d_out, kBnWide);

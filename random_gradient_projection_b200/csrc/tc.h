@@ -64,6 +64,8 @@ cudaError_t tc_backproject(const StepShape& sh, const LayerWs* ws, const LayerIo
 // Per-sample squared norms of one layer using only the library's static device
 // scratch (grape_layer_sqnorms_static).
 size_t tc_static_scratch_bytes();
+// Whether the driver provides the tensor-map encoder every tensor-core kernel needs.
+bool tc_tensor_maps_available();
 size_t tc_static_scratch_needed(int d_in, int d_out, int r, int B, int T);
 cudaError_t tc_layer_sqnorms_static(const void* A, const void* G, int d_in, int d_out, int r, int B,
                                     int T, uint64_t seed, uint32_t layer, uint32_t step, float* out,
