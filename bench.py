@@ -3,9 +3,11 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Workload (default): four 1024 x 1024 linear layers, r = 128, B = 64 samples of
-T = 128 tokens, bf16 A and Gout, fp32 W and Adam moments (``workloads`` name
-``mlp4x1024``).  A "step" is one full pass of the method over one batch:
+Workload (default): the largest single-GPU configuration, a 7B-LLM-shaped slice of four
+decoder blocks (per block Q, K, V, O 4096 x 4096, gate and up 4096 x 11008, down
+11008 x 4096: 28 linear layers), r = 512, B = 16 samples of T = 512 tokens, bf16 A and
+Gout, fp32 W and Adam moments (``workloads`` name ``llm7b_slice``; ``--workload`` picks
+another).  A "step" is one full pass of the method over one batch:
 regenerate P, project, per-sample norms, clip, aggregate, noise + projected
 Adam, back-projection onto W.  Inputs are synthetic (seeded, see ``workloads``)
 and rotate over several distinct per-step sets whose total is far larger than
@@ -61,7 +63,7 @@ def parse(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="mlp4x1024", choices=sorted(WL.WORKLOADS))
+    ap.add_argument("--workload", default="llm7b_slice", choices=sorted(WL.WORKLOADS))
     ap.add_argument("--mode", default="step", choices=["step", "sqnorms"],
                     help="step: the whole DP-GRAPE step; sqnorms: per-sample norm estimates only")
     ap.add_argument("--no-graph", action="store_true",
@@ -107,7 +109,7 @@ class ClockSampler:
     def _poll(self):
         while not self._stop.is_set():
             self.sample()
-            time.sleep(0.002)
+            time.sleep(0.005)
 
     def sample(self):
         if not self.nv:
@@ -184,6 +186,31 @@ def phase_work(w, path: str):
     return out
 
 
+def phase_roofline(work, seconds: float, pk, path: str) -> dict:
+    """The roofline of one phase's launch: the bound its algorithmic work puts nearest
+    (dense bf16 tensor FLOPs at the sustained measured peak, since the phases are timed
+    inside a seconds-long run of steps, or bytes at the measured HBM copy bandwidth) and
+    what the measured time achieves against it.  The CUDA-core path is bound by fp32 FFMA
+    issue: 148 SMs x 128 lanes x 2 flop x the maximum SM clock."""
+    if path != "tc":
+        peak = 148 * 128 * 2 * pk["sm_max_mhz"] * 1e6 / 1e12
+        achieved = work["flops"] / seconds / 1e12
+        return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak,
+                "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x max SM clock"}
+    t_tc = work["flops"] / (pk["bf16_tflops_sustained"] * 1e12)
+    t_hbm = work["bytes"] / (pk["hbm_gbs"] * 1e9)
+    if t_tc > t_hbm:
+        achieved = work["flops"] / seconds / 1e12
+        peak = pk["bf16_tflops_sustained"]
+        return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_source": f"{pk['source']} sustained dense bf16"}
+    achieved = work["bytes"] / seconds / 1e9
+    peak = pk["hbm_gbs"]
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "peak_source": f"{pk['source']} HBM copy"}
+
+
 def sqnorms_work(w):
     """Work of the norm estimate alone: FLOPs of AP = A P and of the per-sample
     (A_i P)^T Gout_i, bytes of A and Gout read once and of the B outputs."""
@@ -233,67 +260,74 @@ def traffic_for(kernel: str, workload: str, path: str, mode: str = "step"):
 # the oracle on the host cores (baseline arm and cpu_baseline)
 # ---------------------------------------------------------------------------------------
 
+def _oracle_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def _oracle_call(O, w, st, h, s, nb, mode) -> float:
+    """Seconds of one oracle step (or norm pass) over the first ``nb`` samples of step s's
+    inputs; drawing the inputs is not timed."""
+    x = WL.make_step_inputs(w, s, samples=list(range(nb)), threads=8)
+    A = [x.as_f64(a) for a in x.A]
+    G = [x.as_f64(g) for g in x.Gout]
+    t0 = time.perf_counter()
+    if mode == "sqnorms":
+        O.sample_norms(A, G, s, h, [di for di, _ in w.layers])
+    else:
+        O.step(st, A, G, s, h)
+    return time.perf_counter() - t0
+
+
 def oracle_samples_per_s(w, target_s: float, max_steps: int = 1000, sub_batch=None, mode="step"):
     """Time the fp64 oracle, as it stands, on samples of the workload's batch.
 
-    Each timed call is one oracle step over ``sub_batch`` samples (the whole batch by
-    default); calls repeat until ``target_s`` of CPU work has been timed.  Input drawing
-    is outside the timed calls.  Returns (samples/s, samples timed, seconds, threads)."""
+    Each timed call is one oracle step over ``sub_batch`` samples; calls repeat until
+    ``target_s`` of CPU work has been timed.  Without ``sub_batch`` a first call over one
+    sample sizes the calls to about a third of the target each (at most the whole batch),
+    so that a large workload still gives a bounded sample.  Input drawing is outside the
+    timed calls.  Returns (samples/s, samples timed, seconds, threads, samples per call)."""
     import oracle.grape_oracle as O
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
-    except Exception:  # noqa: BLE001
-        threads = os.cpu_count() or 1
-    nb = sub_batch or w.B
     h = O.Hyper.of(w)
     st = O.State.init(WL.make_weights(w), w.r)
     done, spent, s = 0, 0.0, 0
+    nb = sub_batch
+    if nb is None:
+        t1 = _oracle_call(O, w, st, h, s, 1, mode)
+        spent, done, s = t1, 1, 1
+        nb = max(1, min(w.B, int(target_s / 3.0 / max(t1, 1e-9))))
     # a target of 0 s means: exactly max_steps calls (the reference arm's warm-up)
     while (spent < target_s or target_s <= 0) and s < max_steps:
-        x = WL.make_step_inputs(w, s, samples=list(range(nb)), threads=8)
-        A = [x.as_f64(a) for a in x.A]
-        G = [x.as_f64(g) for g in x.Gout]
-        t0 = time.perf_counter()
-        if mode == "sqnorms":
-            O.sample_norms(A, G, s, h, [di for di, _ in w.layers])
-        else:
-            O.step(st, A, G, s, h)
-        spent += time.perf_counter() - t0
+        spent += _oracle_call(O, w, st, h, s, nb, mode)
         done += nb
         s += 1
-    return (done / spent if spent > 0 else 0.0), done, spent, threads
+    return (done / spent if spent > 0 else 0.0), done, spent, _oracle_threads(), nb
 
 
 def run_reference(args, rank: int, world: int):
-    """--impl reference: the fp64 oracle timed on the host cores (rank 0 only)."""
+    """--impl reference: the fp64 oracle timed on the host cores (rank 0 only).
+
+    Each step is the oracle's step over the first ``sub`` samples of that step's batch,
+    ``sub`` sized from one untimed single-sample call so that the whole run of
+    warm-up and timed steps takes about two minutes (at most 4 samples per step)."""
     if rank != 0:
         return
     w = WL.get(args.workload)
-    sub = max(1, min(w.B, 4))
-    # warm-up calls (untimed), then K timed calls of a bounded sub-batch each
-    oracle_samples_per_s(w, 0.0, max_steps=max(1, args.warmup), sub_batch=sub, mode=args.mode)
     import oracle.grape_oracle as O
     h = O.Hyper.of(w)
+    t1 = _oracle_call(O, w, O.State.init(WL.make_weights(w), w.r), h, 0, 1, args.mode)
+    per_step = 120.0 / max(1, args.steps + args.warmup)
+    sub = max(1, min(w.B, 4, int(per_step / max(t1, 1e-9))))
+    # warm-up calls (untimed), then K timed calls of a bounded sub-batch each
+    oracle_samples_per_s(w, 0.0, max_steps=max(1, args.warmup), sub_batch=sub, mode=args.mode)
     st = O.State.init(WL.make_weights(w), w.r)
-    times = []
-    for s in range(args.steps):
-        x = WL.make_step_inputs(w, s, samples=list(range(sub)), threads=8)
-        A = [x.as_f64(a) for a in x.A]
-        G = [x.as_f64(g) for g in x.Gout]
-        t0 = time.perf_counter()
-        if args.mode == "sqnorms":
-            O.sample_norms(A, G, s, h, [di for di, _ in w.layers])
-        else:
-            O.step(st, A, G, s, h)
-        times.append(time.perf_counter() - t0)
+    times = [_oracle_call(O, w, st, h, s, sub, args.mode) for s in range(args.steps)]
     total = sum(times)
     value = sub * len(times) / total
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
-    except Exception:  # noqa: BLE001
-        cores = os.cpu_count() or 1
+    cores = _oracle_threads()
     sample = f"{sub} of {w.B} samples per step, all {w.n_layers} layers, fp64 numpy oracle"
     line = {
         "impl": "reference", "metric": METRIC if args.mode == "step" else METRIC_SQNORMS,
@@ -370,6 +404,8 @@ def main(argv=None):
     set_bytes = w.input_bytes()
 
     sq_out = torch.empty(w.B, dtype=torch.float32, device=dev)
+    # the plain step over each input set, its buffers checked and marshalled once
+    bound = [g.bind(A, G, Wd, torch.cuda.current_stream()) for A, G, _ in sets]
 
     def one(s):
         A, G, M = sets[s % n_sets]
@@ -380,7 +416,7 @@ def main(argv=None):
         elif world > 1:
             dp_step(g, A, G, Wd, s)
         else:
-            g.step(A, G, Wd, s)
+            bound[s % n_sets].step(s)
 
     def barrier():
         if world > 1:
@@ -460,17 +496,10 @@ def main(argv=None):
     tot = sum(v["ms_per_launch"] for v in per_phase.values())
     for v in per_phase.values():
         v["share"] = v["ms_per_launch"] / tot if tot > 0 else None
+    for name, v in per_phase.items():
+        v["roofline"] = phase_roofline(work[name], v["ms_per_launch"] / 1e3, pk, path_name)
     dom = max(per_phase, key=lambda k: per_phase[k]["ms_per_launch"])
-    avg_s = per_phase[dom]["ms_per_launch"] / 1e3
-    if path_name == "tc":
-        bound, unit = "hbm", "GB/s"
-        achieved = work[dom]["bytes"] / avg_s / 1e9
-        peak = pk["hbm_gbs"]
-    else:
-        # fp32 FFMA on the CUDA cores: 148 SMs x 128 lanes x 2 flop x max SM clock
-        bound, unit = "alu", "TFLOP/s"
-        achieved = work[dom]["flops"] / avg_s / 1e12
-        peak = 148 * 128 * 2 * pk["sm_max_mhz"] * 1e6 / 1e12
+    dom_roof = per_phase[dom]["roofline"]
     traffic = traffic_for(dom, w.name, path_name, args.mode)
     if masked:
         # the live-token lower bound: the method's work over the kept tokens only
@@ -478,7 +507,7 @@ def main(argv=None):
         flops, byts = step_work(w.replace(T=max(1, int(round(kept)))))
     else:
         flops, byts = step_work(w) if args.mode == "step" else sqnorms_work(w)
-    t_roof = max(flops / (pk["bf16_tflops"] * 1e12), byts / (pk["hbm_gbs"] * 1e9))
+    t_roof = max(flops / (pk["bf16_tflops_sustained"] * 1e12), byts / (pk["hbm_gbs"] * 1e9))
 
     # ---- end to end through the public API: host buffers, copies in the timed region ----
     e2e = None
@@ -555,10 +584,11 @@ def main(argv=None):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, n, secs, cores = oracle_samples_per_s(w, args.cpu_seconds, mode=args.mode)
+        v, n, secs, cores, nb = oracle_samples_per_s(w, args.cpu_seconds, mode=args.mode)
         cpu = {"value": v, "unit": "samples/s", "cores": cores, "kind": "oracle",
-               "sample": f"{n} samples ({n // w.B} full steps of B={w.B}) of {w.name}, "
-                         f"{secs:.1f} s of fp64 numpy oracle time"}
+               "sample": f"{n} samples of {w.name} (oracle steps over {nb} of its B={w.B} "
+                         f"samples, after one over a single sample), {secs:.1f} s of fp64 numpy "
+                         f"oracle time"}
 
     if rank == 0:
         line = {
@@ -581,12 +611,12 @@ def main(argv=None):
                        "cold_l2": {"ms_per_step": cold_ms / n_cold,
                                    "value": world * w.B * n_cold / (cold_ms / 1e3),
                                    "how": f"{n_cold} steps, each after a 256 MB write, timed one by one"}},
-            "roofline": {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,
-                         "unit": unit, "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": pk["source"] if bound != "alu" else
-                         "derived: 148 SMs x 128 FP32 lanes x 2 x max SM clock"},
+            "roofline": {"bound": dom_roof["bound"], "kernel": dom, "achieved": dom_roof["achieved"],
+                         "peak": dom_roof["peak"], "unit": dom_roof["unit"], "frac": dom_roof["frac"],
+                         "traffic": traffic, "peak_source": dom_roof["peak_source"]},
             "step_roofline": {"t_roof_us": t_roof * 1e6, "frac": t_roof / (ms_per_step / 1e3),
-                              "flops": flops, "bytes": byts, "peaks": pk["source"]},
+                              "flops": flops, "bytes": byts,
+                              "peaks": f"{pk['source']}: HBM copy and sustained dense bf16"},
             "phases": per_phase,
             "gpu_launches": launches,
             "clocks": sampler.summary(),

@@ -444,6 +444,15 @@ class GrapeStep:
         self._weights(W)
         grape_step(self.ctx, A, Gout, W, step, stream)
 
+    def bind(self, A, Gout, W, stream=None) -> "BoundStep":
+        """grape_step on fixed buffers: checks A, Gout and W once, marshals their
+        addresses and the stream once, and returns an object whose ``step(s)`` makes
+        only the C call.  For loops that step over the same buffers; the tensors are
+        kept referenced, and must not be resized while the binding is in use."""
+        self._inputs(A, Gout)
+        self._weights(W)
+        return BoundStep(self, A, Gout, W, stream)
+
     def step_host(self, A_host, Gout_host, W, step: int, norms_host=None, stream=None):
         self._inputs(A_host, Gout_host, cuda=False)
         self._weights(W)
@@ -506,3 +515,17 @@ class GrapeStep:
 
     def v(self, l):
         return grape_debug(self.ctx, GRAPE_DBG_V, l, (self.r, self.layers[l][1]))
+
+
+class BoundStep:
+    """grape_step with its buffers and stream marshalled once (GrapeStep.bind)."""
+
+    def __init__(self, owner: GrapeStep, A, Gout, W, stream=None):
+        self.owner = owner
+        self._keep = (list(A), list(Gout), list(W))   # the buffers outlive the binding
+        self._args = (_array(A), _array(Gout), _array(W))
+        self._stream = _stream(stream)
+
+    def step(self, step: int):
+        A, G, W = self._args
+        _check(lib().grape_step(self.owner.ctx, A, G, W, step, self._stream), self.owner.ctx)
