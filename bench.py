@@ -57,6 +57,21 @@ def layer_summary(w) -> str:
 
 
 
+def workload_of(args):
+    """The workload the arguments name, reduced by --layers / --batch if given (its name
+    then records the reduction)."""
+    w = WL.get(args.workload)
+    if args.layers or args.batch:
+        kw = {}
+        if args.layers:
+            kw["n_layers"] = args.layers
+        if args.batch:
+            kw["B"] = args.batch
+        w = WL.scaled(w, **kw)
+        w = w.replace(name=f"{w.name}[{w.n_layers} layers, B={w.B}]")
+    return w
+
+
 def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -71,10 +86,18 @@ def parse(argv=None):
                          "CUDA graph of the step (grape_set_graph)")
     ap.add_argument("--norm", default="direct", choices=["direct", "ghost"],
                     help="per-sample norms by R_i tiles (direct) or by the ghost Gram identity")
+    ap.add_argument("--agg", default="auto", choices=["auto", "recompute", "store"],
+                    help="aggregation S = sum_i c_i R_i: a second contraction over the stacked rows "
+                         "(recompute), a weighted sum of the R_i the norm kernel stored (store), or "
+                         "the library's choice by tokens per sample (auto)")
     ap.add_argument("--mask-capacity", type=int, default=0,
                     help="run masked steps (grape_step_masked) keeping at most this many loss "
                          "tokens per sample; the workload's own token mask is passed in")
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--layers", type=int, default=0,
+                    help="keep only the workload's first N layers (a reduced case for profiling)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="samples per batch instead of the workload's B (a reduced case for profiling)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -156,10 +179,13 @@ def peaks():
                 "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0, "source": "fallback"}
 
 
-def phase_work(w, path: str):
+def phase_work(w, path: str, agg: str = "recompute"):
     """Algorithmic bytes and flops of one launch of each phase (all layers in one call).
 
     Bytes count each operand once at its storage width: the minimum traffic of that phase.
+    With the stored aggregation (``agg`` "store") the norm phase also writes every R_i
+    (bf16, B r d_out per layer) and the aggregation reads them back once: a pass over
+    memory with no contraction.
     """
     el = 4 if w.dtype == "f32" else 2
     ap_el = 4 if path == "simt" else 2
@@ -176,6 +202,10 @@ def phase_work(w, path: str):
     out["aggregate"] = {"bytes": sum(rows * do * el + rows * w.r * ap_el + 4 * w.r * do
                                      for _, do in w.layers),
                         "flops": sum(2 * rows * w.r * do for _, do in w.layers)}
+    if agg == "store":
+        r_bytes = sum(2 * w.B * w.r * do for _, do in w.layers)
+        out["norm"]["bytes"] += r_bytes
+        out["aggregate"] = {"bytes": r_bytes + sum(4 * w.r * do for _, do in w.layers), "flops": 0}
     out["adam"] = {"bytes": sum(w.r * do * (4 + 16 + dr_el) for _, do in w.layers), "flops": 0}
     out["backproject"] = {"bytes": sum(8 * di * do + di * w.r * ap_el + w.r * do * dr_el
                                        for di, do in w.layers),
@@ -315,7 +345,7 @@ def run_reference(args, rank: int, world: int):
     warm-up and timed steps takes about two minutes (at most 4 samples per step)."""
     if rank != 0:
         return
-    w = WL.get(args.workload)
+    w = workload_of(args)
     import oracle.grape_oracle as O
     h = O.Hyper.of(w)
     t1 = _oracle_call(O, w, O.State.init(WL.make_weights(w), w.r), h, 0, 1, args.mode)
@@ -375,7 +405,7 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    w = WL.get(args.workload)
+    w = workload_of(args)
     path = {"auto": grape.GRAPE_PATH_AUTO, "simt": grape.GRAPE_PATH_SIMT,
             "tc": grape.GRAPE_PATH_TC}[args.path]
     masked = args.mask_capacity > 0
@@ -386,6 +416,9 @@ def main(argv=None):
         g.enable_compaction(w.T)
     if args.norm == "ghost":
         g.set_norm_method(grape.GRAPE_NORM_GHOST)
+    g.set_aggregation({"auto": grape.GRAPE_AGG_AUTO, "recompute": grape.GRAPE_AGG_RECOMPUTE,
+                       "store": grape.GRAPE_AGG_STORE}[args.agg])
+    agg_name = "store" if g.aggregation == grape.GRAPE_AGG_STORE else "recompute"
     if not args.no_graph:
         g.set_graph(True)      # grape_step replays one CUDA graph per input set
     path_name = {grape.GRAPE_PATH_SIMT: "simt", grape.GRAPE_PATH_TC: "tc"}[g.path]
@@ -393,7 +426,9 @@ def main(argv=None):
 
     # distinct per-step input sets; ranks draw different samples (input seed only)
     win = w.replace(seed=w.seed + 7919 * rank)
-    n_sets = INPUT_SETS if w.input_bytes() < (1 << 30) else 2
+    # (each set's graph is captured at its first step, so every set is first seen in the
+    # warm-up: no capture falls in the timed region)
+    n_sets = min(INPUT_SETS if w.input_bytes() < (1 << 30) else 2, args.warmup)
     sets = []
     for k in range(n_sets):
         x = WL.make_step_inputs(win, k, threads=16)
@@ -482,7 +517,7 @@ def main(argv=None):
 
     pk = peaks()
     w_run = w.replace(T=args.mask_capacity) if masked else w   # rows the GEMM phases see
-    work = phase_work(w_run, path_name)
+    work = phase_work(w_run, path_name, agg_name)
     if masked:
         work["compact"]["bytes"] = w.B * w.T + (work["compact"]["bytes"] - w_run.B * w_run.T)
     per_phase = {}
@@ -601,6 +636,7 @@ def main(argv=None):
                        "r": w.r, "B_per_gpu": w.B, "global_batch": w.B * world, "T": w.T,
                        "path": path_name, "parallelism": f"dp{world}", "mode": args.mode,
                        "mask_capacity": args.mask_capacity or None, "norm": args.norm,
+                       "aggregation": agg_name if args.mode == "step" else None,
                        "cuda_graph": (not args.no_graph) and args.mode == "step" and not masked and world == 1,
                        "l2": (f"inputs rotate over {n_sets} distinct sets of "
                               f"{set_bytes / 1e6:.0f} MB each (> 126 MB L2)")

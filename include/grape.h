@@ -95,7 +95,8 @@ typedef struct { double lr, beta1, beta2, eps; } grape_adam;
  *  in_dtype          GRAPE_F32 or GRAPE_BF16 (A and Gout)
  *  path              enum grape_path
  * Allocates the Adam moments (zeroed) and the workspace on the current CUDA
- * device; synchronises that device once.  *out receives the handle. */
+ * device; synchronises that device once.  *out receives the handle.  The aggregation
+ * method starts as GRAPE_AGG_AUTO resolves it (grape_set_aggregation). */
 GRAPE_API int grape_create(const grape_layer* layers, int32_t n_layers, int32_t r, double C, double sigma,
                  uint64_t seed, const grape_adam* adam, int32_t B, int32_t T, int32_t in_dtype,
                  int32_t path, grape_ctx** out);
@@ -179,7 +180,7 @@ GRAPE_API int grape_selftest_wait_timeout(int64_t short_ns, int64_t long_ns, int
 
 /* CUDA-graph replay of grape_step (enable != 0; default off).  The step's launches
  * are captured once per set of A, Gout and W pointers (the first grape_step with a
- * set runs as ordinary launches, the second captures it on a library stream), with
+ * set captures them on a library stream, then launches the graph), with
  * their programmatic dependencies, and replayed on the caller's stream (NULL
  * included); each replay rewrites the arguments that change with the step (P's
  * Philox key, Adam's step and bias corrections), so a replay computes exactly what
@@ -204,6 +205,33 @@ GRAPE_API int grape_set_graph(grape_ctx* ctx, int32_t enable);
  * tensor-core path and T <= 128). */
 enum grape_norm_method { GRAPE_NORM_DIRECT = 0, GRAPE_NORM_GHOST = 1 };
 GRAPE_API int grape_set_norm_method(grape_ctx* ctx, int32_t method);
+
+/* How S_l = sum_i c_i R_{i,l} is formed (the aggregation of the clipped projected
+ * per-sample gradients in the closing paragraph of "Metodologia: DP-GRAPE", technical
+ * summary of "Memory-Efficient Differentially Private Training with Gradient Random
+ * Projection").  Clipping needs every layer's ||R_i|| before any R_i can be weighted,
+ * so R_i is either formed twice or kept:
+ *  GRAPE_AGG_RECOMPUTE  S = (diag(c) A P)^T Gout over the B*T stacked token rows: a second
+ *                       contraction of 2 B T r d_out flops per layer (AP is rescaled by
+ *                       c in place first).  No extra memory.
+ *  GRAPE_AGG_STORE      the norm kernel also writes every R_i as bf16 (B x r x d_out per
+ *                       layer, 2 B r sum(d_out) bytes of device memory held by the
+ *                       context); S is then the c-weighted sum of those B matrices, one
+ *                       pass of 2 B r d_out bytes per layer.  R_i is rounded to bf16
+ *                       before the weighted sum (relative 2^-9 per element).
+ *  GRAPE_AGG_AUTO       STORE on the tensor-core path when T >= 256 tokens per sample,
+ *                       where the contraction it saves (proportional to T) costs more than
+ *                       moving R_i twice (independent of T); RECOMPUTE otherwise.  This is
+ *                       what grape_create applies, with the stored R_i in its arena.
+ * The ghost norm (GRAPE_NORM_GHOST) never forms R_i, so a context using it recomputes
+ * whatever this says.  grape_set_aggregation allocates the R_i storage on first asking
+ * for STORE when grape_create did not (GRAPE_ENOMEM if that fails) and keeps it until
+ * grape_destroy.  Errors: GRAPE_EINVAL (unknown method), GRAPE_EUNSUPPORTED (STORE on the
+ * CUDA-core path).  grape_aggregation_of reports the method the next step will use
+ * (RECOMPUTE or STORE). */
+enum grape_agg_method { GRAPE_AGG_AUTO = 0, GRAPE_AGG_RECOMPUTE = 1, GRAPE_AGG_STORE = 2 };
+GRAPE_API int grape_set_aggregation(grape_ctx* ctx, int32_t method);
+GRAPE_API int grape_aggregation_of(const grape_ctx* ctx, int32_t* method);
 
 /* Projection-refresh period K >= 1 (default 1).  P_l of step s is drawn with
  * the step field of its Philox counter set to floor(s / K) instead of s, so one
@@ -280,8 +308,9 @@ GRAPE_API int grape_launch_count(const grape_ctx* ctx, uint64_t* launches);
 GRAPE_API int grape_device_bytes(const grape_ctx* ctx, uint64_t* bytes);
 /* The bytes grape_create would allocate for these arguments, computed on the host with no
  * device call: the Adam moments m and v (8 r d_out per layer), every S_l (4 r d_out), dR,
- * the projection scratch P (d_in r) and AP (B T r) per layer, and the per-sample norm
- * buffers, each block rounded up to 256 bytes.  grape_enable_compaction and the staging of
+ * the projection scratch P (d_in r) and AP (B T r) per layer, the per-sample norm
+ * buffers, and the stored R_i (2 B r d_out per layer) when GRAPE_AGG_AUTO chooses them,
+ * each block rounded up to 256 bytes.  grape_enable_compaction and the staging of
  * grape_step_host allocate separately.  Errors: as grape_create's argument checks
  * (GRAPE_EINVAL; GRAPE_EUNSUPPORTED for the tensor-core path with fp32 inputs).  It does
  * not check that the device supports the tensor-core path. */

@@ -66,8 +66,14 @@ struct grape_ctx {
   uint32_t refresh = 1;
   int64_t p_key = -1;
   int norm_method = GRAPE_NORM_DIRECT;
+  // aggregation (grape_set_aggregation): recompute (diag(c) AP)^T Gout, or sum the R_i the
+  // norm kernel stored; agg is never AUTO.  The stored R_i live in the arena when AUTO
+  // chose them at create, else in rst_buf, allocated when a caller asks for them.
+  int agg = GRAPE_AGG_RECOMPUTE;
+  void* rst_buf = nullptr;
+  bool stores_R() const { return agg == GRAPE_AGG_STORE && norm_method == GRAPE_NORM_DIRECT; }
   // CUDA-graph replay of grape_step (grape_set_graph): one graph per set of A, Gout, W
-  // pointers; the first step with a set runs as ordinary launches, the second captures
+  // pointers; the first step with a set captures it, later ones replay it
   struct StepGraph {
     std::vector<const void*> A, G;
     std::vector<float*> W;
@@ -138,6 +144,20 @@ struct Arena {
 
 size_t in_elsize(int dtype) { return dtype == GRAPE_BF16 ? 2 : 4; }
 
+// GRAPE_AGG_AUTO's choice.  Recomputing the aggregation costs a second contraction of
+// 2 B T r d_out flops per layer (plus a re-read of Gout); storing R_i costs
+// 2 B r d_out bytes written by the norm kernel and read once more.  At the measured
+// tensor and HBM rates the two break even near T ~ kAggStoreMinT tokens per sample.
+constexpr int kAggStoreMinT = 256;
+bool auto_stores_R(int path, int T) { return path == GRAPE_PATH_TC && T >= kAggStoreMinT; }
+
+// Bytes of every layer's stored R_i: B x r x d_out bf16 each.
+size_t rstore_bytes(const grape_layer* layers, int n_layers, int r, int B) {
+  size_t n = 0;
+  for (int l = 0; l < n_layers; ++l) n += static_cast<size_t>(B) * r * layers[l].d_out * 2;
+  return n;
+}
+
 int validate_io(grape_ctx* ctx, const void* const* A, const void* const* G, float* const* W,
                 bool need_ag, bool need_w) {
   if (need_ag && (!A || !G)) return ctx->fail(GRAPE_EINVAL, "A and Gout arrays must not be null");
@@ -206,7 +226,9 @@ int phase(grape_ctx* ctx, int id, const char* what, cudaStream_t st, F&& launch)
 }
 
 // Generate P when its key changed, then AP = A P and the per-sample norm partials.
-int run_project_norm(grape_ctx* ctx, const grape::LayerIo* io, int64_t step, cudaStream_t st) {
+// store_R: the step's norm kernel also writes every R_i for the stored aggregation.
+int run_project_norm(grape_ctx* ctx, const grape::LayerIo* io, int64_t step, cudaStream_t st,
+                     bool store_R) {
   const grape::StepShape& sh = ctx->sh;
   const grape::LayerWs* ws = ctx->ws.data();
   const uint32_t key = static_cast<uint32_t>(step) / ctx->refresh;
@@ -230,7 +252,7 @@ int run_project_norm(grape_ctx* ctx, const grape::LayerIo* io, int64_t step, cud
     return phase(ctx, GRAPE_PHASE_NORM, "per-sample norms", st, [&](int* n) {
       if (ctx->norm_method == GRAPE_NORM_GHOST)
         return grape::tc_project_norm_ghost(sh, ws, io, tc, ctx->partials, st, n);
-      return grape::tc_project_norm(sh, ws, io, tc, ctx->partials, st, n);
+      return grape::tc_project_norm(sh, ws, io, tc, ctx->partials, store_R, st, n);
     });
   }
   rc = phase(ctx, GRAPE_PHASE_PROJECT, "project", st, [&](int* n) {
@@ -250,17 +272,19 @@ int run_accumulate(grape_ctx* ctx, const void* const* A, const void* const* G, i
   for (int l = 0; l < ctx->sh.L; ++l) io[l] = grape::LayerIo{A[l], G[l], nullptr};
   const grape::StepShape& sh = ctx->sh;
   const grape::LayerWs* ws = ctx->ws.data();
-  int rc = run_project_norm(ctx, io.data(), step, st);
+  const bool stored = ctx->path == GRAPE_PATH_TC && ctx->stores_R();
+  int rc = run_project_norm(ctx, io.data(), step, st, stored);
   if (rc) return rc;
   rc = phase(ctx, GRAPE_PHASE_CLIP, "clip", st, [&](int* n) {
     if (ctx->path == GRAPE_PATH_TC)
-      return grape::tc_clip_scale(sh, ws, ctx->tc, ctx->partials, ctx->norms, ctx->clip, st, n);
+      return grape::tc_clip_scale(sh, ws, ctx->tc, ctx->partials, ctx->norms, ctx->clip, !stored, st, n);
     *n = 1;
     return grape::finalize_clip(sh, ctx->partials, ctx->norms, ctx->clip, st);
   });
   if (rc) return rc;
   if (ctx->path == GRAPE_PATH_TC) {
     rc = phase(ctx, GRAPE_PHASE_AGGREGATE, "aggregate", st, [&](int* n) {
+      if (stored) return grape::tc_aggregate_stored(sh, ws, ctx->clip, st, n);
       return grape::tc_aggregate(sh, ws, io.data(), ctx->tc, ctx->clip, st, n);
     });
   } else {
@@ -321,7 +345,7 @@ int step_graph(grape_ctx* ctx, const void* const* A, const void* const* G, float
       break;
     }
   }
-  if (!hit) {   // first sight of this pointer set: ordinary launches, remembered for capture
+  if (!hit) {   // first sight of this pointer set: captured below, then replayed
     if (ctx->graphs.size() >= 8) {
       size_t lru = 0;
       for (size_t k = 1; k < ctx->graphs.size(); ++k)
@@ -333,10 +357,8 @@ int step_graph(grape_ctx* ctx, const void* const* A, const void* const* G, float
     g.A.assign(A, A + L);
     g.G.assign(G, G + L);
     g.W.assign(W, W + L);
-    g.used = ++ctx->graph_tick;
     ctx->graphs.push_back(g);
-    int rc = run_accumulate(ctx, A, G, step, st);
-    return rc ? rc : run_apply(ctx, W, step, 0, st);
+    hit = &ctx->graphs.back();
   }
   hit->used = ++ctx->graph_tick;
   if (!hit->captured) {
@@ -545,6 +567,12 @@ int grape_create(const grape_layer* layers, int32_t n_layers, int32_t r, double 
   size_t off_tc = 0;
   size_t tc_bytes = tc ? grape::tc_workspace_bytes(sh, ctx->ws.data()) : 0;
   if (tc) off_tc = ar.take(tc_bytes);
+  // GRAPE_AGG_AUTO: every layer's stored R_i, when the aggregation sums them
+  const bool store = auto_stores_R(resolved, T);
+  ctx->agg = store ? GRAPE_AGG_STORE : GRAPE_AGG_RECOMPUTE;
+  std::vector<size_t> off_rst(n_layers, SIZE_MAX);
+  if (store)
+    for (int l = 0; l < n_layers; ++l) off_rst[l] = ar.take(static_cast<size_t>(B) * r * layers[l].d_out * 2);
   ctx->arena_bytes = ar.off;
 
   const int fault = fault_alloc_index();
@@ -570,6 +598,7 @@ int grape_create(const grape_layer* layers, int32_t n_layers, int32_t r, double 
     w.m = reinterpret_cast<float*>(at(o.m));
     w.v = reinterpret_cast<float*>(at(o.v));
     w.dR = at(o.dR);
+    w.Rst = reinterpret_cast<__nv_bfloat16*>(at(off_rst[l]));
   }
   ctx->partials = reinterpret_cast<float*>(at(off_part));
   ctx->norms = reinterpret_cast<float*>(at(off_norms));
@@ -821,6 +850,46 @@ int grape_set_norm_method(grape_ctx* ctx, int32_t method) {
   return GRAPE_OK;
 }
 
+int grape_set_aggregation(grape_ctx* ctx, int32_t method) {
+  if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
+  if (method != GRAPE_AGG_AUTO && method != GRAPE_AGG_RECOMPUTE && method != GRAPE_AGG_STORE)
+    return ctx->fail(GRAPE_EINVAL, "method must be GRAPE_AGG_AUTO, GRAPE_AGG_RECOMPUTE or GRAPE_AGG_STORE");
+  int resolved = method;
+  if (resolved == GRAPE_AGG_AUTO)
+    resolved = auto_stores_R(ctx->path, ctx->sh.T) ? GRAPE_AGG_STORE : GRAPE_AGG_RECOMPUTE;
+  if (resolved == GRAPE_AGG_STORE) {
+    if (ctx->path != GRAPE_PATH_TC)
+      return ctx->fail(GRAPE_EUNSUPPORTED, "the stored aggregation runs on the tensor-core path");
+    if (int rc = check_device(ctx)) return rc;
+    if (!ctx->ws[0].Rst) {   // not in the arena: one allocation for every layer's R_i
+      const size_t bytes = rstore_bytes(ctx->layers.data(), ctx->sh.L, ctx->sh.r, ctx->sh.B);
+      void* buf = nullptr;
+      if (fault_alloc_index() == 2 || cudaMalloc(&buf, bytes) != cudaSuccess) {
+        cudaGetLastError();
+        return ctx->fail(GRAPE_ENOMEM, "cudaMalloc of " + std::to_string(bytes) + " bytes for the stored R_i failed");
+      }
+      ctx->rst_buf = buf;
+      char* at = static_cast<char*>(buf);
+      for (int l = 0; l < ctx->sh.L; ++l) {
+        ctx->ws[l].Rst = reinterpret_cast<__nv_bfloat16*>(at);
+        at += static_cast<size_t>(ctx->sh.B) * ctx->sh.r * ctx->layers[l].d_out * 2;
+      }
+    }
+  }
+  if (resolved != ctx->agg) {   // captured graphs hold the other aggregation
+    for (auto& g : ctx->graphs) ctx->drop_graph(g);
+    ctx->graphs.clear();
+  }
+  ctx->agg = resolved;
+  return GRAPE_OK;
+}
+
+int grape_aggregation_of(const grape_ctx* ctx, int32_t* method) {
+  if (!ctx || !method) return set_global(GRAPE_EINVAL, "ctx and method must not be null");
+  *method = ctx->stores_R() && ctx->path == GRAPE_PATH_TC ? GRAPE_AGG_STORE : GRAPE_AGG_RECOMPUTE;
+  return GRAPE_OK;
+}
+
 int grape_set_refresh_period(grape_ctx* ctx, int32_t period) {
   if (!ctx) return set_global(GRAPE_EINVAL, "ctx must not be null");
   if (period < 1) return ctx->fail(GRAPE_EINVAL, "refresh period must be >= 1");
@@ -842,7 +911,7 @@ int grape_sqnorms(grape_ctx* ctx, const void* const* A, const void* const* Gout,
   const NvtxRange range("grape_sqnorms");
   std::vector<grape::LayerIo> io(ctx->sh.L);
   for (int l = 0; l < ctx->sh.L; ++l) io[l] = grape::LayerIo{A[l], Gout[l], nullptr};
-  rc = run_project_norm(ctx, io.data(), step, st);
+  rc = run_project_norm(ctx, io.data(), step, st, false);
   if (rc) return rc;
   return phase(ctx, GRAPE_PHASE_CLIP, "sum norm partials", st, [&](int* n) {
     *n = 1;
@@ -1039,6 +1108,8 @@ int grape_context_bytes(const grape_layer* layers, int32_t n_layers, int32_t r, 
     sh.part_stride = part;
     ar.take(grape::tc_workspace_bytes(sh, ws.data()));
   }
+  if (auto_stores_R(resolved, T))                               // stored R_i (GRAPE_AGG_AUTO)
+    for (int l = 0; l < n_layers; ++l) ar.take(static_cast<size_t>(B) * r * layers[l].d_out * 2);
   *bytes = ar.off;
   return GRAPE_OK;
 }
@@ -1051,6 +1122,7 @@ void grape_destroy(grape_ctx* ctx) {
   for (void* p : ctx->stage_G) cudaFree(p);
   if (ctx->arena) cudaFree(ctx->arena);
   if (ctx->compact_buf) cudaFree(ctx->compact_buf);
+  if (ctx->rst_buf) cudaFree(ctx->rst_buf);
   for (auto& g : ctx->graphs) ctx->drop_graph(g);
   if (ctx->capture_stream) cudaStreamDestroy(ctx->capture_stream);
   delete ctx;

@@ -19,6 +19,8 @@ struct LayerWs {
   float* m;                // r x d_out  Adam first moment
   float* v;                // r x d_out  Adam second moment
   void* dR;                // r x d_out: fp32 (CUDA-core) / bf16 (tensor-core)
+  __nv_bfloat16* Rst;      // B x r x d_out bf16: every R_i, stored for the aggregation
+                           // (tensor-core path with GRAPE_AGG_STORE; null otherwise)
   int part_base;           // first norm-partial slot of (this layer, sample 0)
   int part_count;          // norm-partial slots per sample of this layer
 };

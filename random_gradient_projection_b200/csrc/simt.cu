@@ -213,88 +213,132 @@ __global__ void __launch_bounds__(kThreads) aggregate_kernel(StepShape sh, Layer
 }
 
 // ---- a6: g = (S + sigma C xi) / batch; Adam in the projected space ----------------
-// xi_l[e] = z(seed, l, s, stream 1, e), e = j*d_out + n.  One thread per block of four
-// consecutive elements (float4 accesses when r*d_out is a multiple of 4; every buffer
-// of the library's arena starts on a 256-byte boundary).
+// xi_l[e] = z(seed, l, s, stream 1, e), e = j*d_out + n.  A thread unit is a block of
+// four consecutive elements of one layer (float4 accesses when the layer's r*d_out is a
+// multiple of 4; every buffer of the library's arena starts on a 256-byte boundary).
+// Units of all layers are numbered back to back (begin[l] .. begin[l+1]) and a grid of a
+// few blocks per SM strides over them, so layers of unequal size keep every SM busy and
+// no block is launched without work.
 //
 // After a programmatic (PDL) launch the aggregation that writes S may still be
 // running, so S is read only after griddepcontrol.wait.  m and v were last written by
 // this kernel in the previous step, and every step begins with an ordinary launch
-// (the generation of P) that waits for all earlier work, so they -- and the noise,
-// which depends on nothing -- are read and drawn before the wait.
-__global__ void __launch_bounds__(256) noise_adam_kernel(StepShape sh, LayerTable tab,
-                                                         UpdateScalars u, int dR_bf16) {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int l = blockIdx.y;
-  const LayerWs& w = tab.ws[l];
-  const int64_t n = static_cast<int64_t>(sh.r) * w.d_out;
-  const int64_t q = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  if (4 * q >= n) return;
-  const bool vec = (n % 4) == 0;
-  const float noise_scale = sh.sigma_C;
-  float xi[4] = {0.f, 0.f, 0.f, 0.f};
-  if (noise_scale != 0.0f) {
-    const float4 z = gaussian4(sh.seed, static_cast<uint32_t>(l), u.step, kStreamNoise,
-                               static_cast<uint32_t>(q));
-    xi[0] = z.x; xi[1] = z.y; xi[2] = z.z; xi[3] = z.w;
-  }
-  float m[4] = {0.f, 0.f, 0.f, 0.f}, v[4] = {0.f, 0.f, 0.f, 0.f}, S[4] = {0.f, 0.f, 0.f, 0.f};
-  const int cnt = static_cast<int>((n - 4 * q) < 4 ? (n - 4 * q) : 4);
-  if (vec) {
-    const float4 m4 = reinterpret_cast<const float4*>(w.m)[q];
-    const float4 v4 = reinterpret_cast<const float4*>(w.v)[q];
-    m[0] = m4.x; m[1] = m4.y; m[2] = m4.z; m[3] = m4.w;
-    v[0] = v4.x; v[1] = v4.y; v[2] = v4.z; v[3] = v4.w;
+// (the generation of P) that waits for all earlier work, so the first unit's m and v --
+// and its noise, which depends on nothing -- are read and drawn before the wait.
+struct AdamTable {
+  float* m[GRAPE_MAX_LAYERS];
+  float* v[GRAPE_MAX_LAYERS];
+  const float* S[GRAPE_MAX_LAYERS];
+  void* dR[GRAPE_MAX_LAYERS];
+  int64_t n[GRAPE_MAX_LAYERS];               // elements r * d_out of each layer
+  int64_t begin[GRAPE_MAX_LAYERS + 1];       // first unit of each layer; begin[L] = total
+};
+
+struct AdamUnit {
+  float m[4], v[4], xi[4];
+  int cnt;      // elements in this unit (4 except a layer's last unit)
+  bool vec;     // float4 accesses
+};
+
+__device__ __forceinline__ void adam_load_mv(const AdamTable& t, int l, int64_t q, AdamUnit& a) {
+  const int64_t n = t.n[l];
+  a.cnt = static_cast<int>((n - 4 * q) < 4 ? (n - 4 * q) : 4);
+  a.vec = (n % 4) == 0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) a.m[k] = a.v[k] = 0.0f;
+  if (a.vec) {
+    const float4 m4 = reinterpret_cast<const float4*>(t.m[l])[q];
+    const float4 v4 = reinterpret_cast<const float4*>(t.v[l])[q];
+    a.m[0] = m4.x; a.m[1] = m4.y; a.m[2] = m4.z; a.m[3] = m4.w;
+    a.v[0] = v4.x; a.v[1] = v4.y; a.v[2] = v4.z; a.v[3] = v4.w;
   } else {
 #pragma unroll
     for (int k = 0; k < 4; ++k)
-      if (k < cnt) {
-        m[k] = w.m[4 * q + k];
-        v[k] = w.v[4 * q + k];
+      if (k < a.cnt) {
+        a.m[k] = t.m[l][4 * q + k];
+        a.v[k] = t.v[l][4 * q + k];
       }
   }
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (vec) {
-    const float4 s4 = reinterpret_cast<const float4*>(w.S)[q];
+}
+
+__device__ __forceinline__ void adam_noise(const StepShape& sh, int l, uint32_t step, int64_t q, AdamUnit& a) {
+  if (sh.sigma_C != 0.0f) {
+    const float4 z = gaussian4(sh.seed, static_cast<uint32_t>(l), step, kStreamNoise, static_cast<uint32_t>(q));
+    a.xi[0] = z.x; a.xi[1] = z.y; a.xi[2] = z.z; a.xi[3] = z.w;
+  } else {
+    a.xi[0] = a.xi[1] = a.xi[2] = a.xi[3] = 0.0f;
+  }
+}
+
+__device__ __forceinline__ void adam_finish(const StepShape& sh, const AdamTable& t, const UpdateScalars& u,
+                                            int dR_bf16, int l, int64_t q, AdamUnit& a) {
+  float S[4] = {0.f, 0.f, 0.f, 0.f};
+  if (a.vec) {
+    const float4 s4 = reinterpret_cast<const float4*>(t.S[l])[q];
     S[0] = s4.x; S[1] = s4.y; S[2] = s4.z; S[3] = s4.w;
   } else {
 #pragma unroll
     for (int k = 0; k < 4; ++k)
-      if (k < cnt) S[k] = w.S[4 * q + k];
+      if (k < a.cnt) S[k] = t.S[l][4 * q + k];
   }
   const float b1 = sh.beta1, b2 = sh.beta2;
   const float ob1 = sh.one_minus_beta1, ob2 = sh.one_minus_beta2;
   float d[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const float g = fmaf(noise_scale, xi[k], S[k]) * u.inv_batch;
-    m[k] = fmaf(b1, m[k], ob1 * g);
-    v[k] = fmaf(b2, v[k], ob2 * g * g);
-    d[k] = (m[k] * u.inv_bc1) / (sqrtf(v[k] * u.inv_bc2) + sh.eps);
+    const float g = fmaf(sh.sigma_C, a.xi[k], S[k]) * u.inv_batch;
+    a.m[k] = fmaf(b1, a.m[k], ob1 * g);
+    a.v[k] = fmaf(b2, a.v[k], ob2 * g * g);
+    d[k] = (a.m[k] * u.inv_bc1) / (sqrtf(a.v[k] * u.inv_bc2) + sh.eps);
   }
-  if (vec) {
-    reinterpret_cast<float4*>(w.m)[q] = make_float4(m[0], m[1], m[2], m[3]);
-    reinterpret_cast<float4*>(w.v)[q] = make_float4(v[0], v[1], v[2], v[3]);
+  if (a.vec) {
+    reinterpret_cast<float4*>(t.m[l])[q] = make_float4(a.m[0], a.m[1], a.m[2], a.m[3]);
+    reinterpret_cast<float4*>(t.v[l])[q] = make_float4(a.v[0], a.v[1], a.v[2], a.v[3]);
     if (dR_bf16) {
       const __nv_bfloat162 lo = __floats2bfloat162_rn(d[0], d[1]);
       const __nv_bfloat162 hi = __floats2bfloat162_rn(d[2], d[3]);
-      reinterpret_cast<uint2*>(w.dR)[q] =
+      reinterpret_cast<uint2*>(t.dR[l])[q] =
           make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
     } else {
-      reinterpret_cast<float4*>(w.dR)[q] = make_float4(d[0], d[1], d[2], d[3]);
+      reinterpret_cast<float4*>(t.dR[l])[q] = make_float4(d[0], d[1], d[2], d[3]);
     }
   } else {
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      if (k >= cnt) continue;
+      if (k >= a.cnt) continue;
       const int64_t e = 4 * q + k;
-      w.m[e] = m[k];
-      w.v[e] = v[k];
+      t.m[l][e] = a.m[k];
+      t.v[l][e] = a.v[k];
       if (dR_bf16)
-        static_cast<__nv_bfloat16*>(w.dR)[e] = __float2bfloat16_rn(d[k]);
+        static_cast<__nv_bfloat16*>(t.dR[l])[e] = __float2bfloat16_rn(d[k]);
       else
-        static_cast<float*>(w.dR)[e] = d[k];
+        static_cast<float*>(t.dR[l])[e] = d[k];
     }
+  }
+}
+
+__global__ void __launch_bounds__(256) noise_adam_kernel(StepShape sh, AdamTable t, UpdateScalars u,
+                                                         int dR_bf16) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int64_t total = t.begin[sh.L];
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t unit = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  int l = 0;
+  AdamUnit a;
+  if (unit < total) {   // the first unit's m, v and noise do not depend on the running kernel
+    while (unit >= t.begin[l + 1]) ++l;
+    adam_load_mv(t, l, unit - t.begin[l], a);
+    adam_noise(sh, l, u.step, unit - t.begin[l], a);
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  for (bool first = true; unit < total; unit += stride, first = false) {
+    while (unit >= t.begin[l + 1]) ++l;   // units only grow, so l only moves forward
+    const int64_t q = unit - t.begin[l];
+    if (!first) {
+      adam_load_mv(t, l, q, a);
+      adam_noise(sh, l, u.step, q, a);
+    }
+    adam_finish(sh, t, u, dR_bf16, l, q, a);
   }
 }
 
@@ -423,11 +467,41 @@ cudaError_t simt_aggregate(const StepShape& sh, const LayerWs* ws, const LayerIo
   return cudaGetLastError();
 }
 
+AdamTable make_adam_table(const StepShape& sh, const LayerWs* ws) {
+  AdamTable t{};
+  int64_t at = 0;
+  for (int l = 0; l < sh.L; ++l) {
+    t.m[l] = ws[l].m;
+    t.v[l] = ws[l].v;
+    t.S[l] = ws[l].S;
+    t.dR[l] = ws[l].dR;
+    t.n[l] = static_cast<int64_t>(sh.r) * ws[l].d_out;
+    t.begin[l] = at;
+    at += (t.n[l] + 3) / 4;
+  }
+  t.begin[sh.L] = at;
+  return t;
+}
+
+// Blocks of the noise + Adam grid: 8 resident 256-thread blocks per SM, never more than
+// there are units.
+unsigned adam_blocks(const AdamTable& t, int L) {
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);   // the current device's SM count (the runtime answers from its cache)
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  const int64_t need = (t.begin[L] + 255) / 256;
+  const int64_t fill = static_cast<int64_t>(sms) * 8;
+  const int64_t b = need < fill ? need : fill;
+  return static_cast<unsigned>(b > 0 ? b : 1);
+}
+
 cudaError_t noise_adam(const StepShape& sh, const LayerWs* ws, const UpdateScalars& u, bool dR_bf16,
                        bool pdl, cudaStream_t st) {
-  const LayerTable t = make_table(sh, ws, nullptr);
-  const int64_t q = (static_cast<int64_t>(sh.r) * max_d_out(sh, ws) + 3) / 4;
-  dim3 grid(cdiv(q, 256), sh.L);   // one thread per four elements (no grid-stride loop)
+  const AdamTable t = make_adam_table(sh, ws);
+  const dim3 grid(adam_blocks(t, sh.L));
   if (!pdl) {
     noise_adam_kernel<<<grid, 256, 0, st>>>(sh, t, u, dR_bf16 ? 1 : 0);
     return cudaGetLastError();
@@ -462,7 +536,7 @@ cudaError_t noise_adam_set_node(cudaGraphExec_t exec, cudaGraphNode_t node, cons
   cudaError_t e = cudaGraphKernelNodeGetParams(node, &p);
   if (e != cudaSuccess) return e;
   StepShape a0 = sh;
-  LayerTable a1 = make_table(sh, ws, nullptr);
+  AdamTable a1 = make_adam_table(sh, ws);
   UpdateScalars a2 = u;
   int a3 = dR_bf16 ? 1 : 0;
   void* args[] = {&a0, &a1, &a2, &a3};

@@ -75,7 +75,8 @@ constexpr int kMaxGroup = 16;      // layers per launch
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr uint64_t kDrainLimitNs = 1000000000ull;   // after an abort: wait for loads in flight
 
-enum Mode : int { PROJECT = 0, NORM = 1, AGGREGATE = 2, BACKPROJ = 3, GHOST = 4 };
+// NORMST: NORM that also stores every tile of R_i (bf16) for the stored aggregation.
+enum Mode : int { PROJECT = 0, NORM = 1, AGGREGATE = 2, BACKPROJ = 3, GHOST = 4, NORMST = 5 };
 
 // error word bits
 constexpr int kErrTimeoutProducer = 1;
@@ -139,8 +140,9 @@ inline void set_ext(int (&e)[3], int64_t x, int64_t y, int64_t z) {
 
 template <int MODE>
 struct ModeTraits {
-  static constexpr bool kAMn = (MODE == NORM || MODE == AGGREGATE);
-  static constexpr bool kB3d = (MODE == NORM);
+  static constexpr bool kNorm = (MODE == NORM || MODE == NORMST);
+  static constexpr bool kAMn = (kNorm || MODE == AGGREGATE);
+  static constexpr bool kB3d = kNorm;
 };
 
 template <int BN, int STAGES, int EXTRA = 0, int BCOLS = BN>
@@ -155,6 +157,8 @@ struct Smem {
   static_assert(kStage % 1024 == 0 && kExtraOff % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 };
 
+// NORMST: one staging box per epilogue warp for its 32 rows x 64 columns of R_i in bf16.
+constexpr int kRBox = 32 * 128;
 // BACKPROJ: two W tiles (128 rows x 128 fp32 columns, as four 128B-swizzled boxes of
 // 32 columns) so the TMA load of the next tile's W overlaps this tile's update.
 constexpr int kBnBack = 128;
@@ -162,7 +166,7 @@ constexpr int kWBox = kBM * 128;                 // one 32-column box: 16 KB
 constexpr int kWTile = (kBnBack / 32) * kWBox;   // 64 KB
 template <int MODE>
 struct ModeExtra {
-  static constexpr int kBytes = (MODE == BACKPROJ) ? 2 * kWTile : 0;
+  static constexpr int kBytes = (MODE == BACKPROJ) ? 2 * kWTile : (MODE == NORMST) ? kEpiWarps * kRBox : 0;
 };
 // GHOST stages hold a single 128-row tile, used as both operands of its Gram product.
 template <int MODE, int BN, int STAGES>
@@ -268,10 +272,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       const int pi = producer_of(warp);
       // A and Gout stream once per use; P, AP and dR are re-read by other tiles or
       // by the next phase, so they are kept in L2 preferentially.
+      // (NORMST: neither AP nor Gout is read again after this kernel, and its R stores
+      // share the cache, so both load with the normal priority)
       const uint64_t polA = (MODE == PROJECT || MODE == AGGREGATE || MODE == BACKPROJ)
                                 ? ptx::policy_evict_first()
-                                : ptx::policy_evict_last();
-      const uint64_t polB = (MODE == AGGREGATE) ? ptx::policy_evict_first() : ptx::policy_evict_last();
+                                : (MODE == NORMST) ? ptx::policy_evict_normal() : ptx::policy_evict_last();
+      const uint64_t polB = (MODE == AGGREGATE) ? ptx::policy_evict_first()
+                            : (MODE == NORMST) ? ptx::policy_evict_normal() : ptx::policy_evict_last();
       auto load_a = [&](const TileCoord& c, int kb, int s) {
         uint8_t* sa = smem + s * S::kStage;
         const CUtensorMap* mapA = &p.mapA[c.g];
@@ -279,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         if (MODE == PROJECT || MODE == BACKPROJ) {
           GRAPE_BOX(p.err, p.extA[c.g], 2, kk, c.m_t * kBM, 0)
           ptx::tma_load_2d_hint(sa, mapA, &full[s], kk, c.m_t * kBM, MODE == BACKPROJ ? polB : polA);
-        } else if (MODE == NORM) {
+        } else if (T::kNorm) {
 #pragma unroll
           for (int q = 0; q < kBM / 64; ++q)
             GRAPE_BOX(p.err, p.extA[c.g], 2, c.m_t * kBM + 64 * q, kk, c.s_t)
@@ -374,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             load_a(c, kb, s);
             ensure_wait();
             load_b(c, kb, s);
-          } else if (MODE == NORM || MODE == AGGREGATE) {
+          } else if (T::kNorm || MODE == AGGREGATE) {
             load_b(c, kb, s);
             ensure_wait();
             load_a(c, kb, s);
@@ -489,14 +496,39 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                                   pack_bf16(v[8 * u + 4], v[8 * u + 5]), pack_bf16(v[8 * u + 6], v[8 * u + 7]));
           }
         }
-      } else if (MODE == NORM) {
+      } else if (T::kNorm) {
+        // ||R_i||^2 partial of this tile.  NORMST also stores the tile of R_i as bf16 to
+        // [sample][r][d_out] (L.out): each warp stages its 32 rows x 64 columns in its own
+        // box (row `lane` at 128-byte row `lane`, 16-byte unit u at u ^ (lane & 7), so the
+        // eight lanes writing one unit hit distinct banks), then writes them out four rows
+        // per instruction, eight lanes per row: whole 128-byte lines, where each thread
+        // storing its own row would scatter 16-byte pieces over 32 lines.
         float ss = 0.0f;
+        uint4* rbox = reinterpret_cast<uint4*>(smem + S::kExtraOff + ew * kRBox);
+        __nv_bfloat16* Rst = static_cast<__nv_bfloat16*>(L.out);
 #pragma unroll 1
         for (int cc = 0; cc < kHalf; cc += 64) {
           float v[64];
           ptx::tmem_ld64(tbase + cc, v);
 #pragma unroll
           for (int j = 0; j < 64; ++j) ss = fmaf(v[j], v[j], ss);
+          if (MODE == NORMST && have) {
+            __syncwarp();   // the previous chunk's rows have been read out of the box
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              rbox[lane * 8 + (u ^ (lane & 7))] =
+                  make_uint4(pack_bf16(v[8 * u + 0], v[8 * u + 1]), pack_bf16(v[8 * u + 2], v[8 * u + 3]),
+                             pack_bf16(v[8 * u + 4], v[8 * u + 5]), pack_bf16(v[8 * u + 6], v[8 * u + 7]));
+            __syncwarp();
+            const int u = lane & 7;
+            __nv_bfloat16* base = Rst + (static_cast<size_t>(c.s_t) * L.M + c.m_t * kBM + q * 32) * L.ldo +
+                                  col0 + cc + 8 * u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int rr = 4 * i + (lane >> 3);
+              *reinterpret_cast<uint4*>(base + static_cast<size_t>(rr) * L.ldo) = rbox[rr * 8 + (u ^ (rr & 7))];
+            }
+          }
         }
         if (!have) ss = 0.0f;
 #pragma unroll
@@ -801,22 +833,28 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
 }
 
 // ---- P_l in bf16, row-major d_in x r: element e = k*r + j ----------------------------
+// A thread unit is Philox block q of one layer (elements 4q .. 4q+3); the units of all
+// layers are numbered back to back (begin[l] .. begin[l+1]) and a grid of a few blocks
+// per SM strides over them, so layers of unequal size keep every SM busy.
 struct PTable {
   __nv_bfloat16* P16[GRAPE_MAX_LAYERS];
-  int d_in[GRAPE_MAX_LAYERS];
+  int64_t begin[GRAPE_MAX_LAYERS + 1];   // first unit of each layer; begin[L] = total
+  int L;
 };
 
 __global__ void __launch_bounds__(256) gen_P_bf16_kernel(PTable t, uint64_t seed, uint32_t step, int r) {
   ptx::griddep_launch_dependents();
-  const int l = blockIdx.y;
-  const int64_t nq = static_cast<int64_t>(t.d_in[l]) * r / 4;   // r is a multiple of 64
   const float scale = rsqrtf(static_cast<float>(r));
-  uint2* out = reinterpret_cast<uint2*>(t.P16[l]);
-  for (int64_t q = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; q < nq;
-       q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+  const int64_t total = t.begin[t.L];
+  int l = 0;
+  for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < total;
+       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    while (u >= t.begin[l + 1]) ++l;   // u only grows, so l only moves forward
+    const int64_t q = u - t.begin[l];
     const float4 z = gaussian4(seed, static_cast<uint32_t>(l), step, kStreamProjection,
                                static_cast<uint32_t>(q));
-    out[q] = make_uint2(pack_bf16(z.x * scale, z.y * scale), pack_bf16(z.z * scale, z.w * scale));
+    reinterpret_cast<uint2*>(t.P16[l])[q] =
+        make_uint2(pack_bf16(z.x * scale, z.y * scale), pack_bf16(z.z * scale, z.w * scale));
   }
 }
 
@@ -831,7 +869,8 @@ struct ApTable {
 };
 
 __global__ void __launch_bounds__(256) clip_scale_kernel(ApTable t, int r, int T, int part_stride, float C,
-                                                         const float* partials, float* norms, float* clip) {
+                                                         const float* partials, float* norms, float* clip,
+                                                         int rescale) {
   __shared__ float red[8];
   __shared__ float c_sh;
   ptx::griddep_launch_dependents();
@@ -857,7 +896,7 @@ __global__ void __launch_bounds__(256) clip_scale_kernel(ApTable t, int r, int T
   }
   __syncthreads();
   const float c = c_sh;
-  if (c == 1.0f) return;
+  if (c == 1.0f || !rescale) return;
   uint4* rows = reinterpret_cast<uint4*>(t.AP[l] + static_cast<size_t>(i) * T * r);
   const size_t n8 = static_cast<size_t>(T) * r / 8;   // 8 bf16 per 16-byte vector
   constexpr int kBatch = 8;                            // loads in flight per thread
@@ -880,6 +919,59 @@ __global__ void __launch_bounds__(256) clip_scale_kernel(ApTable t, int r, int T
       }
       rows[k] = x[u];
     }
+  }
+}
+
+// ---- S_l = sum_i c_i R_i over the R_i the norm kernel stored ------------------------
+// The stored variant of the aggregation: every R_{i,l} (r x d_out) was written as bf16
+// by the norm kernel to [sample][r][d_out], so S is a c-weighted sum of B streams, an
+// HBM-bound pass over B*r*d_out*2 bytes instead of a second contraction over the B*T
+// stacked rows.  Thread unit u covers 8 consecutive elements of one layer (16 bytes per
+// sample); units of all layers are numbered back to back (begin[l] .. begin[l+1]) so
+// the grid covers layers of unequal size evenly.  Samples are summed in order 0..B-1
+// with fmaf, so the result does not depend on timing.
+struct StoredAggTable {
+  const __nv_bfloat16* R[GRAPE_MAX_LAYERS];   // [B][r][d_out] bf16
+  float* S[GRAPE_MAX_LAYERS];                  // [r][d_out] fp32
+  int64_t begin[GRAPE_MAX_LAYERS + 1];         // first unit of each layer; begin[L] = total
+};
+
+__device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4& x, float c) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __bfloat1622float2(h[e]);
+    acc[2 * e] = fmaf(c, f.x, acc[2 * e]);
+    acc[2 * e + 1] = fmaf(c, f.y, acc[2 * e + 1]);
+  }
+}
+
+__global__ void __launch_bounds__(256) aggregate_stored_kernel(StoredAggTable t, int L, int B,
+                                                               const float* clip) {
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();   // R_i from the norm kernel, c_i from the clip kernel
+  const int64_t total = t.begin[L];
+  int l = 0;
+  for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < total;
+       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    while (u >= t.begin[l + 1]) ++l;   // u only grows, so l only moves forward
+    const int64_t e = u - t.begin[l];                       // unit within the layer
+    const int64_t n8 = t.begin[l + 1] - t.begin[l];         // units per sample
+    const uint4* R = reinterpret_cast<const uint4*>(t.R[l]) + e;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    constexpr int kBatch = 8;   // loads in flight per thread
+    int i = 0;
+    for (; i + kBatch <= B; i += kBatch) {
+      uint4 x[kBatch];
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) x[k] = __ldcs(R + static_cast<int64_t>(i + k) * n8);
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) acc_bf16x8(acc, x[k], __ldg(clip + i + k));
+    }
+    for (; i < B; ++i) acc_bf16x8(acc, __ldcs(R + static_cast<int64_t>(i) * n8), __ldg(clip + i));
+    float4* S = reinterpret_cast<float4*>(t.S[l]) + 2 * e;
+    S[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    S[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
 }
 
@@ -914,13 +1006,13 @@ bool map_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint3
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// fp32 row-major [rows][cols] as a 2-D map with a (32 x 128) box, 128-byte swizzle.
-bool map_2d_f32(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
+// fp32 row-major [rows][cols] as a 2-D map with a (32 x box_rows) box, 128-byte swizzle.
+bool map_2d_f32(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows = kBM) {
   auto enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 4};
-  cuuint32_t box[2] = {32, kBM};
+  cuuint32_t box[2] = {32, box_rows};
   cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1211,19 +1303,29 @@ int* tc_error_word(const TcWorkspace& tc) {
   return tc.host_state ? static_cast<HostState*>(tc.host_state)->err : nullptr;
 }
 
-cudaError_t tc_generate_P(const StepShape& sh, const LayerWs* ws, const TcWorkspace&, uint32_t step,
-                          cudaStream_t st, int* launches) {
+namespace {
+PTable make_p_table(const StepShape& sh, const LayerWs* ws) {
   PTable t{};
-  int64_t most = 0;
+  int64_t at = 0;
   for (int l = 0; l < sh.L; ++l) {
     t.P16[l] = ws[l].P16;
-    t.d_in[l] = ws[l].d_in;
-    const int64_t q = static_cast<int64_t>(ws[l].d_in) * sh.r / 4;
-    most = q > most ? q : most;
+    t.begin[l] = at;
+    at += static_cast<int64_t>(ws[l].d_in) * sh.r / 4;   // r is a multiple of 64
   }
-  int gx = cdiv(most, 256);
-  gx = gx < 1184 ? gx : 1184;
-  gen_P_bf16_kernel<<<dim3(gx, sh.L), 256, 0, st>>>(t, sh.seed, step, sh.r);
+  t.begin[sh.L] = at;
+  t.L = sh.L;
+  return t;
+}
+}  // namespace
+
+cudaError_t tc_generate_P(const StepShape& sh, const LayerWs* ws, const TcWorkspace&, uint32_t step,
+                          cudaStream_t st, int* launches) {
+  const PTable t = make_p_table(sh, ws);
+  // 8 resident 256-thread blocks per SM, never more than there are units
+  int64_t gx = (t.begin[sh.L] + 255) / 256;
+  const int64_t fill = static_cast<int64_t>(sm_count()) * 8;
+  gx = gx < fill ? gx : fill;
+  gen_P_bf16_kernel<<<static_cast<unsigned>(gx > 0 ? gx : 1), 256, 0, st>>>(t, sh.seed, step, sh.r);
   ++*launches;
   return cudaGetLastError();
 }
@@ -1235,11 +1337,7 @@ cudaError_t tc_generate_P_set_node(cudaGraphExec_t exec, cudaGraphNode_t node, c
   cudaKernelNodeParams p{};
   cudaError_t e = cudaGraphKernelNodeGetParams(node, &p);
   if (e != cudaSuccess) return e;
-  PTable a0{};
-  for (int l = 0; l < sh.L; ++l) {
-    a0.P16[l] = ws[l].P16;
-    a0.d_in[l] = ws[l].d_in;
-  }
+  PTable a0 = make_p_table(sh, ws);
   uint64_t a1 = sh.seed;
   uint32_t a2 = key;
   int a3 = sh.r;
@@ -1282,7 +1380,8 @@ cudaError_t tc_project(const StepShape& sh, const LayerWs* ws, const LayerIo* io
 }
 
 cudaError_t tc_project_norm(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
-                            const TcWorkspace& tc, float* partials, cudaStream_t st, int* launches) {
+                            const TcWorkspace& tc, float* partials, bool store_R, cudaStream_t st,
+                            int* launches) {
   HostState& hs = *static_cast<HostState*>(tc.host_state);
   GroupParams& gp = hs.gp;
   std::memset(&gp, 0, sizeof(gp));
@@ -1295,6 +1394,7 @@ cudaError_t tc_project_norm(const StepShape& sh, const LayerWs* ws, const LayerI
           return map_3d(m, io[l].G, sh.B, sh.T, ws[l].d_out);
         }))
       return false;
+    if (store_R && !ws[l].Rst) return false;
     GRAPE_EXT(gp.extA[g], sh.r, sh.T, sh.B)
     GRAPE_EXT(gp.extB[g], ws[l].d_out, sh.T, sh.B)
     GroupLayer& L = gp.lay[g];
@@ -1305,9 +1405,12 @@ cudaError_t tc_project_norm(const StepShape& sh, const LayerWs* ws, const LayerI
     L.M = sh.r;
     L.N = ws[l].d_out;
     L.part_base = ws[l].part_base;
+    L.out = store_R ? ws[l].Rst : nullptr;   // R_l as [B][r][d_out] bf16
+    L.ldo = ws[l].d_out;
     *tiles = L.mt * L.nt * sh.B;
     return true;
   };
+  if (store_R) return run_mode<NORMST, kBnWide, kStagesNorm>(hs, sh.L, st, launches, fill, gp);
   return run_mode<NORM, kBnWide, kStagesNorm>(hs, sh.L, st, launches, fill, gp);
 }
 
@@ -1349,13 +1452,34 @@ cudaError_t tc_project_norm_ghost(const StepShape& sh, const LayerWs* ws, const 
 }
 
 cudaError_t tc_clip_scale(const StepShape& sh, const LayerWs* ws, const TcWorkspace&,
-                          const float* partials, float* norms, float* clip, cudaStream_t st,
-                          int* launches) {
+                          const float* partials, float* norms, float* clip, bool rescale_ap,
+                          cudaStream_t st, int* launches) {
   ApTable t{};
   for (int l = 0; l < sh.L; ++l) t.AP[l] = static_cast<__nv_bfloat16*>(ws[l].AP);
   ++*launches;
-  return launch_pdl(clip_scale_kernel, dim3(sh.B, sh.L), dim3(256), 0, st, t, sh.r, sh.T, sh.part_stride,
-                    sh.C, partials, norms, clip);
+  return launch_pdl(clip_scale_kernel, dim3(sh.B, rescale_ap ? sh.L : 1), dim3(256), 0, st, t, sh.r, sh.T,
+                    sh.part_stride, sh.C, partials, norms, clip, rescale_ap ? 1 : 0);
+}
+
+cudaError_t tc_aggregate_stored(const StepShape& sh, const LayerWs* ws, const float* clip, cudaStream_t st,
+                                int* launches) {
+  StoredAggTable t{};
+  int64_t at = 0;
+  for (int l = 0; l < sh.L; ++l) {
+    if (!ws[l].Rst) return cudaErrorInvalidValue;
+    t.R[l] = ws[l].Rst;
+    t.S[l] = ws[l].S;
+    t.begin[l] = at;
+    at += static_cast<int64_t>(sh.r) * ws[l].d_out / 8;   // d_out % 256 == 0 on this path
+  }
+  t.begin[sh.L] = at;
+  // enough 256-thread blocks to fill every SM (8 per SM), never more than there are units
+  int64_t blocks = (at + 255) / 256;
+  const int64_t fill = static_cast<int64_t>(sm_count()) * 8;
+  blocks = blocks < fill ? blocks : fill;
+  ++*launches;
+  return launch_pdl(aggregate_stored_kernel, dim3(static_cast<unsigned>(blocks > 0 ? blocks : 1)), dim3(256), 0,
+                    st, t, sh.L, sh.B, clip);
 }
 
 namespace {

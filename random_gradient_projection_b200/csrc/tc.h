@@ -51,13 +51,20 @@ cudaError_t tc_project(const StepShape& sh, const LayerWs* ws, const LayerIo* io
 bool tc_ghost_supported(const StepShape& sh);
 cudaError_t tc_project_norm_ghost(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                                   const TcWorkspace& tc, float* partials, cudaStream_t st, int* launches);
+// store_R: also write every R_i (bf16) to ws[l].Rst for tc_aggregate_stored.
 cudaError_t tc_project_norm(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
-                            const TcWorkspace& tc, float* partials, cudaStream_t st, int* launches);
+                            const TcWorkspace& tc, float* partials, bool store_R, cudaStream_t st,
+                            int* launches);
+// n_i and c_i; with rescale_ap, AP is also scaled in place by c_i for tc_aggregate.
 cudaError_t tc_clip_scale(const StepShape& sh, const LayerWs* ws, const TcWorkspace& tc,
-                          const float* partials, float* norms, float* clip, cudaStream_t st,
-                          int* launches);
+                          const float* partials, float* norms, float* clip, bool rescale_ap,
+                          cudaStream_t st, int* launches);
+// S = (diag(c) AP)^T Gout over the stacked rows (AP already scaled by c).
 cudaError_t tc_aggregate(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                          const TcWorkspace& tc, const float* clip, cudaStream_t st, int* launches);
+// S = sum_i c_i R_i over the R_i stored by tc_project_norm(store_R = true).
+cudaError_t tc_aggregate_stored(const StepShape& sh, const LayerWs* ws, const float* clip, cudaStream_t st,
+                                int* launches);
 cudaError_t tc_backproject(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                            const TcWorkspace& tc, float lr, cudaStream_t st, int* launches);
 

@@ -34,8 +34,10 @@ EXPORTS = (
     "grape_launch_count", "grape_layer_sqnorms_static", "grape_set_refresh_period", "grape_sqnorms",
     "grape_enable_compaction", "grape_step_masked", "grape_live_counts", "grape_set_norm_method",
     "grape_set_graph", "grape_selftest_wait_timeout", "grape_S_all", "grape_context_bytes",
+    "grape_set_aggregation", "grape_aggregation_of",
 )
 GRAPE_NORM_DIRECT, GRAPE_NORM_GHOST = 0, 1
+GRAPE_AGG_AUTO, GRAPE_AGG_RECOMPUTE, GRAPE_AGG_STORE = 0, 1, 2
 PHASES = ("gen_P", "project", "norm", "clip", "aggregate", "adam", "backproject", "compact")   # GRAPE_N_PHASES
 
 
@@ -93,6 +95,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "grape_set_graph": ([vp, i32], i32),
         "grape_selftest_wait_timeout": ([i64, i64, ctypes.POINTER(i32)], i32),
         "grape_S_all": ([vp, ctypes.POINTER(vp), ctypes.POINTER(i64)], i32),
+        "grape_set_aggregation": ([vp, i32], i32),
+        "grape_aggregation_of": ([vp, ctypes.POINTER(i32)], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -191,6 +195,16 @@ def grape_set_graph(ctx: int, enable: bool):
 
 def grape_set_norm_method(ctx: int, method: int):
     _check(lib().grape_set_norm_method(ctx, method), ctx)
+
+
+def grape_set_aggregation(ctx: int, method: int):
+    _check(lib().grape_set_aggregation(ctx, method), ctx)
+
+
+def grape_aggregation_of(ctx: int) -> int:
+    out = ctypes.c_int32()
+    _check(lib().grape_aggregation_of(ctx, ctypes.byref(out)), ctx)
+    return out.value
 
 
 def grape_enable_compaction(ctx: int, T_full: int):
@@ -376,6 +390,15 @@ class GrapeStep:
     def set_norm_method(self, method: int):
         """GRAPE_NORM_DIRECT (default) or GRAPE_NORM_GHOST (tensor-core path, T <= 128)."""
         grape_set_norm_method(self.ctx, method)
+
+    def set_aggregation(self, method: int):
+        """GRAPE_AGG_AUTO (the default), GRAPE_AGG_RECOMPUTE or GRAPE_AGG_STORE."""
+        grape_set_aggregation(self.ctx, method)
+
+    @property
+    def aggregation(self) -> int:
+        """The aggregation the next step uses: GRAPE_AGG_RECOMPUTE or GRAPE_AGG_STORE."""
+        return grape_aggregation_of(self.ctx)
 
     def enable_compaction(self, T_full: int):
         """Inputs of T_full tokens per sample, compacted to this context's T kept tokens."""

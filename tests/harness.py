@@ -39,11 +39,14 @@ def snapshot(g, n_layers: int) -> dict:
             "dR": [g.dR(l) for l in range(n_layers)]}
 
 
-def run_library(w, steps: int, path: int, capture=True):
-    """Run ``steps`` steps through the C ABI; return per-step intermediates and final state."""
+def run_library(w, steps: int, path: int, capture=True, setup=None):
+    """Run ``steps`` steps through the C ABI; return per-step intermediates and final state.
+    ``setup(g)`` configures the context before the first step."""
     import torch
     from random_gradient_projection_b200 import GrapeStep
     g = GrapeStep.for_workload(w, path=path)
+    if setup:
+        setup(g)
     Ws = [torch.from_numpy(x).cuda() for x in W.make_weights(w)]
     trace = []
     for s in range(steps):

@@ -133,6 +133,19 @@ def test_context_bytes_is_the_documented_arena(lib):
     assert tiny == 1024 + 2048 + 2048 + 1024 + 1024 + 1024 + 3 * 256
 
 
+def test_context_bytes_counts_the_stored_R_i_when_auto_chooses_them(lib):
+    """GRAPE_AGG_AUTO stores every R_i (B x r x d_out bf16) on the tensor-core path from
+    T = 256 tokens per sample: one more token adds B r 2 bytes of AP and the store's
+    B r d_out 2 bytes; the CUDA-core path never stores."""
+    from random_gradient_projection_b200 import grape
+    a = grape.grape_context_bytes([(1024, 1024)], 128, 4, 255, grape.GRAPE_BF16)
+    b = grape.grape_context_bytes([(1024, 1024)], 128, 4, 256, grape.GRAPE_BF16)
+    assert b - a == 4 * 128 * 2 + 4 * 128 * 1024 * 2
+    c = grape.grape_context_bytes([(1024, 1024)], 128, 4, 255, grape.GRAPE_BF16, grape.GRAPE_PATH_SIMT)
+    d = grape.grape_context_bytes([(1024, 1024)], 128, 4, 256, grape.GRAPE_BF16, grape.GRAPE_PATH_SIMT)
+    assert d - c == 4 * 128 * 4
+
+
 def test_context_bytes_grows_with_r_times_d_out_not_d_in_times_d_out(lib):
     """Optimizer state is O(r x layers): doubling d_in changes only P (d_in r), never the
     moments; the moments alone are 8 r d_out per layer."""

@@ -104,6 +104,48 @@ def test_step_matches_oracle(case, path):
     print(case, "tc" if path == TC else "simt", {k: f"{v:.2e}" for k, v in worst.items()})
 
 
+STORE_CASES = ["mlp_2x1024_B4", "vit_qkv_down_B3", "longctx_1layer_T1000", "r512_T130", "20_layers",
+               "ragged_d_in_tc", "T1_bf16_tc", "no_noise_bf16"]
+
+
+@pytest.mark.parametrize("case", STORE_CASES)
+@pytest.mark.parametrize("agg", [grape.GRAPE_AGG_STORE, grape.GRAPE_AGG_RECOMPUTE], ids=["store", "recompute"])
+def test_aggregation_methods_match_oracle(case, agg):
+    """Both aggregations, forced whatever GRAPE_AGG_AUTO would pick for the shape: S from
+    the R_i the norm kernel stored (bf16), and S from the second contraction over the
+    stacked rows, each against the oracle's sum of the clipped R_i."""
+    w, steps = CASES[case]
+    lib = run_library(w, steps, TC, setup=lambda g: g.set_aggregation(agg))
+    orc = run_oracle(w, steps)
+    worst = compare(w, lib, orc, 2e-2, steps)
+    print(case, "store" if agg == grape.GRAPE_AGG_STORE else "recompute",
+          {k: f"{v:.2e}" for k, v in worst.items()})
+
+
+def test_auto_aggregation_follows_tokens_per_sample():
+    """AUTO stores R_i from T = 256 tokens per sample on; the ghost norm forms no R_i and
+    so recomputes; the CUDA-core path refuses STORE."""
+    base = W.Workload("agg_auto", ((256, 256),), r=128, B=2, T=255, dtype="bf16", C=1.0,
+                      sigma=1.0, steps=1)
+    g = GrapeStep.for_workload(base, path=TC)
+    assert g.aggregation == grape.GRAPE_AGG_RECOMPUTE
+    g.close()
+    g = GrapeStep.for_workload(base.replace(T=256), path=TC)
+    assert g.aggregation == grape.GRAPE_AGG_STORE
+    g.close()
+    g = GrapeStep.for_workload(base.replace(T=64), path=TC)
+    g.set_aggregation(grape.GRAPE_AGG_STORE)
+    assert g.aggregation == grape.GRAPE_AGG_STORE
+    g.set_norm_method(grape.GRAPE_NORM_GHOST)
+    assert g.aggregation == grape.GRAPE_AGG_RECOMPUTE
+    g.close()
+    g = GrapeStep.for_workload(base, path=SIMT)
+    with pytest.raises(GrapeError) as e:
+        g.set_aggregation(grape.GRAPE_AGG_STORE)
+    assert e.value.code == grape.GRAPE_EUNSUPPORTED
+    g.close()
+
+
 def test_bench_workload_full_size_tc():
     """The benchmarked workload (4 x 1024^2, r = 128, B = 64, T = 128) at full size on the
     tensor-core path, two steps, against the oracle on the whole batch."""
