@@ -37,6 +37,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <array>
 #include <cstdint>
 #include <cstdio>
@@ -651,6 +652,414 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   }
 }
 
+// ---- back-projection with P resident in tensor memory -------------------------------
+// W -= lr P dR in tiles of 128 rows x 128 columns of W with K = r, with the A operand
+// (the 128 x r block of P under the tile) read by the MMA from TMEM instead of shared
+// memory.  The layers of a launch are cut into consecutive spans of at least four
+// tiles per CTA (a single layer when it is that large).  Span by span, each CTA takes a
+// contiguous range of the span's T tiles (numbered layer by layer, row block by row
+// block): T / grid of them, one more for T % grid of the CTAs, with the CTAs that take
+// the extra tile rotating from span to span, so the whole launch is balanced to within
+// one tile and all CTAs work on the same span at once (its P and dR stay in L2).  A work unit is the part of a CTA's range in one
+// 128-row block: the block of P is written into TMEM once per unit, and per tile only
+// dR (r x 128 bf16, from L2) and W (from DRAM) stream through shared memory, which
+// holds nothing but those streams.  Next to
+// tc_gemm_kernel<BACKPROJ>, which loads P with every tile, this moves 192 instead of
+// 320 bytes from L2 into the SM per 64 bytes of W read, with the same bytes in flight.
+//
+// W streams through a ring of 32-column boxes (128 rows x 32 fp32, 16 KB) that runs
+// ahead of the tiles; each epilogue warp updates its 32 rows of a box in shared memory
+// and stores them with a TMA tile store; a box's slot is reloaded once its four row
+// quarters have been read out.
+//
+// TMEM: two 128 x 128 fp32 accumulators (columns 0..255) and NPB P blocks of r/2
+// columns each (lane = row of P, two bf16 of consecutive k per 32-bit column).
+// Warps: 0 loads dR (written earlier in the step, after griddepcontrol.wait); 1 owns TMEM
+// and issues the MMAs; 2-9 are the epilogue (warp w: lane quarter w % 4, column half
+// (w - 2) / 4); 10 loads W (written by the previous step, whose work every step's first,
+// ordinary launch waits for, so its loads start at once); 11-14 write P into TMEM (warp
+// w: lane quarter w % 4, one row of P per thread, read from global memory).
+struct BptLayer {
+  int tiles_begin;   // first tile of this layer in its span
+  int M;             // rows of W and of P (d_in)
+  int mt, nt;        // 128-row blocks of W, 128-column tiles of W
+  const __nv_bfloat16* P;   // d_in x r, row-major
+};
+
+struct BptParams {
+  CUtensorMap mapDR[kMaxGroup];   // dR: bf16 r x d_out, boxes of 64 x 64
+  CUtensorMap mapW[kMaxGroup];    // W: fp32 d_in x d_out, load boxes of 32 columns x 128 rows
+  CUtensorMap mapWs[kMaxGroup];   // W, store boxes of 32 columns x 32 rows
+  BptLayer lay[kMaxGroup];
+  int n_layers;
+  int n_spans;
+  int span_first[kMaxGroup + 1];   // first layer of each span; span_first[n_spans] = n_layers
+  int span_tiles[kMaxGroup];
+  int span_rot[kMaxGroup];         // CTA b takes the range of position (b + rot) % grid
+  int r;
+  float lr;
+  int* err;
+#ifdef GRAPE_CHECKED
+  int extDR[kMaxGroup][3];
+  int extW[kMaxGroup][3];
+#endif
+};
+
+struct BptUnit {
+  int g, m_t, n0, n1;   // layer in the launch, row block, tiles [n0, n1)
+};
+
+// This CTA's units in order: span by span, its range of the span's tiles cut at the
+// ends of layers and of row blocks.
+struct BptWalk {
+  int sp, g, cur, t1;   // span, layer, next tile of the span, end of this CTA's range in it
+  __device__ __forceinline__ void range(const BptParams& p) {
+    const int T = p.span_tiles[sp];
+    const int G = static_cast<int>(gridDim.x);
+    const int base = T / G, extra = T % G;
+    const int b = (static_cast<int>(blockIdx.x) + p.span_rot[sp]) % G;
+    cur = b * base + min(b, extra);
+    t1 = cur + base + (b < extra ? 1 : 0);
+    g = p.span_first[sp];
+  }
+  __device__ __forceinline__ void start(const BptParams& p) {
+    sp = 0;
+    range(p);
+  }
+  // The next unit; false when the CTA has none left.
+  __device__ __forceinline__ bool next(const BptParams& p, BptUnit& x) {
+    while (cur >= t1) {
+      if (++sp >= p.n_spans) return false;
+      range(p);
+    }
+    while (g + 1 < p.span_first[sp + 1] && cur >= p.lay[g + 1].tiles_begin) ++g;
+    const BptLayer& L = p.lay[g];
+    const int t = cur - L.tiles_begin;
+    x.g = g;
+    x.m_t = t / L.nt;
+    x.n0 = t % L.nt;
+    x.n1 = min(L.nt, x.n0 + (t1 - cur));
+    cur += x.n1 - x.n0;
+    return true;
+  }
+};
+
+// DRS dR stages and NW W boxes in shared memory.
+template <int DRS, int NW>
+struct BptSmem {
+  static constexpr int kDRStage = kBK * kBnBack * 2;        // 64 x 128 bf16: 16 KB
+  static constexpr int kDROff = 0;
+  static constexpr int kWOff = DRS * kDRStage;
+  static constexpr int kBarOff = kWOff + NW * kWBox;
+  static constexpr int kBytes = kBarOff + 512 + 1024;       // barriers + alignment slack
+  static_assert(kBytes <= 232448, "exceeds the shared memory of a CTA");
+};
+constexpr int kBptThreads = 32 * 15;
+constexpr int kBptWProducer = 10;
+constexpr int kBptPWriter0 = 11;    // warps 11..14
+constexpr uint32_t kBptTmemCols = 512;
+constexpr int kBptDRS = 6;
+constexpr int kBptNW = 8;
+
+// PK = r / 64 k-blocks, NPB P blocks in TMEM (PK * 32 columns each).
+template <int PK, int NPB>
+__global__ void __launch_bounds__(kBptThreads, 1) tc_backproj_tmem_kernel(const __grid_constant__ BptParams p) {
+  constexpr int DRS = kBptDRS, NW = kBptNW;
+  using S = BptSmem<DRS, NW>;
+  constexpr uint32_t kIdesc = ptx::idesc_bf16(kBM, kBnBack, false, true);   // A K-major (TMEM), dR N-major
+  constexpr int kBoxes = kBnBack / 32;                                     // W boxes per tile
+  constexpr uint32_t kPCols = PK * 32;                                     // TMEM columns of one P block
+  static_assert(2 * kBnBack + NPB * kPCols <= kBptTmemCols, "TMEM columns");
+  static_assert((2 * NPB + 2 * DRS + 4 + 2 * NW) * 8 + 16 <= 512, "barrier area");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* pfull = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
+  uint64_t* pempty = pfull + NPB;
+  uint64_t* full = pempty + NPB;
+  uint64_t* empty = full + DRS;
+  uint64_t* accfull = empty + DRS;     // [2]
+  uint64_t* accempty = accfull + 2;    // [2]
+  uint64_t* wfull = accempty + 2;      // [NW]
+  uint64_t* wfree = wfull + NW;        // [NW]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wfree + NW);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto wait = [&](uint64_t* bar, uint32_t parity) {
+    return ptx::mbar_wait_or_abort(bar, parity, kWaitLimitNs, abort_flag);
+  };
+  ptx::griddep_launch_dependents();
+
+  if (warp == 0 && lane == 0) {
+    *abort_flag = 0;
+    for (int b = 0; b < NPB; ++b) {
+      ptx::mbar_init(&pfull[b], 4);    // the four P-writing warps
+      ptx::mbar_init(&pempty[b], 1);
+    }
+    for (int st = 0; st < DRS; ++st) {
+      ptx::mbar_init(&full[st], 1);
+      ptx::mbar_init(&empty[st], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&accfull[b], 1);
+      ptx::mbar_init(&accempty[b], kEpiWarps);
+    }
+    for (int sl = 0; sl < NW; ++sl) {
+      ptx::mbar_init(&wfull[sl], 1);
+      ptx::mbar_init(&wfree[sl], 4);   // the four row quarters of a box
+    }
+    ptx::fence_mbar_init();
+    for (int g = 0; g < p.n_layers; ++g) {
+      ptx::prefetch_tmap(&p.mapDR[g]);
+      ptx::prefetch_tmap(&p.mapW[g]);
+      ptx::prefetch_tmap(&p.mapWs[g]);
+    }
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, kBptTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_p = tmem + 2 * kBnBack;   // P blocks after the two accumulators
+
+  if (warp == 0) {
+    // ---------------- dR ----------------
+    if (lane == 0) {
+      const uint64_t pol = ptx::policy_evict_last();   // dR is read by every row block
+      ptx::griddep_wait();
+      uint32_t it = 0, it_issued = 0;
+      bool ok = true;
+      BptWalk walk;
+      walk.start(p);
+      BptUnit x;
+      while (ok && walk.next(p, x)) {
+        for (int n = x.n0; ok && n < x.n1; ++n) {
+#pragma unroll 1
+          for (int kb = 0; kb < PK; ++kb, ++it) {
+            const int st = it % DRS;
+            const uint32_t use = it / DRS;
+            if (use > 0 && !wait(&empty[st], (use - 1) & 1)) {
+              atomicOr(p.err, kErrTimeoutProducer);
+              ok = false;
+              break;
+            }
+            uint8_t* ddst = smem + S::kDROff + st * S::kDRStage;
+            ptx::mbar_arrive_expect_tx(&full[st], S::kDRStage);
+#pragma unroll
+            for (int h = 0; h < kBnBack / 64; ++h)
+              GRAPE_BOX(p.err, p.extDR[x.g], 2, n * kBnBack + 64 * h, kb * kBK, 0)
+              ptx::tma_load_2d_hint(ddst + h * 8192, &p.mapDR[x.g], &full[st], n * kBnBack + 64 * h, kb * kBK, pol);
+            it_issued = it + 1;
+          }
+        }
+      }
+      if (*abort_flag)   // leave none of this thread's loads in flight into shared memory
+        for (uint32_t k = it_issued > DRS ? it_issued - DRS : 0; k < it_issued; ++k)
+          ptx::mbar_wait(&full[k % DRS], (k / DRS) & 1, kDrainLimitNs);
+    }
+  } else if (warp == kBptWProducer) {
+    // ---------------- W boxes ----------------
+    if (lane == 0) {
+      const uint64_t pol = ptx::policy_evict_first();
+      uint32_t wi = 0, w_issued = 0;
+      bool ok = true;
+      BptWalk walk;
+      walk.start(p);
+      BptUnit x;
+      while (ok && walk.next(p, x)) {
+        for (int n = x.n0; ok && n < x.n1; ++n) {
+#pragma unroll 1
+          for (int j = 0; j < kBoxes; ++j, ++wi) {
+            const int sl = wi % NW;
+            const uint32_t use = wi / NW;
+            if (use > 0 && !wait(&wfree[sl], (use - 1) & 1)) {
+              atomicOr(p.err, kErrTimeoutProducer);
+              ok = false;
+              break;
+            }
+            ptx::mbar_arrive_expect_tx(&wfull[sl], kWBox);
+            GRAPE_BOX(p.err, p.extW[x.g], 4, n * kBnBack + 32 * j, x.m_t * kBM, 0)
+            ptx::tma_load_2d_hint(smem + S::kWOff + sl * kWBox, &p.mapW[x.g], &wfull[sl], n * kBnBack + 32 * j,
+                                  x.m_t * kBM, pol);
+            w_issued = wi + 1;
+          }
+        }
+      }
+      if (*abort_flag)
+        for (uint32_t k = w_issued > NW ? w_issued - NW : 0; k < w_issued; ++k)
+          ptx::mbar_wait(&wfull[k % NW], (k / NW) & 1, kDrainLimitNs);
+    }
+  } else if (warp >= kBptPWriter0) {
+    // ---------------- P into TMEM: one row of the block per thread ----------------
+    const int q = warp & 3;                       // TMEM lanes 32q .. 32q+31
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    ptx::griddep_wait();                          // P is generated earlier in this step
+    uint32_t ui = 0;
+    BptWalk walk;
+    walk.start(p);
+    BptUnit x;
+    for (; walk.next(p, x); ++ui) {
+      const BptLayer& L = p.lay[x.g];
+      const int pb = ui % NPB;
+      const uint32_t puse = ui / NPB;
+      if (puse > 0 && !wait(&pempty[pb], (puse - 1) & 1)) {
+        atomicOr(p.err, kErrTimeoutProducer);
+        break;
+      }
+      ptx::tc_fence_after();
+      const int m = x.m_t * kBM + q * 32 + lane;
+      const bool valid = m < L.M;                 // rows past d_in are zero
+      const uint4* src = reinterpret_cast<const uint4*>(L.P + static_cast<size_t>(valid ? m : 0) * p.r);
+      // 64 bf16 (32 TMEM columns, eight 16-byte loads) per chunk; the next chunk's loads
+      // are in flight while this chunk is stored
+      uint32_t now[32], nxt[32];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint4 v = valid ? __ldg(src + k) : make_uint4(0u, 0u, 0u, 0u);
+        now[4 * k] = v.x; now[4 * k + 1] = v.y; now[4 * k + 2] = v.z; now[4 * k + 3] = v.w;
+      }
+#pragma unroll 1
+      for (int c = 0; c < PK; ++c) {
+        if (c + 1 < PK) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint4 v = valid ? __ldg(src + (c + 1) * 8 + k) : make_uint4(0u, 0u, 0u, 0u);
+            nxt[4 * k] = v.x; nxt[4 * k + 1] = v.y; nxt[4 * k + 2] = v.z; nxt[4 * k + 3] = v.w;
+          }
+        }
+        ptx::tmem_st32(tmem_p + lane_base + pb * kPCols + c * 32, now);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) now[k] = nxt[k];
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&pfull[pb]);
+    }
+  } else if (warp == 1) {
+    // ---------------- UMMA issuer ----------------
+    if (lane == 0) {
+      uint32_t ui = 0, ti = 0, it = 0;
+      bool ok = true;
+      BptWalk walk;
+      walk.start(p);
+      BptUnit x;
+      for (; ok && walk.next(p, x); ++ui) {
+        const int pb = ui % NPB;
+        if (!wait(&pfull[pb], (ui / NPB) & 1)) {
+          atomicOr(p.err, kErrTimeoutMma);
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t a0 = tmem_p + pb * kPCols;
+        for (int n = x.n0; ok && n < x.n1; ++n, ++ti) {
+          const int b = ti & 1;
+          const uint32_t use = ti >> 1;
+          if (use > 0 && !wait(&accempty[b], (use - 1) & 1)) {
+            atomicOr(p.err, kErrTimeoutMma);
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t d = tmem + b * kBnBack;
+#pragma unroll 1
+          for (int kb = 0; kb < PK; ++kb, ++it) {
+            const int st = it % DRS;
+            if (!wait(&full[st], (it / DRS) & 1)) {
+              atomicOr(p.err, kErrTimeoutMma);
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t b_base = ptx::smem_u32(smem + S::kDROff + st * S::kDRStage);
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k)   // 16 k per MMA: 8 TMEM columns of A
+              ptx::umma_bf16_tmem_a(d, a0 + kb * 32 + k * 8, ptx::desc_sw128(b_base + k * 2048, 8192, 1024),
+                                    kIdesc, (kb > 0 || k > 0) ? 1u : 0u);
+            ptx::umma_commit(&empty[st]);
+          }
+          ptx::umma_commit(&accfull[b]);
+        }
+        ptx::umma_commit(&pempty[pb]);   // the unit's MMAs, the last readers of this P block
+      }
+    }
+  } else {
+    // ---------------- epilogue: warps 2..9 ----------------
+    const int ew = warp - 2;
+    const int q = warp & 3;          // TMEM lanes (rows) 32q .. 32q+31
+    const int h = ew >> 2;           // column half of the tile: W boxes 2h, 2h+1
+    const int row = q * 32 + lane;
+    const float lr = p.lr;
+    uint32_t ti = 0;
+    BptWalk walk;
+    walk.start(p);
+    BptUnit x;
+    while (walk.next(p, x)) {
+      for (int n = x.n0; n < x.n1; ++n, ++ti) {
+        const int b = ti & 1;
+        const bool got = wait(&accfull[b], (ti >> 1) & 1);
+        if (!got) atomicOr(p.err, kErrTimeoutEpilogue);
+        ptx::tc_fence_after();
+#pragma unroll 1
+        for (int jj = 0; jj < 2; ++jj) {
+          const int j = 2 * h + jj;
+          const uint32_t wi = ti * kBoxes + j;
+          const int sl = wi % NW;
+          const bool wgot = wait(&wfull[sl], (wi / NW) & 1);
+          if (!wgot) atomicOr(p.err, kErrTimeoutEpilogue);
+          float v[32];
+          ptx::tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + b * kBnBack + j * 32, v);
+          uint8_t* box = smem + S::kWOff + sl * kWBox;
+          const bool act = got && wgot;
+          if (act) {
+            // row `row` of the box: 16-byte unit uu at uu ^ (row & 7) (128-byte swizzle)
+#pragma unroll
+            for (int uu = 0; uu < 8; ++uu) {
+              float4* w4 = reinterpret_cast<float4*>(box + row * 128 + ((uu ^ (row & 7)) * 16));
+              float4 w = *w4;
+              w.x = fmaf(-lr, v[4 * uu + 0], w.x);
+              w.y = fmaf(-lr, v[4 * uu + 1], w.y);
+              w.z = fmaf(-lr, v[4 * uu + 2], w.z);
+              w.w = fmaf(-lr, v[4 * uu + 3], w.w);
+              *w4 = w;
+            }
+            ptx::fence_proxy_async_smem();   // the rows are next read by the TMA store
+          }
+          __syncwarp();
+          if (lane == 0) {
+            // (a row quarter wholly past the last row of W has nothing to store)
+            if (act && x.m_t * kBM + q * 32 < p.lay[x.g].M) {
+              GRAPE_BOX(p.err, p.extW[x.g], 4, n * kBnBack + 32 * j, x.m_t * kBM + q * 32, 0)
+              ptx::tma_store_2d(&p.mapWs[x.g], box + q * 32 * 128, n * kBnBack + 32 * j, x.m_t * kBM + q * 32);
+              ptx::bulk_commit_group();
+              ptx::bulk_wait_group_read0();
+            }
+            ptx::mbar_arrive(&wfree[sl]);
+          }
+        }
+        // this accumulator may be overwritten by the tile after next
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&accempty[b]);
+      }
+    }
+    if (lane == 0) ptx::bulk_wait_group0();   // this warp's W stores complete
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kBptTmemCols);
+  }
+}
+
 // ---- aggregation with the K split across a thread-block cluster --------------------
 // For few output tiles (r x d_out is small next to K = B*T): the CS CTAs of a cluster
 // share one 128 x BN output tile of S and each runs 1/CS of the stacked token rows.
@@ -1083,10 +1492,11 @@ struct HostState {
   std::vector<CUtensorMap> mapAP2;      // AP as [B*T][r] (AGGREGATE A operand)
   std::vector<CUtensorMap> mapDR;       // dR as [r][d_out] (BACKPROJ B operand)
   // per-step maps, cached by pointer
-  std::vector<MapCache> cacheA, cacheG3, cacheG2, cacheW, cacheG3k;
+  std::vector<MapCache> cacheA, cacheG3, cacheG2, cacheW, cacheG3k, cacheWs;
   int* err = nullptr;
   int bn_project = 128;
   GroupParams gp;   // host staging of one launch's kernel parameters
+  BptParams bp;     // the same for tc_backproj_tmem_kernel
 };
 
 int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
@@ -1267,6 +1677,7 @@ cudaError_t tc_init(const StepShape& sh, const LayerWs* ws, void* scratch, size_
   hs->cacheG3k.resize(sh.L);
   hs->cacheG2.resize(sh.L);
   hs->cacheW.resize(sh.L);
+  hs->cacheWs.resize(sh.L);
   const uint64_t rows = static_cast<uint64_t>(sh.B) * sh.T;
   for (int l = 0; l < sh.L; ++l) {
     hs->d_in.push_back(ws[l].d_in);
@@ -1605,8 +2016,93 @@ cudaError_t tc_aggregate(const StepShape& sh, const LayerWs* ws, const LayerIo* 
   return cudaSuccess;
 }
 
+namespace {
+
+template <int PK, int NPB>
+cudaError_t launch_backproj_tmem(BptParams& bp, cudaStream_t st) {
+  using S = BptSmem<kBptDRS, kBptNW>;
+  const void* kern = reinterpret_cast<const void*>(tc_backproj_tmem_kernel<PK, NPB>);
+  int per_sm = 0;
+  cudaError_t e = configure_kernel(kern, S::kBytes, kBptThreads, &per_sm);
+  if (e != cudaSuccess) return e;
+  int most = 0;   // no more CTAs than the largest span has tiles
+  for (int k = 0; k < bp.n_spans; ++k) most = std::max(most, bp.span_tiles[k]);
+  if (most <= 0) return cudaSuccess;
+  int grid = sm_count() * per_sm;
+  grid = grid < most ? grid : most;
+  // the CTAs that take a span's extra tiles follow on from those of the span before
+  int rot = 0;
+  for (int k = 0; k < bp.n_spans; ++k) {
+    bp.span_rot[k] = rot;
+    rot = ((rot - bp.span_tiles[k] % grid) % grid + grid) % grid;
+  }
+  return launch_maybe_pdl(true, tc_backproj_tmem_kernel<PK, NPB>, dim3(grid), dim3(kBptThreads), S::kBytes, st,
+                          bp);
+}
+
+}  // namespace
+
+// The kernel with P in TMEM measured faster at r = 512 (the 7B slice: 1.73 against
+// 1.81-1.94 ms per step's back-projection) and slower at r = 256 and 128 (ViT-B: 172
+// against 150-157 us; long context: 192 against 169-176 us; MLP: 14.7 against
+// 13.8-14.8 us), where the streamed kernel's P tile is small.
+bool tc_backproj_p_in_tmem(int r) { return r == 512; }
+
+cudaError_t tc_backproject_streamed(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
+                                    const TcWorkspace& tc, float lr, cudaStream_t st, int* launches);
+
 cudaError_t tc_backproject(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                            const TcWorkspace& tc, float lr, cudaStream_t st, int* launches) {
+  if (!tc_backproj_p_in_tmem(sh.r)) return tc_backproject_streamed(sh, ws, io, tc, lr, st, launches);
+  HostState& hs = *static_cast<HostState*>(tc.host_state);
+  BptParams& bp = hs.bp;
+  for (int l0 = 0; l0 < sh.L; l0 += kMaxGroup) {
+    const int n = (sh.L - l0) < kMaxGroup ? (sh.L - l0) : kMaxGroup;
+    std::memset(&bp, 0, sizeof(bp));
+    bp.err = hs.err;
+    bp.lr = lr;
+    bp.r = sh.r;
+    bp.n_layers = n;
+    const int grid_full = sm_count();   // one CTA per SM (the kernel allocates TMEM)
+    int span_tiles = 0;
+    for (int g = 0; g < n; ++g) {
+      const int l = l0 + g;
+      bp.mapDR[g] = hs.mapDR[l];
+      if (!hs.cacheW[l].get(io[l].W, &bp.mapW[g], [&](CUtensorMap* m) {
+            return map_2d_f32(m, io[l].W, ws[l].d_in, ws[l].d_out);
+          }) ||
+          !hs.cacheWs[l].get(io[l].W, &bp.mapWs[g], [&](CUtensorMap* m) {
+            return map_2d_f32(m, io[l].W, ws[l].d_in, ws[l].d_out, 32);
+          }))
+        return cudaErrorInvalidValue;
+      GRAPE_EXT(bp.extDR[g], ws[l].d_out, sh.r, 1)
+      GRAPE_EXT(bp.extW[g], ws[l].d_out, ws[l].d_in, 1)
+      BptLayer& L = bp.lay[g];
+      L.M = ws[l].d_in;
+      L.mt = cdiv(ws[l].d_in, kBM);
+      L.nt = cdiv(ws[l].d_out, kBnBack);
+      L.P = ws[l].P16;
+      // spans of at least four tiles per CTA
+      if (span_tiles == 0) bp.span_first[bp.n_spans] = g;
+      L.tiles_begin = span_tiles;
+      span_tiles += L.mt * L.nt;
+      if (span_tiles >= 4 * grid_full || g == n - 1) {
+        bp.span_tiles[bp.n_spans++] = span_tiles;
+        span_tiles = 0;
+      }
+    }
+    bp.span_first[bp.n_spans] = n;
+    cudaError_t e = launch_backproj_tmem<8, 1>(bp, st);   // r = 512: one 256-column P block
+    if (e != cudaSuccess) return e;
+    ++*launches;
+  }
+  return cudaSuccess;
+}
+
+// W -= lr P dR with P loaded by TMA with every tile (tc_gemm_kernel<BACKPROJ>): the
+// projection widths whose P block does not fit in TMEM next to the accumulators.
+cudaError_t tc_backproject_streamed(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
+                                    const TcWorkspace& tc, float lr, cudaStream_t st, int* launches) {
   HostState& hs = *static_cast<HostState*>(tc.host_state);
   GroupParams& gp = hs.gp;
   std::memset(&gp, 0, sizeof(gp));
