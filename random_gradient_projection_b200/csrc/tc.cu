@@ -770,6 +770,11 @@ __global__ void __launch_bounds__(kBptThreads, 1) tc_backproj_tmem_kernel(const 
   constexpr int kBoxes = kBnBack / 32;                                     // W boxes per tile
   constexpr uint32_t kPCols = PK * 32;                                     // TMEM columns of one P block
   static_assert(2 * kBnBack + NPB * kPCols <= kBptTmemCols, "TMEM columns");
+  // A slot of the W ring must only ever hold boxes of one column half, so that the four
+  // warps that wait on its wfull barrier have consumed its previous use themselves: a
+  // parity wait cannot tell a phase two ahead from the one behind, and a warp of the other
+  // half waiting for the slot's next use would pass at once on the previous phase.
+  static_assert(NW % kBoxes == 0, "W ring slots must map to one box position of a tile");
   static_assert((2 * NPB + 2 * DRS + 4 + 2 * NW) * 8 + 16 <= 512, "barrier area");
 
   extern __shared__ uint8_t smem_raw[];
