@@ -200,9 +200,13 @@ GRAPE_API int grape_set_graph(grape_ctx* ctx, int32_t enable);
  *                     calls orthogonal to DP-GRAPE; the DP-SGD-RC summary costs it at
  *                     O(B T^2 (p + d)) per linear layer).  It costs 2 T^2 (r + d_out) flops
  *                     per sample and layer against 2 T r d_out, so it pays for short T.
+ *                     The Grams are taken in 128 x 128 blocks of 128-token blocks a <= b
+ *                     (off-diagonal blocks counted twice), so any T is accepted.
  * Both give the same value up to rounding; the step, grape_sqnorms and clipping use it.
+ * The ghost norm forms no R_i, so its steps use the recomputed aggregation whatever
+ * grape_set_aggregation says.
  * Errors: GRAPE_EINVAL (unknown method); GRAPE_EUNSUPPORTED (ghost needs the
- * tensor-core path and T <= 128). */
+ * tensor-core path). */
 enum grape_norm_method { GRAPE_NORM_DIRECT = 0, GRAPE_NORM_GHOST = 1 };
 GRAPE_API int grape_set_norm_method(grape_ctx* ctx, int32_t method);
 

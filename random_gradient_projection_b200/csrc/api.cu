@@ -841,7 +841,7 @@ int grape_set_norm_method(grape_ctx* ctx, int32_t method) {
     return ctx->fail(GRAPE_EINVAL, "method must be GRAPE_NORM_DIRECT or GRAPE_NORM_GHOST");
   if (method == GRAPE_NORM_GHOST &&
       (ctx->path != GRAPE_PATH_TC || !grape::tc_ghost_supported(ctx->sh)))
-    return ctx->fail(GRAPE_EUNSUPPORTED, "the ghost norm runs on the tensor-core path with T <= 128");
+    return ctx->fail(GRAPE_EUNSUPPORTED, "the ghost norm runs on the tensor-core path");
   if (method != ctx->norm_method) {   // captured graphs hold the other norm kernel
     for (auto& g : ctx->graphs) ctx->drop_graph(g);
     ctx->graphs.clear();

@@ -94,6 +94,7 @@ struct GroupLayer {
   int part_base;     // NORM, GHOST: first partial slot of this layer
   int slots;         // GHOST: partial slots of this layer per sample (the first gets the sum)
   int kfirst;        // GHOST: k-blocks of Gout, loaded before the k-blocks of AP
+  int nb;            // GHOST: 128-token blocks of a sample, ceil(T / 128)
 };
 
 struct GroupParams {
@@ -169,9 +170,20 @@ template <int MODE>
 struct ModeExtra {
   static constexpr int kBytes = (MODE == BACKPROJ) ? 2 * kWTile : (MODE == NORMST) ? kEpiWarps * kRBox : 0;
 };
-// GHOST stages hold a single 128-row tile, used as both operands of its Gram product.
+// GHOST stages hold the 128-token blocks a and b of a sample (one block when a == b),
+// whose Gram block X_a X_b^T the stage's MMAs accumulate.
 template <int MODE, int BN, int STAGES>
-using SmemOf = Smem<BN, STAGES, ModeExtra<MODE>::kBytes, MODE == GHOST ? 0 : BN>;
+using SmemOf = Smem<BN, STAGES, ModeExtra<MODE>::kBytes, BN>;
+
+// GHOST: the pairs of token blocks (a, b), a <= b, of one (sample, layer) tile, in order;
+// every other mode has one round per tile.
+struct GhostPairs {
+  int a = 0, b = 0;
+  __device__ __forceinline__ void next(int nb) {
+    if (++b == nb) b = ++a;
+  }
+};
+__device__ __forceinline__ int ghost_rounds(int nb) { return nb * (nb + 1) / 2; }
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
@@ -344,6 +356,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++tcp) {
         const TileCoord c = decode_tile(p, tile, MODE);
+        const int rounds = (MODE == GHOST) ? ghost_rounds(p.lay[c.g].nb) : 1;
+        GhostPairs gp_;
         if (MODE == BACKPROJ && pi == 0 && tcp > 0) {
           // this tile's W into buffer tcp & 1, once the store of the tile before last
           // has finished reading it
@@ -356,6 +370,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
           load_w(c, wb);
           ++wissued;
         }
+        for (int round = 0; ok && round < rounds; ++round) {
+        if (MODE == GHOST && round > 0) gp_.next(p.lay[c.g].nb);
         for (int kb = c.kb0; kb < c.kb1; ++kb, ++it) {
           if (static_cast<int>(it % kNP) != pi) continue;
           const int s = it % STAGES;
@@ -365,20 +381,31 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             ok = false;
             break;
           }
-          ptx::mbar_arrive_expect_tx(&full[s], S::kStage);
           if (MODE == GHOST) {
-            // rows 0..127 of the sample (past T: zeros); Gout first, then AP (after the wait)
+            // token blocks a and b of the sample (rows past T: zeros), one box when a == b;
+            // Gout's k-blocks first, then AP's (after the wait)
             const int kf = p.lay[c.g].kfirst;
+            const int na = gp_.a == gp_.b ? 1 : 2;
+            ptx::mbar_arrive_expect_tx(&full[s], na * S::kABytes);
             uint8_t* st_ = smem + s * S::kStage;
-            if (kb < kf) {
-              GRAPE_BOX(p.err, p.extB[c.g], 2, kb * kBK, 0, c.s_t)
-              ptx::tma_load_3d_hint(st_, &p.mapB[c.g], &full[s], kb * kBK, 0, c.s_t, polB);
-            } else {
-              ensure_wait();
-              GRAPE_BOX(p.err, p.extA[c.g], 2, (kb - kf) * kBK, 0, c.s_t)
-              ptx::tma_load_3d_hint(st_, &p.mapA[c.g], &full[s], (kb - kf) * kBK, 0, c.s_t, polA);
+            if (kb >= kf) ensure_wait();
+            const CUtensorMap* map = kb < kf ? &p.mapB[c.g] : &p.mapA[c.g];
+            const int x = (kb < kf ? kb : kb - kf) * kBK;
+            const uint64_t pol = kb < kf ? polB : polA;
+            for (int k = 0; k < na; ++k) {
+              const int y = (k == 0 ? gp_.a : gp_.b) * kBM;
+              if (kb < kf)
+                GRAPE_BOX(p.err, p.extB[c.g], 2, x, y, c.s_t)
+                ptx::tma_load_3d_hint(st_ + k * S::kABytes, map, &full[s], x, y, c.s_t, pol);
+              else
+                GRAPE_BOX(p.err, p.extA[c.g], 2, x, y, c.s_t)
+                ptx::tma_load_3d_hint(st_ + k * S::kABytes, map, &full[s], x, y, c.s_t, pol);
             }
-          } else if (MODE == PROJECT) {
+            issued_end = it + 1;
+            continue;
+          }
+          ptx::mbar_arrive_expect_tx(&full[s], S::kStage);
+          if (MODE == PROJECT) {
             load_a(c, kb, s);
             ensure_wait();
             load_b(c, kb, s);
@@ -392,6 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             load_b(c, kb, s);
           }
           issued_end = it + 1;
+        }
         }
       }
       if (*abort_flag) {
@@ -409,12 +437,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     if (lane == 0) {
       uint32_t it = 0, tc = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++tc) {
+      for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
         const TileCoord c = decode_tile(p, tile, MODE);
+        const int rounds = (MODE == GHOST) ? ghost_rounds(p.lay[c.g].nb) : 1;
+        GhostPairs gp_;
+        for (int round = 0; ok && round < rounds; ++round, ++tc) {
+        if (MODE == GHOST && round > 0) gp_.next(p.lay[c.g].nb);
         const int b = tc & 1;
         const uint32_t use = tc >> 1;
         if (use > 0 && !wait(&accempty[b], (use - 1) & 1)) {
           atomicOr(p.err, kErrTimeoutMma);
+          ok = false;
           break;
         }
         ptx::tc_fence_after();
@@ -431,17 +464,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
           const uint32_t a_base = ptx::smem_u32(smem + s * S::kStage);
           const uint32_t b_base = a_base + S::kABytes;
           if (MODE == GHOST) {
-            // the stage's tile X (128 rows, 64 K-major columns) as both operands: D += X X^T,
-            // into the Gout Gram (first accumulator) or the AP Gram (second)
+            // the stage's blocks X_a, X_b (128 rows, 64 K-major columns each; X_b is X_a
+            // when a == b): D += X_a X_b^T, into the Gout Gram block (first accumulator) or
+            // the AP Gram block (second)
             const int kf = p.lay[c.g].kfirst;
             const bool second = kb >= kf;
             const uint32_t dd = d + (second ? BN : 0);
             const int kstart = second ? kf : c.kb0;
+            const uint32_t bx = gp_.a == gp_.b ? a_base : a_base + S::kABytes;
 #pragma unroll
-            for (int k = 0; k < kBK / 16; ++k) {
-              const uint64_t xd = ptx::desc_sw128(a_base + k * 32, 16, 1024);
-              ptx::umma_bf16(dd, xd, xd, kIdesc, (kb > kstart || k > 0) ? 1u : 0u);
-            }
+            for (int k = 0; k < kBK / 16; ++k)
+              ptx::umma_bf16(dd, ptx::desc_sw128(a_base + k * 32, 16, 1024), ptx::desc_sw128(bx + k * 32, 16, 1024),
+                             kIdesc, (kb > kstart || k > 0) ? 1u : 0u);
           } else {
 #pragma unroll
             for (int k = 0; k < kBK / 16; ++k) {
@@ -456,6 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
           ptx::umma_commit(&empty[s]);
         }
         ptx::umma_commit(&accfull[b]);
+        }
       }
     }
   } else if (warp < 2 + kEpiWarps) {
@@ -469,10 +504,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     constexpr int kHalf = BN / 2;
     // The epilogue warps walk every tile even after a failed wait (their waits then
     // return at once), so the named barriers below are always reached by all of them.
-    uint32_t tc = 0;
-    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++tc) {
+    uint32_t tc = 0, tcount = 0;
+    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++tcount) {
       const TileCoord c = decode_tile(p, tile, MODE);
       const GroupLayer& L = p.lay[c.g];
+      const int rounds = (MODE == GHOST) ? ghost_rounds(L.nb) : 1;
+      GhostPairs gp_;
+      float gsum = 0.0f;   // GHOST: this thread's share of the sample's squared norm
+      for (int round = 0; round < rounds; ++round, ++tc) {
+      if (MODE == GHOST && round > 0) gp_.next(L.nb);
       const int b = tc & 1;
       const uint32_t use = tc >> 1;
       const bool got = wait(&accfull[b], use & 1);
@@ -544,7 +584,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
           p.partials[static_cast<size_t>(c.s_t) * p.part_stride + L.part_base + c.m_t * L.nt + c.n_t] = tot;
         }
       } else if (MODE == GHOST) {
-        // sum over this warp's 32 rows x 64 columns of (Gout Gram) * (AP Gram)
+        // this thread's row x 64 columns of (Gout Gram block) * (AP Gram block); an
+        // off-diagonal block (a < b) stands for its transpose (b, a) too
         float ss = 0.0f;
 #pragma unroll 1
         for (int cc = 0; cc < kHalf; cc += 32) {
@@ -554,23 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
 #pragma unroll
           for (int j = 0; j < 32; ++j) ss = fmaf(x[j], y[j], ss);
         }
-        if (!have) ss = 0.0f;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        float* rb = red + (tc & 1) * kEpiWarps;
-        if (lane == 0) rb[ew] = ss;
-        epi_bar();
-        if (ew == 0) {
-          // the layer's first slot holds the norm, its other slots zero (the clip sums them all)
-          float* slot = p.partials + static_cast<size_t>(c.s_t) * p.part_stride + L.part_base;
-          for (int k = lane; k < L.slots; k += 32) {
-            float tot = 0.0f;
-            if (k == 0)
-#pragma unroll
-              for (int w2 = 0; w2 < kEpiWarps; ++w2) tot += rb[w2];
-            slot[k] = tot;
-          }
-        }
+        if (have) gsum = fmaf(gp_.a == gp_.b ? 1.0f : 2.0f, ss, gsum);
       } else if (MODE == AGGREGATE) {
         const int m = c.m_t * kBM + row;
         float* dst = static_cast<float*>(L.out);
@@ -635,10 +660,30 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
           ptx::mbar_arrive(&wfree[b]);
         }
       }
-      // this accumulator may be overwritten by the tile after next
+      // this accumulator may be overwritten by the round after next
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&accempty[b]);
+      }
+      if (MODE == GHOST) {
+        // the sample's squared norm for this layer: the sum over the 8 warps, in order
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) gsum += __shfl_xor_sync(0xffffffffu, gsum, o);
+        float* rb = red + (tcount & 1) * kEpiWarps;
+        if (lane == 0) rb[ew] = gsum;
+        epi_bar();
+        if (ew == 0) {
+          // the layer's first slot holds the norm, its other slots zero (the clip sums them all)
+          float* slot = p.partials + static_cast<size_t>(c.s_t) * p.part_stride + L.part_base;
+          for (int k = lane; k < L.slots; k += 32) {
+            float tot = 0.0f;
+            if (k == 0)
+#pragma unroll
+              for (int w2 = 0; w2 < kEpiWarps; ++w2) tot += rb[w2];
+            slot[k] = tot;
+          }
+        }
+      }
     }
   }
 
@@ -1484,7 +1529,7 @@ constexpr int kStagesAgg = 4;          // 4 x 48 KB
 constexpr int kStagesBack = 3;         // 3 x 32 KB stages + 2 x 64 KB W tiles
 constexpr int kBnAggCluster = 128;     // cluster-split aggregation: 6 x 32 KB
 constexpr int kStagesAggCluster = 6;
-constexpr int kStagesGhost = 12;       // 12 x 16 KB: one 128-row tile per stage
+constexpr int kStagesGhost = 6;        // 6 x 32 KB: the two 128-token blocks of a Gram block
 
 struct HostState {
   int L = 0, r = 0, B = 0, T = 0;
@@ -1493,7 +1538,7 @@ struct HostState {
   std::vector<CUtensorMap> mapP_mn;     // P16 as the MN-major B operand of PROJECT
   std::vector<CUtensorMap> mapP_k;      // P16 as the K-major A operand of BACKPROJ
   std::vector<CUtensorMap> mapAP3;      // AP as [B][T][r] (NORM A operand)
-  std::vector<CUtensorMap> mapAP3k;     // AP as [B][T][r], 128-row boxes (GHOST, T <= 128)
+  std::vector<CUtensorMap> mapAP3k;     // AP as [B][T][r], 128-row boxes (GHOST)
   std::vector<CUtensorMap> mapAP2;      // AP as [B*T][r] (AGGREGATE A operand)
   std::vector<CUtensorMap> mapDR;       // dR as [r][d_out] (BACKPROJ B operand)
   // per-step maps, cached by pointer
@@ -1690,7 +1735,7 @@ cudaError_t tc_init(const StepShape& sh, const LayerWs* ws, void* scratch, size_
     bool ok = map_2d(&hs->mapP_mn[l], ws[l].P16, ws[l].d_in, sh.r, 64, 64) &&
               map_2d(&hs->mapP_k[l], ws[l].P16, ws[l].d_in, sh.r, 64, kBM) &&
               map_3d(&hs->mapAP3[l], ws[l].AP, sh.B, sh.T, sh.r) &&
-              (sh.T > kBM || map_3d(&hs->mapAP3k[l], ws[l].AP, sh.B, sh.T, sh.r, kBM)) &&
+              map_3d(&hs->mapAP3k[l], ws[l].AP, sh.B, sh.T, sh.r, kBM) &&
               map_2d(&hs->mapAP2[l], ws[l].AP, rows, sh.r, 64, 64) &&
               map_2d(&hs->mapDR[l], ws[l].dR, sh.r, ws[l].d_out, 64, 64);
     if (!ok) {
@@ -1830,13 +1875,14 @@ cudaError_t tc_project_norm(const StepShape& sh, const LayerWs* ws, const LayerI
   return run_mode<NORM, kBnWide, kStagesNorm>(hs, sh.L, st, launches, fill, gp);
 }
 
-bool tc_ghost_supported(const StepShape& sh) { return sh.T <= kBM; }
+bool tc_ghost_supported(const StepShape& sh) { (void)sh; return true; }
 
 // Per-sample squared norms by the ghost identity ||(A_i P)^T Gout_i||^2 =
-// <(A_i P)(A_i P)^T, Gout_i Gout_i^T>_F: one 128 x 128 Gram tile pair per (sample, layer).
+// <(A_i P)(A_i P)^T, Gout_i Gout_i^T>_F: one tile per (sample, layer), which runs over the
+// pairs a <= b of 128-token blocks of the sample, each a 128 x 128 block of both T x T
+// Gram matrices (off-diagonal blocks counted twice, for their transposes).
 cudaError_t tc_project_norm_ghost(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                                   const TcWorkspace& tc, float* partials, cudaStream_t st, int* launches) {
-  if (sh.T > kBM) return cudaErrorInvalidValue;
   HostState& hs = *static_cast<HostState*>(tc.host_state);
   GroupParams& gp = hs.gp;
   std::memset(&gp, 0, sizeof(gp));
@@ -1857,6 +1903,7 @@ cudaError_t tc_project_norm_ghost(const StepShape& sh, const LayerWs* ws, const 
     L.ns = sh.B;
     L.kfirst = cdiv(ws[l].d_out, kBK);
     L.kblocks = L.kfirst + cdiv(sh.r, kBK);
+    L.nb = cdiv(sh.T, kBM);
     L.M = sh.T;
     L.N = sh.T;
     L.part_base = ws[l].part_base;

@@ -388,7 +388,7 @@ class GrapeStep:
         grape_set_graph(self.ctx, enable)
 
     def set_norm_method(self, method: int):
-        """GRAPE_NORM_DIRECT (default) or GRAPE_NORM_GHOST (tensor-core path, T <= 128)."""
+        """GRAPE_NORM_DIRECT (default) or GRAPE_NORM_GHOST (tensor-core path)."""
         grape_set_norm_method(self.ctx, method)
 
     def set_aggregation(self, method: int):
