@@ -623,7 +623,9 @@ def main(argv=None):
         cpu = {"value": v, "unit": "samples/s", "cores": cores, "kind": "oracle",
                "sample": f"{n} samples of {w.name} (oracle steps over {nb} of its B={w.B} "
                          f"samples, after one over a single sample), {secs:.1f} s of fp64 numpy "
-                         f"oracle time"}
+                         f"oracle time; every oracle step also draws each layer's P and noise "
+                         f"in numpy, a cost per step that a sample of few samples does not "
+                         f"spread"}
 
     if rank == 0:
         line = {
