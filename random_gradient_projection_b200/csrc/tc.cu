@@ -577,11 +577,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         float* rb = red + (tc & 1) * kEpiWarps;
         if (lane == 0) rb[ew] = ss;
         epi_bar();
-        if (ew == 0 && lane == 0) {
+        // one partial slot per 128 columns of d_out (the slot layout every norm kernel
+        // shares): column half `lane` of the tile is the sum over its four warps
+        static_assert(!T::kNorm || BN == 256, "a norm tile is two 128-column slots");
+        if (ew == 0 && lane < 2) {
           float tot = 0.0f;
 #pragma unroll
-          for (int k = 0; k < kEpiWarps; ++k) tot += rb[k];
-          p.partials[static_cast<size_t>(c.s_t) * p.part_stride + L.part_base + c.m_t * L.nt + c.n_t] = tot;
+          for (int k = 0; k < 4; ++k) tot += rb[4 * lane + k];
+          p.partials[static_cast<size_t>(c.s_t) * p.part_stride + L.part_base + c.m_t * (2 * L.nt) +
+                     2 * c.n_t + lane] = tot;
         }
       } else if (MODE == GHOST) {
         // this thread's row x 64 columns of (Gout Gram block) * (AP Gram block); an
@@ -751,34 +755,46 @@ struct BptParams {
 };
 
 struct BptUnit {
-  int g, m_t, n0, n1;   // layer in the launch, row block, tiles [n0, n1)
+  int g, m_t, n0, n1;   // layer in the launch, row block (a sample in the norm kernel), tiles [n0, n1)
 };
 
-// This CTA's units in order: span by span, its range of the span's tiles cut at the
-// ends of layers and of row blocks.
-struct BptWalk {
-  int sp, g, cur, t1;   // span, layer, next tile of the span, end of this CTA's range in it
-  __device__ __forceinline__ void range(const BptParams& p) {
+// One position's units in order: span by span, its range of the span's tiles cut at
+// the ends of layers and of row blocks.  A position is a CTA (back-projection) or a
+// group of CTAs that walk the same tiles (norms); `npos` positions share each span.
+// The params need n_spans, span_first, span_tiles, span_rot and per layer
+// tiles_begin and nt.
+struct SpanWalk {
+  int sp, g, cur, t1;   // span, layer, next tile of the span, end of this position's range in it
+  int npos, pos;
+  template <class Pm>
+  __device__ __forceinline__ void range(const Pm& p) {
     const int T = p.span_tiles[sp];
-    const int G = static_cast<int>(gridDim.x);
-    const int base = T / G, extra = T % G;
-    const int b = (static_cast<int>(blockIdx.x) + p.span_rot[sp]) % G;
+    const int base = T / npos, extra = T % npos;
+    const int b = (pos + p.span_rot[sp]) % npos;
     cur = b * base + min(b, extra);
     t1 = cur + base + (b < extra ? 1 : 0);
     g = p.span_first[sp];
   }
-  __device__ __forceinline__ void start(const BptParams& p) {
+  template <class Pm>
+  __device__ __forceinline__ void start(const Pm& p, int npos_, int pos_) {
+    npos = npos_;
+    pos = pos_;
     sp = 0;
     range(p);
   }
-  // The next unit; false when the CTA has none left.
-  __device__ __forceinline__ bool next(const BptParams& p, BptUnit& x) {
+  template <class Pm>
+  __device__ __forceinline__ void start(const Pm& p) {
+    start(p, static_cast<int>(gridDim.x), static_cast<int>(blockIdx.x));
+  }
+  // The next unit; false when the position has none left.
+  template <class Pm>
+  __device__ __forceinline__ bool next(const Pm& p, BptUnit& x) {
     while (cur >= t1) {
       if (++sp >= p.n_spans) return false;
       range(p);
     }
     while (g + 1 < p.span_first[sp + 1] && cur >= p.lay[g + 1].tiles_begin) ++g;
-    const BptLayer& L = p.lay[g];
+    const auto& L = p.lay[g];
     const int t = cur - L.tiles_begin;
     x.g = g;
     x.m_t = t / L.nt;
@@ -788,6 +804,7 @@ struct BptWalk {
     return true;
   }
 };
+using BptWalk = SpanWalk;
 
 // DRS dR stages and NW W boxes in shared memory.
 template <int DRS, int NW>
@@ -1107,6 +1124,393 @@ __global__ void __launch_bounds__(kBptThreads, 1) tc_backproj_tmem_kernel(const 
     __syncwarp();
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kBptTmemCols);
+  }
+}
+
+// ---- per-sample norms and stored R_i with (A_i P)^T resident in tensor memory -------
+// R_i = (A_i P)^T Gout_i in tiles of 128 rows (a block of the r projection rows) x 256
+// columns of d_out with K = T, the A operand -- the 128 x T block of (A_i P)^T -- read
+// by the MMA from TMEM.  The mr = r / 128 row blocks of a sample run side by side on mr
+// CTAs (a group): CTA b is row block b % mr of group b / mr.  The groups split the
+// launch's column tiles (layer, sample, 256 columns of d_out, in that order) into
+// contiguous ranges balanced to within one tile, and the CTAs of a group walk the same
+// column tiles at the same pace, so a Gout tile is read from DRAM once and from L2 by
+// the mr SMs.  A work unit is the part of a range in one sample: its block of
+// (A_i P)^T enters TMEM once, and per tile only Gout (T x 256 bf16) streams through
+// shared memory.  tc_gemm_kernel<NORMST> moves 128 x T of AP and T x 256 of Gout from L2
+// per 128 x 256 tile; this kernel moves the Gout part alone, 512 T instead of 768 T
+// bytes per 65536 T flops, and its MMAs, with A from TMEM, issue faster than that
+// kernel's with both operands in shared memory.  Every tile's R_i is stored (bf16,
+// [sample][r][d_out]) for the stored aggregation.
+//
+// A unit's block enters TMEM in 64-token chunks, loaded by TMA as two 64-token x 64-row
+// boxes of AP (tokens past T zero-filled) through the same ring of stages as Gout: the
+// ring holds, in order, the chunks of unit 0, its Gout stages, the chunks of unit 1, its
+// Gout stages, and so on, so a unit's chunks load while the previous unit's last Gout
+// stages are consumed, and the ring keeps all the shared memory that the R staging
+// leaves.  Warps 10-13 read the chunks out of shared memory transposed (thread = row of
+// (A_i P)^T, two tokens per 32-bit column) and store them with tcgen05.st.  Gout tokens
+// past T are zero-filled too.
+//
+// TMEM: one 128 x 256 fp32 accumulator (columns 0..255) and the block of (A_i P)^T
+// (columns 256..511: T <= 512).  With one accumulator the MMAs of a tile wait until the
+// epilogue has loaded the previous tile into registers, which it does first, before any
+// other work on it.  The writers of a unit's block wait until the MMAs of the previous
+// unit are done, which is also what keeps the shared ring's parity waits sound.  An
+// mbarrier parity wait for phase k of a slot returns at once while phase k - 1 is still
+// open, so a consumer may wait for a ring position only once the position NS earlier
+// has been loaded.  The MMAs' positions follow their unit's chunks, which the writers
+// have consumed; the writers' positions follow the previous unit's Gout stages, which
+// the MMAs have consumed.  (With a second block the writers would run a unit ahead of
+// the MMAs and wait on slots whose previous Gout stage had not been loaded yet.)
+//
+// Warps: 0 issues the ring's loads (after griddepcontrol.wait: AP is written earlier
+// in the step); 1 owns TMEM and issues the MMAs; 2-9 are the epilogue (warp w: lane
+// quarter w % 4, 128-column half (w - 2) / 4), which sums the squares of each half into
+// its partial slot and writes the tile of R_i; 10-13 write the chunks into TMEM.
+constexpr int kNtBN = 256;
+
+struct NtLayer {
+  int tiles_begin;   // first column tile of this layer in its span
+  int nt;            // 256-column tiles of d_out
+  int d_out;
+  int part_base;     // first partial slot of this layer
+  __nv_bfloat16* Rst;   // R_l as [B][r][d_out] bf16
+};
+
+struct NtParams {
+  CUtensorMap mapG[kMaxGroup];    // Gout: bf16 (d_out, T, B), boxes of 64 x 64 x 1
+  CUtensorMap mapAP[kMaxGroup];   // AP: bf16 (r, T, B), boxes of 64 x 64 x 1
+  NtLayer lay[kMaxGroup];
+  int n_layers;
+  int n_spans;
+  int span_first[kMaxGroup + 1];
+  int span_tiles[kMaxGroup];
+  int span_rot[kMaxGroup];
+  int r;
+  int mr;        // 128-row blocks of r: CTAs per group
+  int groups;
+  int kblocks;   // 64-token chunks: ceil(T / 64)
+  int part_stride;
+  float* partials;
+  int* err;
+#ifdef GRAPE_CHECKED
+  int extG[kMaxGroup][3];
+  int extAP[kMaxGroup][3];
+#endif
+};
+
+struct NtSmem {
+  static constexpr int kStage = kBK * kNtBN * 2;   // 64 tokens x 256 columns of Gout: 32 KB
+  static constexpr int kAStage = kBK * kBM * 2;    // a chunk, 64 tokens x 128 rows of AP: 16 KB
+  static constexpr int kStages = 6;
+  static constexpr int kRBoxOff = kStages * kStage;
+  static constexpr int kBarOff = kRBoxOff + kEpiWarps * kRBox;
+  static constexpr int kBytes = kBarOff + 512 + 1024;   // barriers + alignment slack
+  static_assert(kBytes <= 232448, "exceeds the shared memory of a CTA");
+};
+constexpr int kNtThreads = 32 * 14;
+constexpr int kNtAWriter0 = 10;   // warps 10..13
+constexpr uint32_t kNtTmemCols = 512;
+
+__device__ __forceinline__ void nt_writer_bar() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+
+__global__ void __launch_bounds__(kNtThreads, 1) tc_norm_tmem_kernel(const __grid_constant__ NtParams p) {
+  using S = NtSmem;
+  constexpr int NS = S::kStages;
+  constexpr uint32_t kIdesc = ptx::idesc_bf16(kBM, kNtBN, false, true);   // A K-major (TMEM), Gout N-major
+  constexpr uint32_t kACols = 256;                                     // the block: 512 tokens at most
+  static_assert(kNtBN + kACols <= kNtTmemCols, "TMEM columns");
+  static_assert((2 * NS + 4) * 8 + 16 + 2 * kEpiWarps * 4 <= 512, "barrier area");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
+  uint64_t* empty = full + NS;
+  uint64_t* pfull = empty + NS;      // the block of (A_i P)^T is in TMEM
+  uint64_t* pempty = pfull + 1;      // the block's MMAs are done
+  uint64_t* accfull = pempty + 1;
+  uint64_t* accempty = accfull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  float* red = reinterpret_cast<float*>(tmem_slot + 4);   // [2][kEpiWarps]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mblk = static_cast<int>(blockIdx.x) % p.mr;
+  const int group = static_cast<int>(blockIdx.x) / p.mr;
+  const int kbn = p.kblocks;
+  auto wait = [&](uint64_t* bar, uint32_t parity) {
+    return ptx::mbar_wait_or_abort(bar, parity, kWaitLimitNs, abort_flag);
+  };
+  ptx::griddep_launch_dependents();
+
+  if (warp == 0 && lane == 0) {
+    *abort_flag = 0;
+    for (int st = 0; st < NS; ++st) {
+      ptx::mbar_init(&full[st], 1);
+      ptx::mbar_init(&empty[st], 1);
+    }
+    ptx::mbar_init(pfull, 4);   // the four TMEM-writing warps
+    ptx::mbar_init(pempty, 1);
+    ptx::mbar_init(accfull, 1);
+    ptx::mbar_init(accempty, kEpiWarps);
+    ptx::fence_mbar_init();
+    for (int g = 0; g < p.n_layers; ++g) {
+      ptx::prefetch_tmap(&p.mapG[g]);
+      ptx::prefetch_tmap(&p.mapAP[g]);
+    }
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, kNtTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_a = tmem + kNtBN;   // the block of (A_i P)^T after the accumulator
+
+  if (warp == 0) {
+    // ---------------- the ring: each unit's chunks of AP, then its Gout stages ----------------
+    if (lane == 0) {
+      // Gout is read by the group's mr CTAs at about the same time, then never again;
+      // AP is not read again in the step
+      const uint64_t polG = ptx::policy_evict_normal();
+      const uint64_t polA = ptx::policy_evict_first();
+      ptx::griddep_wait();   // AP is written earlier in this step
+      uint32_t it = 0, it_issued = 0;
+      bool ok = true;
+      SpanWalk walk;
+      walk.start(p, p.groups, group);
+      BptUnit x;
+      auto next_slot = [&](int& st) {
+        st = it % NS;
+        const uint32_t use = it / NS;
+        if (use > 0 && !wait(&empty[st], (use - 1) & 1)) {
+          atomicOr(p.err, kErrTimeoutProducer);
+          ok = false;
+        }
+        return ok;
+      };
+      while (ok && walk.next(p, x)) {
+#pragma unroll 1
+        for (int c = 0; c < kbn; ++c, ++it) {
+          int st;
+          if (!next_slot(st)) break;
+          uint8_t* dst = smem + st * S::kStage;
+          ptx::mbar_arrive_expect_tx(&full[st], S::kAStage);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            GRAPE_BOX(p.err, p.extAP[x.g], 2, mblk * kBM + 64 * h, c * kBK, x.m_t)
+            ptx::tma_load_3d_hint(dst + h * 8192, &p.mapAP[x.g], &full[st], mblk * kBM + 64 * h, c * kBK, x.m_t,
+                                  polA);
+          it_issued = it + 1;
+        }
+        for (int n = x.n0; ok && n < x.n1; ++n) {
+#pragma unroll 1
+          for (int kb = 0; kb < kbn; ++kb, ++it) {
+            int st;
+            if (!next_slot(st)) break;
+            uint8_t* dst = smem + st * S::kStage;
+            ptx::mbar_arrive_expect_tx(&full[st], S::kStage);
+#pragma unroll
+            for (int h = 0; h < kNtBN / 64; ++h)
+              GRAPE_BOX(p.err, p.extG[x.g], 2, n * kNtBN + 64 * h, kb * kBK, x.m_t)
+              ptx::tma_load_3d_hint(dst + h * 8192, &p.mapG[x.g], &full[st], n * kNtBN + 64 * h, kb * kBK, x.m_t,
+                                    polG);
+            it_issued = it + 1;
+          }
+        }
+      }
+      if (*abort_flag)   // leave none of this thread's loads in flight into shared memory
+        for (uint32_t k = it_issued > NS ? it_issued - NS : 0; k < it_issued; ++k)
+          ptx::mbar_wait(&full[k % NS], (k / NS) & 1, kDrainLimitNs);
+    }
+  } else if (warp >= kNtAWriter0) {
+    // ---------------- (A_i P)^T into TMEM: one row of the block per thread ----------------
+    const int q = warp & 3;                                   // TMEM lanes 32q .. 32q+31
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const int j = q * 32 + lane;                              // row of the block: column of AP
+    const int box = j >> 6, u = (j & 63) >> 3, e = j & 7;     // its box, 16-byte unit and element
+    // The four warps walk every unit even after a failed wait (their waits then return
+    // at once), so the named barrier below is always reached by all of them.
+    uint32_t ui = 0, it = 0;
+    bool ok = true;
+    SpanWalk walk;
+    walk.start(p, p.groups, group);
+    BptUnit x;
+    for (; walk.next(p, x); ++ui) {
+      if (ui > 0 && !wait(pempty, (ui - 1) & 1)) {
+        atomicOr(p.err, kErrTimeoutProducer);
+        ok = false;
+      }
+      ok = __all_sync(0xffffffffu, ok);   // tcgen05.st is warp-wide: one decision per warp
+      ptx::tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < kbn; ++c, ++it) {
+        const int st = it % NS;
+        if (!wait(&full[st], (it / NS) & 1)) {
+          atomicOr(p.err, kErrTimeoutProducer);
+          ok = false;
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        // token t of this column sits in row t of the box, 16-byte unit u ^ (t & 7)
+        // (128-byte swizzle); the 32 lanes read 64 consecutive bytes of one row
+        const uint8_t* col = smem + st * S::kStage + box * 8192 + e * 2;
+        uint32_t v[32];
+#pragma unroll
+        for (int tt = 0; tt < 32; ++tt) {
+          const int t0 = 2 * tt, t1 = 2 * tt + 1;
+          const uint32_t lo = *reinterpret_cast<const uint16_t*>(col + t0 * 128 + ((u ^ (t0 & 7)) << 4));
+          const uint32_t hi = *reinterpret_cast<const uint16_t*>(col + t1 * 128 + ((u ^ (t1 & 7)) << 4));
+          v[tt] = lo | (hi << 16);
+        }
+        nt_writer_bar();   // all four warps have read the chunk: its slot is free
+        if (warp == kNtAWriter0 && lane == 0) ptx::mbar_arrive(&empty[st]);
+        if (ok) ptx::tmem_st32(tmem_a + lane_base + c * 32, v);
+      }
+      it += (x.n1 - x.n0) * kbn;   // the unit's Gout stages
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (ok && lane == 0) ptx::mbar_arrive(pfull);
+    }
+  } else if (warp == 1) {
+    // ---------------- UMMA issuer ----------------
+    if (lane == 0) {
+      uint32_t ui = 0, ti = 0, it = 0;
+      bool ok = true;
+      SpanWalk walk;
+      walk.start(p, p.groups, group);
+      BptUnit x;
+      for (; ok && walk.next(p, x); ++ui) {
+        it += kbn;   // the unit's chunks of AP, consumed by the TMEM writers
+        if (!wait(pfull, ui & 1)) {
+          atomicOr(p.err, kErrTimeoutMma);
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t a0 = tmem_a;
+        for (int n = x.n0; ok && n < x.n1; ++n, ++ti) {
+          // the epilogue has the previous tile in registers
+          if (ti > 0 && !wait(accempty, (ti - 1) & 1)) {
+            atomicOr(p.err, kErrTimeoutMma);
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+#pragma unroll 1
+          for (int kb = 0; kb < kbn; ++kb, ++it) {
+            const int st = it % NS;
+            if (!wait(&full[st], (it / NS) & 1)) {
+              atomicOr(p.err, kErrTimeoutMma);
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t b_base = ptx::smem_u32(smem + st * S::kStage);
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k)   // 16 tokens per MMA: 8 TMEM columns of A
+              ptx::umma_bf16_tmem_a(tmem, a0 + kb * 32 + k * 8, ptx::desc_sw128(b_base + k * 2048, 8192, 1024),
+                                    kIdesc, (kb > 0 || k > 0) ? 1u : 0u);
+            ptx::umma_commit(&empty[st]);
+          }
+          ptx::umma_commit(accfull);
+        }
+        ptx::umma_commit(pempty);   // the unit's MMAs, the last readers of the block
+      }
+    }
+  } else {
+    // ---------------- epilogue: warps 2..9 ----------------
+    const int ew = warp - 2;
+    const int q = warp & 3;          // TMEM lanes (rows of the tile) 32q .. 32q+31
+    const int h = ew >> 2;           // 128-column half of the tile
+    uint4* rbox = reinterpret_cast<uint4*>(smem + S::kRBoxOff + ew * kRBox);
+    const uint32_t tsrc = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 128;
+    uint32_t ti = 0;
+    SpanWalk walk;
+    walk.start(p, p.groups, group);
+    BptUnit x;
+    // The epilogue warps walk every tile even after a failed wait (their waits then
+    // return at once), so the named barrier below is always reached by all of them.
+    while (walk.next(p, x)) {
+      const NtLayer& L = p.lay[x.g];
+      const int s = x.m_t;
+      for (int n = x.n0; n < x.n1; ++n, ++ti) {
+        const bool got = wait(accfull, ti & 1);
+        if (!got) atomicOr(p.err, kErrTimeoutEpilogue);
+        ptx::tc_fence_after();
+        // The MMAs of the next tile wait for this hand-over, so its path is short: load
+        // the first 64 columns, square them into four independent sums and stage them as
+        // bf16 in this warp's box (row `lane` at 128-byte row `lane`, unit uu at
+        // uu ^ (lane & 7)), load the other 64, release the accumulator, and only then
+        // work on those.
+        float sq[4] = {0.f, 0.f, 0.f, 0.f};
+        float v[64];
+        ptx::tmem_ld64(tsrc, v);
+#pragma unroll
+        for (int k = 0; k < 64; ++k) sq[k & 3] = fmaf(v[k], v[k], sq[k & 3]);
+        auto stage = [&]() {
+          __syncwarp();   // every lane has read the box's previous rows out
+#pragma unroll
+          for (int uu = 0; uu < 8; ++uu)
+            rbox[lane * 8 + (uu ^ (lane & 7))] =
+                make_uint4(pack_bf16(v[8 * uu + 0], v[8 * uu + 1]), pack_bf16(v[8 * uu + 2], v[8 * uu + 3]),
+                           pack_bf16(v[8 * uu + 4], v[8 * uu + 5]), pack_bf16(v[8 * uu + 6], v[8 * uu + 7]));
+          __syncwarp();
+        };
+        // the box's 32 rows x 64 columns out as whole 128-byte row pieces, four rows per
+        // instruction, to columns h * 128 + cc * 64 of the tile
+        auto write_out = [&](int cc) {
+          const int uu = lane & 7;
+          uint4* dst = reinterpret_cast<uint4*>(
+              L.Rst + (static_cast<size_t>(s) * p.r + mblk * kBM + q * 32 + (lane >> 3)) * L.d_out + n * kNtBN +
+              h * 128 + cc * 64 + 8 * uu);
+          const int step = L.d_out / 2;   // four rows of bf16, in 16-byte units
+#pragma unroll 2
+          for (int i = 0; i < 8; ++i) {
+            const int rr = 4 * i + (lane >> 3);
+            dst[i * step] = rbox[rr * 8 + (uu ^ (rr & 7))];
+          }
+        };
+        stage();
+        ptx::tmem_ld64(tsrc + 64, v);
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(accempty);
+#pragma unroll
+        for (int k = 0; k < 64; ++k) sq[k & 3] = fmaf(v[k], v[k], sq[k & 3]);
+        if (got) {
+          write_out(0);
+          stage();
+          write_out(1);
+        }
+        float ss = (sq[0] + sq[1]) + (sq[2] + sq[3]);
+        if (!got) ss = 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        float* rb = red + (ti & 1) * kEpiWarps;
+        if (lane == 0) rb[ew] = ss;
+        epi_bar();
+        // one partial slot per 128 columns: column half `lane` is its four warps' sum
+        if (ew == 0 && lane < 2) {
+          float tot = 0.0f;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) tot += rb[4 * lane + k];
+          p.partials[static_cast<size_t>(s) * p.part_stride + L.part_base + mblk * (2 * L.nt) + 2 * n + lane] =
+              tot;
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kNtTmemCols);
   }
 }
 
@@ -1547,6 +1951,12 @@ struct HostState {
   int bn_project = 128;
   GroupParams gp;   // host staging of one launch's kernel parameters
   BptParams bp;     // the same for tc_backproj_tmem_kernel
+  NtParams np;      // the same for tc_norm_tmem_kernel
+  // GRAPE_NORM_TMEM in the environment when the context is created: 0 runs the norms on
+  // tc_gemm_kernel<NORM / NORMST> for every T, 1 runs tc_norm_tmem_kernel wherever it
+  // can (stored R_i, T <= 512); unset, tc_norm_a_in_tmem decides by T (a measurement
+  // and test knob: both kernels compute the same partial slots and R_i)
+  int norm_tmem = -1;
 };
 
 int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
@@ -1698,7 +2108,8 @@ bool tc_supported(int device, const grape_layer* layers, int n_layers, int r, in
   return true;
 }
 
-int tc_partials_per_sample(int r, int d_out) { return cdiv(r, kBM) * cdiv(d_out, kBnWide); }
+// One slot per 128 x 128 tile of R_i (row block of r, 128 columns of d_out).
+int tc_partials_per_sample(int r, int d_out) { return cdiv(r, kBM) * cdiv(d_out, 128); }
 
 size_t tc_workspace_bytes(const StepShape&, const LayerWs*) {
   return 256;  // error word
@@ -1712,6 +2123,7 @@ cudaError_t tc_init(const StepShape& sh, const LayerWs* ws, void* scratch, size_
   hs->B = sh.B;
   hs->T = sh.T;
   hs->bn_project = sh.r == 128 ? 128 : 256;
+  if (const char* v = std::getenv("GRAPE_NORM_TMEM")) hs->norm_tmem = std::strcmp(v, "0") == 0 ? 0 : 1;
   char* base = static_cast<char*>(scratch);
   size_t off = 0;
   hs->err = reinterpret_cast<int*>(base + off);
@@ -1840,10 +2252,88 @@ cudaError_t tc_project(const StepShape& sh, const LayerWs* ws, const LayerIo* io
   return run_mode<PROJECT, 256, kStagesProject256>(hs, sh.L, st, launches, fill, gp, !first_in_step);
 }
 
+namespace {
+
+cudaError_t launch_norm_tmem(NtParams& np, cudaStream_t st) {
+  using S = NtSmem;
+  const void* kern = reinterpret_cast<const void*>(tc_norm_tmem_kernel);
+  int per_sm = 0;
+  cudaError_t e = configure_kernel(kern, S::kBytes, kNtThreads, &per_sm);
+  if (e != cudaSuccess) return e;
+  int most = 0;   // no more groups than the largest span has column tiles
+  for (int k = 0; k < np.n_spans; ++k) most = std::max(most, np.span_tiles[k]);
+  if (most <= 0) return cudaSuccess;
+  int groups = sm_count() * per_sm / np.mr;   // one CTA per SM (the kernel allocates TMEM)
+  groups = std::max(1, std::min(groups, most));
+  np.groups = groups;
+  int rot = 0;
+  for (int k = 0; k < np.n_spans; ++k) {
+    np.span_rot[k] = rot;
+    rot = ((rot - np.span_tiles[k] % groups) % groups + groups) % groups;
+  }
+  return launch_maybe_pdl(true, tc_norm_tmem_kernel, dim3(groups * np.mr), dim3(kNtThreads), S::kBytes, st, np);
+}
+
+}  // namespace
+
+// The norm kernel with (A_i P)^T in TMEM stores R_i and holds a block of
+// ceil(T / 64) * 32 columns next to its accumulator: T up to 512.  Against
+// tc_gemm_kernel<NORMST> it measured faster from T = 257 on (7B slice, T = 512: 1.37
+// against 1.52 ms per step's norms) and slower at ViT-B's T = 197, where its block
+// changes more often per tile.  `mode` is the GRAPE_NORM_TMEM knob: 0 never, 1 for
+// every T it can take, -1 (unset) by that measurement.
+bool tc_norm_a_in_tmem(int T, bool store_R, int mode) {
+  if (!store_R || mode == 0 || T < 1 || T > 512) return false;
+  return mode == 1 || T > 256;
+}
+
 cudaError_t tc_project_norm(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                             const TcWorkspace& tc, float* partials, bool store_R, cudaStream_t st,
                             int* launches) {
   HostState& hs = *static_cast<HostState*>(tc.host_state);
+  if (tc_norm_a_in_tmem(sh.T, store_R, hs.norm_tmem)) {
+    NtParams& np = hs.np;
+    for (int l0 = 0; l0 < sh.L; l0 += kMaxGroup) {
+      const int n = (sh.L - l0) < kMaxGroup ? (sh.L - l0) : kMaxGroup;
+      std::memset(&np, 0, sizeof(np));
+      np.err = hs.err;
+      np.partials = partials;
+      np.part_stride = sh.part_stride;
+      np.r = sh.r;
+      np.mr = cdiv(sh.r, kBM);
+      np.kblocks = cdiv(sh.T, kBK);
+      np.n_layers = n;
+      // one span: the groups share nothing, so each takes one contiguous range of the
+      // whole launch (the fewest unit starts)
+      np.n_spans = 1;
+      np.span_first[0] = 0;
+      np.span_first[1] = n;
+      int tiles = 0;
+      for (int g = 0; g < n; ++g) {
+        const int l = l0 + g;
+        np.mapAP[g] = hs.mapAP3[l];
+        if (!hs.cacheG3[l].get(io[l].G, &np.mapG[g], [&](CUtensorMap* m) {
+              return map_3d(m, io[l].G, sh.B, sh.T, ws[l].d_out);
+            }))
+          return cudaErrorInvalidValue;
+        if (!ws[l].Rst) return cudaErrorInvalidValue;
+        GRAPE_EXT(np.extAP[g], sh.r, sh.T, sh.B)
+        GRAPE_EXT(np.extG[g], ws[l].d_out, sh.T, sh.B)
+        NtLayer& L = np.lay[g];
+        L.tiles_begin = tiles;
+        L.nt = cdiv(ws[l].d_out, kNtBN);   // d_out % 256 == 0 on this path
+        L.d_out = ws[l].d_out;
+        L.part_base = ws[l].part_base;
+        L.Rst = ws[l].Rst;
+        tiles += sh.B * L.nt;
+      }
+      np.span_tiles[0] = tiles;
+      cudaError_t e = launch_norm_tmem(np, st);
+      if (e != cudaSuccess) return e;
+      ++*launches;
+    }
+    return cudaSuccess;
+  }
   GroupParams& gp = hs.gp;
   std::memset(&gp, 0, sizeof(gp));
   gp.err = hs.err;
@@ -2233,7 +2723,7 @@ size_t tc_static_scratch_bytes() { return kStaticScratchBytes; }
 bool tc_tensor_maps_available() { return encode_fn() != nullptr; }
 
 size_t tc_static_scratch_needed(int d_in, int d_out, int r, int B, int T) {
-  const size_t slots = static_cast<size_t>(cdiv(r, kBM)) * cdiv(d_out, kBnWide);
+  const size_t slots = static_cast<size_t>(tc_partials_per_sample(r, d_out));
   return 256 + round256(static_cast<size_t>(d_in) * r * 2) +
          round256(static_cast<size_t>(B) * T * r * 2) + round256(static_cast<size_t>(B) * slots * 4);
 }
@@ -2264,7 +2754,7 @@ cudaError_t tc_layer_sqnorms_static(const void* A, const void* G, int d_in, int 
   __nv_bfloat16* AP = reinterpret_cast<__nv_bfloat16*>(base + 256 + round256(static_cast<size_t>(d_in) * r * 2));
   float* partials = reinterpret_cast<float*>(reinterpret_cast<char*>(AP) +
                                              round256(static_cast<size_t>(B) * T * r * 2));
-  const int slots = cdiv(r, kBM) * cdiv(d_out, kBnWide);
+  const int slots = tc_partials_per_sample(r, d_out);
   const int64_t rows = static_cast<int64_t>(B) * T;
 
   // The error word is the only state that must start at zero; P, AP and every

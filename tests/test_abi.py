@@ -121,13 +121,14 @@ def test_context_bytes_is_the_documented_arena(lib):
     B = 64, T = 128, bf16, tensor-core path), block by block, each rounded up to 256 B:
     every S_l 4 r sum(d_out) = 2 MiB; per layer P 2 d_in r = 256 KiB, AP 2 B T r = 2 MiB,
     m and v 4 r d_out = 512 KiB each, dR 2 r d_out = 256 KiB; then the norm partials
-    (B x 16 slots x 4 B), norms, clip factors and the 256-byte error word."""
+    (B x 32 slots x 4 B: one per 128 x 128 tile of each R_i, 8 per layer), norms, clip
+    factors and the 256-byte error word."""
     from random_gradient_projection_b200 import grape
     layers = [(1024, 1024)] * 4
     KiB, MiB = 1024, 1 << 20
     per_layer = 256 * KiB + 2 * MiB + 2 * 512 * KiB + 256 * KiB
-    expect = 2 * MiB + 4 * per_layer + 64 * 16 * 4 + 256 + 256 + 256
-    assert grape.grape_context_bytes(layers, 128, 64, 128, grape.GRAPE_BF16) == expect == 16_782_080
+    expect = 2 * MiB + 4 * per_layer + 64 * 32 * 4 + 256 + 256 + 256
+    assert grape.grape_context_bytes(layers, 128, 64, 128, grape.GRAPE_BF16) == expect == 16_786_176
     # the fp32 CUDA-core path: fp32 P, AP and dR, one 64 x 64 partial slot per layer here
     tiny = grape.grape_context_bytes([(64, 32)], 8, 4, 16, grape.GRAPE_F32)
     assert tiny == 1024 + 2048 + 2048 + 1024 + 1024 + 1024 + 3 * 256

@@ -77,6 +77,13 @@ CASES = {
     # ragged last M tile of W, both at the edge of their TMA boxes
     "ragged_d_in_tc": (W.Workload("ragged_din", ((520, 256), (136, 512)), r=128, B=3, T=40,
                                   dtype="bf16", C=1.0, sigma=0.8, steps=2), 2),
+    # the norm kernel's one 256-column block of (A_i P)^T in TMEM (T in 257..512): eight
+    # 64-token chunks, the last one ragged, r = 256 (groups of two CTAs)
+    "r256_T500": (W.Workload("r256_T500", ((512, 768), (768, 512)), r=256, B=3, T=500,
+                             dtype="bf16", C=1.0, sigma=0.7, steps=2), 2),
+    # the per-layer shape of the 7B-slice workload at small widths: r = 512, T = 512
+    "r512_T512": (W.Workload("r512_T512", ((512, 1024), (1024, 512)), r=512, B=2, T=512,
+                             dtype="bf16", C=1.0, sigma=1.0, steps=2), 2),
 }
 
 
@@ -105,7 +112,7 @@ def test_step_matches_oracle(case, path):
 
 
 STORE_CASES = ["mlp_2x1024_B4", "vit_qkv_down_B3", "longctx_1layer_T1000", "r512_T130", "20_layers",
-               "ragged_d_in_tc", "T1_bf16_tc", "no_noise_bf16"]
+               "ragged_d_in_tc", "T1_bf16_tc", "no_noise_bf16", "r256_T500", "r512_T512"]
 
 
 @pytest.mark.parametrize("case", STORE_CASES)
@@ -120,6 +127,37 @@ def test_aggregation_methods_match_oracle(case, agg):
     worst = compare(w, lib, orc, 2e-2, steps)
     print(case, "store" if agg == grape.GRAPE_AGG_STORE else "recompute",
           {k: f"{v:.2e}" for k, v in worst.items()})
+
+
+# (the TMEM norm kernel takes T <= 512 and only with the stored aggregation)
+TMEM_NORM_CASES = ["T1_bf16_tc", "r512_T130", "vit_qkv_down_B3", "20_layers", "ragged_d_in_tc", "r256_T500"]
+
+
+@pytest.mark.parametrize("case", TMEM_NORM_CASES)
+def test_both_norm_kernels_match_oracle_and_each_other(case, monkeypatch):
+    """With the stored aggregation the norms run on the kernel that keeps (A_i P)^T in
+    TMEM for 256 < T <= 512 and on the streamed kernel otherwise.  GRAPE_NORM_TMEM=1 and
+    =0 force one or the other for every T up to 512: T = 1, a ragged last 64-token chunk,
+    more layers than one launch holds, r = 128 / 256 / 512.  Each against the oracle,
+    and against each other: the same bf16 products summed in fp32 in another order, so
+    the norms and the S built from the stored R_i agree far inside the parity
+    tolerance."""
+    w, steps = CASES[case]
+    store = lambda g: g.set_aggregation(grape.GRAPE_AGG_STORE)   # noqa: E731
+    runs = {}
+    for mode in ("0", "1"):
+        monkeypatch.setenv("GRAPE_NORM_TMEM", mode)
+        runs[mode] = run_library(w, steps, TC, setup=store)
+    monkeypatch.delenv("GRAPE_NORM_TMEM")
+    orc = run_oracle(w, steps)
+    for mode, lib in runs.items():
+        worst = compare(w, lib, orc, 2e-2, steps)
+        print(case, "tmem" if mode == "1" else "streamed", {k: f"{v:.2e}" for k, v in worst.items()})
+    for t in range(steps):
+        a, b = runs["0"]["trace"][t], runs["1"]["trace"][t]
+        assert rel_fro(a["norms"], b["norms"]) < 1e-4, t
+        for l in range(w.n_layers):
+            assert rel_fro(a["S"][l], b["S"][l]) < 1e-3, (t, l)
 
 
 def test_auto_aggregation_follows_tokens_per_sample():
