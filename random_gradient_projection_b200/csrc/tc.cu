@@ -709,33 +709,44 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
 // contiguous range of the span's T tiles (numbered layer by layer, row block by row
 // block): T / grid of them, one more for T % grid of the CTAs, with the CTAs that take
 // the extra tile rotating from span to span, so the whole launch is balanced to within
-// one tile and all CTAs work on the same span at once (its P and dR stay in L2).  A work unit is the part of a CTA's range in one
-// 128-row block: the block of P is written into TMEM once per unit, and per tile only
-// dR (r x 128 bf16, from L2) and W (from DRAM) stream through shared memory, which
-// holds nothing but those streams.  Next to
-// tc_gemm_kernel<BACKPROJ>, which loads P with every tile, this moves 192 instead of
-// 320 bytes from L2 into the SM per 64 bytes of W read, with the same bytes in flight.
+// one tile and all CTAs work on the same span at once (its P and dR stay in L2).  A
+// work unit is the part of a CTA's range in one 128-row block: the block of P is
+// written into TMEM once per unit, and per tile only dR (r x 128 bf16, from L2) and W
+// (from DRAM) stream through shared memory, which holds nothing but those streams.
+// Next to tc_gemm_kernel<BACKPROJ>, which loads P with every tile, this moves 192
+// instead of 320 bytes from L2 into the SM per 64 bytes of W read, with the same bytes
+// in flight.
+//
+// The block of P comes by TMA in 64-column chunks (128 rows x 64 bf16, 16 KB, rows past
+// d_in zero-filled) through the dR ring: the ring holds, in order, the chunks of unit 0,
+// its dR stages, the chunks of unit 1, its dR stages, and so on, so a unit's chunks are
+// loaded while the previous unit's last dR stages are consumed.  The writers of a unit's
+// block wait until the MMAs of the previous unit are done, which keeps the ring's parity
+// waits sound: a consumer waits for a ring position only once the position DRS earlier
+// has been loaded (an mbarrier parity wait for phase k returns at once while phase k - 1
+// is still open).
 //
 // W streams through a ring of 32-column boxes (128 rows x 32 fp32, 16 KB) that runs
 // ahead of the tiles; each epilogue warp updates its 32 rows of a box in shared memory
 // and stores them with a TMA tile store; a box's slot is reloaded once its four row
 // quarters have been read out.
 //
-// TMEM: two 128 x 128 fp32 accumulators (columns 0..255) and NPB P blocks of r/2
-// columns each (lane = row of P, two bf16 of consecutive k per 32-bit column).
-// Warps: 0 loads dR (written earlier in the step, after griddepcontrol.wait); 1 owns TMEM
-// and issues the MMAs; 2-9 are the epilogue (warp w: lane quarter w % 4, column half
-// (w - 2) / 4); 10 loads W (written by the previous step, whose work every step's first,
-// ordinary launch waits for, so its loads start at once); 11-14 write P into TMEM (warp
-// w: lane quarter w % 4, one row of P per thread, read from global memory).
+// TMEM: two 128 x 128 fp32 accumulators (columns 0..255) and the P block of r/2 columns
+// (lane = row of P, two bf16 of consecutive k per 32-bit column).
+// Warps: 0 loads the ring, P chunks and dR (both written earlier in the step, after
+// griddepcontrol.wait); 1 owns TMEM and issues the MMAs; 2-9 are the epilogue (warp w:
+// lane quarter w % 4, column half (w - 2) / 4); 10 loads W (written by the previous
+// step, whose work every step's first, ordinary launch waits for, so its loads start at
+// once); 11-14 write P into TMEM (warp w: lane quarter w % 4, one row of P per thread,
+// read from its chunk in shared memory).
 struct BptLayer {
   int tiles_begin;   // first tile of this layer in its span
   int M;             // rows of W and of P (d_in)
   int mt, nt;        // 128-row blocks of W, 128-column tiles of W
-  const __nv_bfloat16* P;   // d_in x r, row-major
 };
 
 struct BptParams {
+  CUtensorMap mapP[kMaxGroup];    // P: bf16 d_in x r, boxes of 64 columns x 128 rows
   CUtensorMap mapDR[kMaxGroup];   // dR: bf16 r x d_out, boxes of 64 x 64
   CUtensorMap mapW[kMaxGroup];    // W: fp32 d_in x d_out, load boxes of 32 columns x 128 rows
   CUtensorMap mapWs[kMaxGroup];   // W, store boxes of 32 columns x 32 rows
@@ -749,6 +760,7 @@ struct BptParams {
   float lr;
   int* err;
 #ifdef GRAPE_CHECKED
+  int extP[kMaxGroup][3];
   int extDR[kMaxGroup][3];
   int extW[kMaxGroup][3];
 #endif
@@ -806,10 +818,10 @@ struct SpanWalk {
 };
 using BptWalk = SpanWalk;
 
-// DRS dR stages and NW W boxes in shared memory.
+// DRS ring stages (dR, or a chunk of P) and NW W boxes in shared memory.
 template <int DRS, int NW>
 struct BptSmem {
-  static constexpr int kDRStage = kBK * kBnBack * 2;        // 64 x 128 bf16: 16 KB
+  static constexpr int kDRStage = kBK * kBnBack * 2;        // 64 x 128 bf16: 16 KB (a P chunk too)
   static constexpr int kDROff = 0;
   static constexpr int kWOff = DRS * kDRStage;
   static constexpr int kBarOff = kWOff + NW * kWBox;
@@ -819,32 +831,35 @@ struct BptSmem {
 constexpr int kBptThreads = 32 * 15;
 constexpr int kBptWProducer = 10;
 constexpr int kBptPWriter0 = 11;    // warps 11..14
+
+__device__ __forceinline__ void bpt_writer_bar() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 constexpr uint32_t kBptTmemCols = 512;
 constexpr int kBptDRS = 6;
 constexpr int kBptNW = 8;
 
-// PK = r / 64 k-blocks, NPB P blocks in TMEM (PK * 32 columns each).
-template <int PK, int NPB>
+// PK = r / 64 k-blocks: the P block takes PK * 32 TMEM columns.
+template <int PK>
 __global__ void __launch_bounds__(kBptThreads, 1) tc_backproj_tmem_kernel(const __grid_constant__ BptParams p) {
   constexpr int DRS = kBptDRS, NW = kBptNW;
   using S = BptSmem<DRS, NW>;
   constexpr uint32_t kIdesc = ptx::idesc_bf16(kBM, kBnBack, false, true);   // A K-major (TMEM), dR N-major
   constexpr int kBoxes = kBnBack / 32;                                     // W boxes per tile
   constexpr uint32_t kPCols = PK * 32;                                     // TMEM columns of one P block
-  static_assert(2 * kBnBack + NPB * kPCols <= kBptTmemCols, "TMEM columns");
+  static_assert(2 * kBnBack + kPCols <= kBptTmemCols, "TMEM columns");
+  static_assert(S::kDRStage == kBK * kBM * 2, "a P chunk fills one ring stage");
   // A slot of the W ring must only ever hold boxes of one column half, so that the four
   // warps that wait on its wfull barrier have consumed its previous use themselves: a
   // parity wait cannot tell a phase two ahead from the one behind, and a warp of the other
   // half waiting for the slot's next use would pass at once on the previous phase.
   static_assert(NW % kBoxes == 0, "W ring slots must map to one box position of a tile");
-  static_assert((2 * NPB + 2 * DRS + 4 + 2 * NW) * 8 + 16 <= 512, "barrier area");
+  static_assert((2 + 2 * DRS + 4 + 2 * NW) * 8 + 16 <= 512, "barrier area");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* pfull = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
-  uint64_t* pempty = pfull + NPB;
-  uint64_t* full = pempty + NPB;
+  uint64_t* pfull = reinterpret_cast<uint64_t*>(smem + S::kBarOff);   // the P block is in TMEM
+  uint64_t* pempty = pfull + 1;                                          // its MMAs are done
+  uint64_t* full = pempty + 1;
   uint64_t* empty = full + DRS;
   uint64_t* accfull = empty + DRS;     // [2]
   uint64_t* accempty = accfull + 2;    // [2]
@@ -861,10 +876,8 @@ __global__ void __launch_bounds__(kBptThreads, 1) tc_backproj_tmem_kernel(const 
 
   if (warp == 0 && lane == 0) {
     *abort_flag = 0;
-    for (int b = 0; b < NPB; ++b) {
-      ptx::mbar_init(&pfull[b], 4);    // the four P-writing warps
-      ptx::mbar_init(&pempty[b], 1);
-    }
+    ptx::mbar_init(pfull, 4);    // the four P-writing warps
+    ptx::mbar_init(pempty, 1);
     for (int st = 0; st < DRS; ++st) {
       ptx::mbar_init(&full[st], 1);
       ptx::mbar_init(&empty[st], 1);
@@ -879,6 +892,7 @@ __global__ void __launch_bounds__(kBptThreads, 1) tc_backproj_tmem_kernel(const 
     }
     ptx::fence_mbar_init();
     for (int g = 0; g < p.n_layers; ++g) {
+      ptx::prefetch_tmap(&p.mapP[g]);
       ptx::prefetch_tmap(&p.mapDR[g]);
       ptx::prefetch_tmap(&p.mapW[g]);
       ptx::prefetch_tmap(&p.mapWs[g]);
@@ -892,12 +906,12 @@ __global__ void __launch_bounds__(kBptThreads, 1) tc_backproj_tmem_kernel(const 
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_p = tmem + 2 * kBnBack;   // P blocks after the two accumulators
+  const uint32_t tmem_p = tmem + 2 * kBnBack;   // the P block after the two accumulators
 
   if (warp == 0) {
-    // ---------------- dR ----------------
+    // ---------------- the ring: each unit's chunks of P, then its dR stages ----------------
     if (lane == 0) {
-      const uint64_t pol = ptx::policy_evict_last();   // dR is read by every row block
+      const uint64_t pol = ptx::policy_evict_last();   // dR and P are read by many units
       ptx::griddep_wait();
       uint32_t it = 0, it_issued = 0;
       bool ok = true;
@@ -905,6 +919,21 @@ __global__ void __launch_bounds__(kBptThreads, 1) tc_backproj_tmem_kernel(const 
       walk.start(p);
       BptUnit x;
       while (ok && walk.next(p, x)) {
+#pragma unroll 1
+        for (int c = 0; c < PK; ++c, ++it) {
+          const int st = it % DRS;
+          const uint32_t use = it / DRS;
+          if (use > 0 && !wait(&empty[st], (use - 1) & 1)) {
+            atomicOr(p.err, kErrTimeoutProducer);
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(&full[st], S::kDRStage);
+          GRAPE_BOX(p.err, p.extP[x.g], 2, c * kBK, x.m_t * kBM, 0)
+          ptx::tma_load_2d_hint(smem + S::kDROff + st * S::kDRStage, &p.mapP[x.g], &full[st], c * kBK, x.m_t * kBM,
+                                pol);
+          it_issued = it + 1;
+        }
         for (int n = x.n0; ok && n < x.n1; ++n) {
 #pragma unroll 1
           for (int kb = 0; kb < PK; ++kb, ++it) {
@@ -965,48 +994,49 @@ __global__ void __launch_bounds__(kBptThreads, 1) tc_backproj_tmem_kernel(const 
     // ---------------- P into TMEM: one row of the block per thread ----------------
     const int q = warp & 3;                       // TMEM lanes 32q .. 32q+31
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    ptx::griddep_wait();                          // P is generated earlier in this step
-    uint32_t ui = 0;
+    const int row = q * 32 + lane;                // row of the block
+    // The four warps walk every unit even after a failed wait (their waits then return
+    // at once), so the named barrier below is always reached by all of them.
+    uint32_t ui = 0, it = 0;
+    bool ok = true;
     BptWalk walk;
     walk.start(p);
     BptUnit x;
     for (; walk.next(p, x); ++ui) {
-      const BptLayer& L = p.lay[x.g];
-      const int pb = ui % NPB;
-      const uint32_t puse = ui / NPB;
-      if (puse > 0 && !wait(&pempty[pb], (puse - 1) & 1)) {
+      if (ui > 0 && !wait(pempty, (ui - 1) & 1)) {
         atomicOr(p.err, kErrTimeoutProducer);
-        break;
+        ok = false;
       }
+      ok = __all_sync(0xffffffffu, ok);   // tcgen05.st is warp-wide: one decision per warp
       ptx::tc_fence_after();
-      const int m = x.m_t * kBM + q * 32 + lane;
-      const bool valid = m < L.M;                 // rows past d_in are zero
-      const uint4* src = reinterpret_cast<const uint4*>(L.P + static_cast<size_t>(valid ? m : 0) * p.r);
-      // 64 bf16 (32 TMEM columns, eight 16-byte loads) per chunk; the next chunk's loads
-      // are in flight while this chunk is stored
-      uint32_t now[32], nxt[32];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint4 v = valid ? __ldg(src + k) : make_uint4(0u, 0u, 0u, 0u);
-        now[4 * k] = v.x; now[4 * k + 1] = v.y; now[4 * k + 2] = v.z; now[4 * k + 3] = v.w;
-      }
 #pragma unroll 1
-      for (int c = 0; c < PK; ++c) {
-        if (c + 1 < PK) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint4 v = valid ? __ldg(src + (c + 1) * 8 + k) : make_uint4(0u, 0u, 0u, 0u);
-            nxt[4 * k] = v.x; nxt[4 * k + 1] = v.y; nxt[4 * k + 2] = v.z; nxt[4 * k + 3] = v.w;
-          }
+      for (int c = 0; c < PK; ++c, ++it) {
+        const int st = it % DRS;
+        if (!wait(&full[st], (it / DRS) & 1)) {
+          atomicOr(p.err, kErrTimeoutProducer);
+          ok = false;
         }
-        ptx::tmem_st32(tmem_p + lane_base + pb * kPCols + c * 32, now);
+        ok = __all_sync(0xffffffffu, ok);
+        // row `row` of the chunk: 16-byte unit uu at uu ^ (row & 7) (128-byte swizzle)
+        const uint4* src = reinterpret_cast<const uint4*>(smem + S::kDROff + st * S::kDRStage + row * 128);
+        uint32_t v[32];
 #pragma unroll
-        for (int k = 0; k < 32; ++k) now[k] = nxt[k];
+        for (int uu = 0; uu < 8; ++uu) {
+          const uint4 w = src[uu ^ (row & 7)];
+          v[4 * uu] = w.x;
+          v[4 * uu + 1] = w.y;
+          v[4 * uu + 2] = w.z;
+          v[4 * uu + 3] = w.w;
+        }
+        bpt_writer_bar();   // all four warps have read the chunk: its slot is free
+        if (warp == kBptPWriter0 && lane == 0) ptx::mbar_arrive(&empty[st]);
+        if (ok) ptx::tmem_st32(tmem_p + lane_base + c * 32, v);
       }
+      it += (x.n1 - x.n0) * PK;   // the unit's dR stages
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&pfull[pb]);
+      if (ok && lane == 0) ptx::mbar_arrive(pfull);
     }
   } else if (warp == 1) {
     // ---------------- UMMA issuer ----------------
@@ -1017,13 +1047,13 @@ __global__ void __launch_bounds__(kBptThreads, 1) tc_backproj_tmem_kernel(const 
       walk.start(p);
       BptUnit x;
       for (; ok && walk.next(p, x); ++ui) {
-        const int pb = ui % NPB;
-        if (!wait(&pfull[pb], (ui / NPB) & 1)) {
+        it += PK;   // the unit's chunks of P, consumed by the TMEM writers
+        if (!wait(pfull, ui & 1)) {
           atomicOr(p.err, kErrTimeoutMma);
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t a0 = tmem_p + pb * kPCols;
+        const uint32_t a0 = tmem_p;
         for (int n = x.n0; ok && n < x.n1; ++n, ++ti) {
           const int b = ti & 1;
           const uint32_t use = ti >> 1;
@@ -1052,7 +1082,7 @@ __global__ void __launch_bounds__(kBptThreads, 1) tc_backproj_tmem_kernel(const 
           }
           ptx::umma_commit(&accfull[b]);
         }
-        ptx::umma_commit(&pempty[pb]);   // the unit's MMAs, the last readers of this P block
+        ptx::umma_commit(pempty);   // the unit's MMAs, the last readers of the P block
       }
     }
   } else {
@@ -2560,10 +2590,10 @@ cudaError_t tc_aggregate(const StepShape& sh, const LayerWs* ws, const LayerIo* 
 
 namespace {
 
-template <int PK, int NPB>
+template <int PK>
 cudaError_t launch_backproj_tmem(BptParams& bp, cudaStream_t st) {
   using S = BptSmem<kBptDRS, kBptNW>;
-  const void* kern = reinterpret_cast<const void*>(tc_backproj_tmem_kernel<PK, NPB>);
+  const void* kern = reinterpret_cast<const void*>(tc_backproj_tmem_kernel<PK>);
   int per_sm = 0;
   cudaError_t e = configure_kernel(kern, S::kBytes, kBptThreads, &per_sm);
   if (e != cudaSuccess) return e;
@@ -2578,7 +2608,7 @@ cudaError_t launch_backproj_tmem(BptParams& bp, cudaStream_t st) {
     bp.span_rot[k] = rot;
     rot = ((rot - bp.span_tiles[k] % grid) % grid + grid) % grid;
   }
-  return launch_maybe_pdl(true, tc_backproj_tmem_kernel<PK, NPB>, dim3(grid), dim3(kBptThreads), S::kBytes, st,
+  return launch_maybe_pdl(true, tc_backproj_tmem_kernel<PK>, dim3(grid), dim3(kBptThreads), S::kBytes, st,
                           bp);
 }
 
@@ -2609,6 +2639,7 @@ cudaError_t tc_backproject(const StepShape& sh, const LayerWs* ws, const LayerIo
     int span_tiles = 0;
     for (int g = 0; g < n; ++g) {
       const int l = l0 + g;
+      bp.mapP[g] = hs.mapP_k[l];
       bp.mapDR[g] = hs.mapDR[l];
       if (!hs.cacheW[l].get(io[l].W, &bp.mapW[g], [&](CUtensorMap* m) {
             return map_2d_f32(m, io[l].W, ws[l].d_in, ws[l].d_out);
@@ -2617,13 +2648,13 @@ cudaError_t tc_backproject(const StepShape& sh, const LayerWs* ws, const LayerIo
             return map_2d_f32(m, io[l].W, ws[l].d_in, ws[l].d_out, 32);
           }))
         return cudaErrorInvalidValue;
+      GRAPE_EXT(bp.extP[g], sh.r, ws[l].d_in, 1)
       GRAPE_EXT(bp.extDR[g], ws[l].d_out, sh.r, 1)
       GRAPE_EXT(bp.extW[g], ws[l].d_out, ws[l].d_in, 1)
       BptLayer& L = bp.lay[g];
       L.M = ws[l].d_in;
       L.mt = cdiv(ws[l].d_in, kBM);
       L.nt = cdiv(ws[l].d_out, kBnBack);
-      L.P = ws[l].P16;
       // spans of at least four tiles per CTA
       if (span_tiles == 0) bp.span_first[bp.n_spans] = g;
       L.tiles_begin = span_tiles;
@@ -2634,7 +2665,7 @@ cudaError_t tc_backproject(const StepShape& sh, const LayerWs* ws, const LayerIo
       }
     }
     bp.span_first[bp.n_spans] = n;
-    cudaError_t e = launch_backproj_tmem<8, 1>(bp, st);   // r = 512: one 256-column P block
+    cudaError_t e = launch_backproj_tmem<8>(bp, st);   // r = 512: a 256-column P block
     if (e != cudaSuccess) return e;
     ++*launches;
   }

@@ -81,6 +81,10 @@ CASES = {
     # 64-token chunks, the last one ragged, r = 256 (groups of two CTAs)
     "r256_T500": (W.Workload("r256_T500", ((512, 768), (768, 512)), r=256, B=3, T=500,
                              dtype="bf16", C=1.0, sigma=0.7, steps=2), 2),
+    # r = 512 (the back-projection with P in TMEM) with d_in off the 128-row block: the
+    # last block of P is partly past d_in (8 of its 128 rows)
+    "r512_ragged_d_in": (W.Workload("r512_ragged", ((520, 256), (648, 512)), r=512, B=2, T=40,
+                                    dtype="bf16", C=1.0, sigma=0.8, steps=2), 2),
     # the per-layer shape of the 7B-slice workload at small widths: r = 512, T = 512
     "r512_T512": (W.Workload("r512_T512", ((512, 1024), (1024, 512)), r=512, B=2, T=512,
                              dtype="bf16", C=1.0, sigma=1.0, steps=2), 2),
