@@ -202,11 +202,15 @@ def phase_work(w, path: str, agg: str = "recompute"):
     out["aggregate"] = {"bytes": sum(rows * do * el + rows * w.r * ap_el + 4 * w.r * do
                                      for _, do in w.layers),
                         "flops": sum(2 * rows * w.r * do for _, do in w.layers)}
+    out["adam"] = {"bytes": sum(w.r * do * (4 + 16 + dr_el) for _, do in w.layers), "flops": 0}
     if agg == "store":
         r_bytes = sum(2 * w.B * w.r * do for _, do in w.layers)
         out["norm"]["bytes"] += r_bytes
         out["aggregate"] = {"bytes": r_bytes + sum(4 * w.r * do for _, do in w.layers), "flops": 0}
-    out["adam"] = {"bytes": sum(w.r * do * (4 + 16 + dr_el) for _, do in w.layers), "flops": 0}
+        # a one-process step sums the R_i inside noise + Adam: R_i read, S written (kept
+        # for inspection), m and v read and written, dR written; S is not read back
+        out["aggregate_adam"] = {"bytes": r_bytes + sum(w.r * do * (4 + 16 + dr_el) for _, do in w.layers),
+                                 "flops": 0}
     out["backproject"] = {"bytes": sum(8 * di * do + di * w.r * ap_el + w.r * do * dr_el
                                        for di, do in w.layers),
                           "flops": sum(2 * di * w.r * do for di, do in w.layers)}

@@ -302,7 +302,9 @@ enum grape_phase {
   GRAPE_PHASE_ADAM = 5,         /* noise + projected Adam */
   GRAPE_PHASE_BACKPROJECT = 6,  /* W -= lr P dR */
   GRAPE_PHASE_COMPACT = 7,      /* live-token scan and gather (grape_step_masked) */
-  GRAPE_N_PHASES = 8
+  GRAPE_PHASE_AGGREGATE_ADAM = 8, /* S = sum_i c_i R_i fused with noise + Adam: a step with
+                                     the stored aggregation, in place of phases 4 and 5 */
+  GRAPE_N_PHASES = 9
 };
 GRAPE_API int grape_profile(grape_ctx* ctx, int32_t enable);
 GRAPE_API int grape_profile_read(grape_ctx* ctx, double* ms_out, int64_t* count_out);

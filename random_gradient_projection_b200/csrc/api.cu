@@ -72,6 +72,12 @@ struct grape_ctx {
   int agg = GRAPE_AGG_RECOMPUTE;
   void* rst_buf = nullptr;
   bool stores_R() const { return agg == GRAPE_AGG_STORE && norm_method == GRAPE_NORM_DIRECT; }
+  // A one-process step with the stored aggregation sums the R_i inside the noise + Adam
+  // kernel (tc_aggregate_adam); grape_accumulate / grape_apply keep them apart, since S
+  // is all-reduced in between.  GRAPE_FUSE_ADAM=0 in the environment at grape_create
+  // keeps them apart in every step too (a measurement knob: both give the same bits).
+  bool fuse_adam = true;
+  bool fuses_adam() const { return fuse_adam && path == GRAPE_PATH_TC && stores_R(); }
   // CUDA-graph replay of grape_step (grape_set_graph): one graph per set of A, Gout, W
   // pointers; the first step with a set captures it, later ones replay it
   struct StepGraph {
@@ -81,6 +87,7 @@ struct grape_ctx {
     cudaGraph_t graph = nullptr;
     cudaGraphExec_t exec = nullptr;
     cudaGraphNode_t gen_p = nullptr, adam = nullptr;
+    bool adam_fused = false;   // the Adam node is tc_aggregate_adam's
     uint64_t launches = 0, used = 0;
   };
   bool graph_on = false;
@@ -266,8 +273,10 @@ int run_project_norm(grape_ctx* ctx, const grape::LayerIo* io, int64_t step, cud
   });
 }
 
+// defer_stored: with the stored aggregation, leave the sum of the R_i to the fused noise +
+// Adam kernel of run_apply (a one-process step).
 int run_accumulate(grape_ctx* ctx, const void* const* A, const void* const* G, int64_t step,
-                   cudaStream_t st) {
+                   cudaStream_t st, bool defer_stored = false) {
   std::vector<grape::LayerIo> io(ctx->sh.L);
   for (int l = 0; l < ctx->sh.L; ++l) io[l] = grape::LayerIo{A[l], G[l], nullptr};
   const grape::StepShape& sh = ctx->sh;
@@ -282,6 +291,10 @@ int run_accumulate(grape_ctx* ctx, const void* const* A, const void* const* G, i
     return grape::finalize_clip(sh, ctx->partials, ctx->norms, ctx->clip, st);
   });
   if (rc) return rc;
+  if (stored && defer_stored) {
+    ctx->last_step = step;
+    return GRAPE_OK;
+  }
   if (ctx->path == GRAPE_PATH_TC) {
     rc = phase(ctx, GRAPE_PHASE_AGGREGATE, "aggregate", st, [&](int* n) {
       if (stored) return grape::tc_aggregate_stored(sh, ws, ctx->clip, st, n);
@@ -309,23 +322,38 @@ grape::UpdateScalars update_scalars(const grape_ctx* ctx, int64_t step, int64_t 
   return u;
 }
 
-int run_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_total, cudaStream_t st) {
+// fused: the aggregation was deferred (run_accumulate's defer_stored), and this step's
+// noise + Adam kernel sums the stored R_i first.
+int run_apply(grape_ctx* ctx, float* const* W, int64_t step, int64_t batch_total, cudaStream_t st,
+              bool fused = false) {
   const grape::UpdateScalars u = update_scalars(ctx, step, batch_total);
   std::vector<grape::LayerIo> io(ctx->sh.L);
   for (int l = 0; l < ctx->sh.L; ++l) io[l] = grape::LayerIo{nullptr, nullptr, W[l]};
   const bool tc = ctx->path == GRAPE_PATH_TC;
   const grape::StepShape& sh = ctx->sh;
   const grape::LayerWs* ws = ctx->ws.data();
-  int rc = phase(ctx, GRAPE_PHASE_ADAM, "noise + adam", st, [&](int* n) {
-    *n = 1;
-    return grape::noise_adam(sh, ws, u, tc, tc, st);
-  });
+  int rc = fused ? phase(ctx, GRAPE_PHASE_AGGREGATE_ADAM, "aggregate + noise + adam", st,
+                         [&](int* n) { return grape::tc_aggregate_adam(sh, ws, u, ctx->clip, st, n); })
+                 : phase(ctx, GRAPE_PHASE_ADAM, "noise + adam", st, [&](int* n) {
+                     *n = 1;
+                     return grape::noise_adam(sh, ws, u, tc, tc, st);
+                   });
   if (rc) return rc;
   return phase(ctx, GRAPE_PHASE_BACKPROJECT, "back-project", st, [&](int* n) {
     if (tc) return grape::tc_backproject(sh, ws, io.data(), ctx->tc, sh.lr, st, n);
     *n = 1;
     return grape::simt_backproject(sh, ws, io.data(), sh.lr, st);
   });
+}
+
+// One whole step in one process: accumulate, then apply, the stored aggregation fused
+// into noise + Adam where the context does that.
+int run_step(grape_ctx* ctx, const void* const* A, const void* const* G, float* const* W, int64_t step,
+             cudaStream_t st) {
+  const bool fuse = ctx->fuses_adam();
+  int rc = run_accumulate(ctx, A, G, step, st, fuse);
+  if (rc) return rc;
+  return run_apply(ctx, W, step, 0, st, fuse);
 }
 
 // grape_step through a CUDA graph (see StepGraph).  Capture records the same launches as
@@ -371,8 +399,7 @@ int step_graph(grape_ctx* ctx, const void* const* A, const void* const* G, float
     ctx->p_key = -1;   // the graph always contains the generation of P
     cudaError_t e = cudaStreamBeginCapture(ctx->capture_stream, cudaStreamCaptureModeThreadLocal);
     if (e != cudaSuccess) return ctx->cuda_fail(e, "cudaStreamBeginCapture");
-    int rc = run_accumulate(ctx, A, G, step, ctx->capture_stream);
-    if (!rc) rc = run_apply(ctx, W, step, 0, ctx->capture_stream);
+    int rc = run_step(ctx, A, G, W, step, ctx->capture_stream);
     cudaGraph_t graph = nullptr;
     e = cudaStreamEndCapture(ctx->capture_stream, &graph);
     hit->launches = ctx->launches - l0;
@@ -400,7 +427,10 @@ int step_graph(grape_ctx* ctx, const void* const* A, const void* const* G, float
       cudaKernelNodeParams kp{};
       if (cudaGraphKernelNodeGetParams(nd, &kp) != cudaSuccess) continue;
       if (kp.func == gen_fn) hit->gen_p = nd;
-      if (kp.func == grape::noise_adam_func()) hit->adam = nd;
+      if (kp.func == grape::noise_adam_func() || kp.func == grape::tc_aggregate_adam_func()) {
+        hit->adam = nd;
+        hit->adam_fused = kp.func == grape::tc_aggregate_adam_func();
+      }
     }
     if (!hit->gen_p || !hit->adam) {
       ctx->drop_graph(*hit);
@@ -414,8 +444,10 @@ int step_graph(grape_ctx* ctx, const void* const* A, const void* const* G, float
                       ? grape::tc_generate_P_set_node(hit->exec, hit->gen_p, sh, ctx->ws.data(), key)
                       : grape::simt_generate_P_set_node(hit->exec, hit->gen_p, sh, ctx->ws.data(), key);
   if (e == cudaSuccess)
-    e = grape::noise_adam_set_node(hit->exec, hit->adam, sh, ctx->ws.data(), update_scalars(ctx, step, 0),
-                                   ctx->path == GRAPE_PATH_TC);
+    e = hit->adam_fused ? grape::tc_aggregate_adam_set_node(hit->exec, hit->adam, sh, ctx->ws.data(),
+                                                            update_scalars(ctx, step, 0), ctx->clip)
+                        : grape::noise_adam_set_node(hit->exec, hit->adam, sh, ctx->ws.data(),
+                                                     update_scalars(ctx, step, 0), ctx->path == GRAPE_PATH_TC);
   if (e == cudaSuccess) e = cudaGraphLaunch(hit->exec, st);
   if (e != cudaSuccess) return ctx->cuda_fail(e, "graph replay");
   ctx->launches += hit->launches;
@@ -570,6 +602,7 @@ int grape_create(const grape_layer* layers, int32_t n_layers, int32_t r, double 
   // GRAPE_AGG_AUTO: every layer's stored R_i, when the aggregation sums them
   const bool store = auto_stores_R(resolved, T);
   ctx->agg = store ? GRAPE_AGG_STORE : GRAPE_AGG_RECOMPUTE;
+  if (const char* v = std::getenv("GRAPE_FUSE_ADAM")) ctx->fuse_adam = std::strcmp(v, "0") != 0;
   std::vector<size_t> off_rst(n_layers, SIZE_MAX);
   if (store)
     for (int l = 0; l < n_layers; ++l) off_rst[l] = ar.take(static_cast<size_t>(B) * r * layers[l].d_out * 2);
@@ -638,9 +671,7 @@ int grape_step(grape_ctx* ctx, const void* const* A, const void* const* Gout, fl
     return step_graph(ctx, A, Gout, W, step, st);
   }
   const NvtxRange range("grape_step");
-  rc = run_accumulate(ctx, A, Gout, step, st);
-  if (rc) return rc;
-  return run_apply(ctx, W, step, 0, st);
+  return run_step(ctx, A, Gout, W, step, st);
 }
 
 int grape_step_host(grape_ctx* ctx, const void* const* A_host, const void* const* Gout_host,
@@ -679,9 +710,7 @@ int grape_step_host(grape_ctx* ctx, const void* const* A_host, const void* const
                           cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) return ctx->cuda_fail(e, "host-to-device copy");
   }
-  rc = run_accumulate(ctx, ctx->stage_A.data(), ctx->stage_G.data(), step, st);
-  if (rc) return rc;
-  rc = run_apply(ctx, W, step, 0, st);
+  rc = run_step(ctx, ctx->stage_A.data(), ctx->stage_G.data(), W, step, st);
   if (rc) return rc;
   if (norms_host) {
     cudaError_t e = cudaMemcpyAsync(norms_host, ctx->norms, ctx->sh.B * sizeof(float),
@@ -808,9 +837,7 @@ int grape_step_masked(grape_ctx* ctx, const void* const* A, const void* const* G
                                  ctx->comp_idx, st);
   });
   if (rc) return rc;
-  rc = run_accumulate(ctx, ctx->comp_A.data(), ctx->comp_G.data(), step, st);
-  if (rc) return rc;
-  return run_apply(ctx, W, step, 0, st);
+  return run_step(ctx, ctx->comp_A.data(), ctx->comp_G.data(), W, step, st);
 }
 
 int grape_live_counts(grape_ctx* ctx, int32_t* counts_host) {

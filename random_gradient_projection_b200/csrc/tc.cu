@@ -1868,6 +1868,104 @@ __global__ void __launch_bounds__(256) aggregate_stored_kernel(StoredAggTable t,
   }
 }
 
+// ---- the stored aggregation fused with noise + projected Adam (one-process step) ----
+// S = sum_i c_i R_i, then g = (S + sigma C xi) / batch and the Adam update, per unit of
+// eight consecutive elements of one layer's r x d_out: the same per-element arithmetic,
+// in the same order, as aggregate_stored_kernel followed by noise_adam_kernel (the noise
+// of elements 8e .. 8e+7 is Philox blocks 2e and 2e+1 of the noise stream), so the two
+// forms give the same bits.  S is still written, for grape_debug; what the fusion saves
+// is S's re-read and a launch, and the noise's Philox and Box-Muller work runs under
+// the R_i stream instead of after it.  The unit's m, v and noise, which depend on no
+// kernel of the step, are fetched before griddepcontrol.wait for the first unit.
+struct AggAdamTable {
+  const __nv_bfloat16* R[GRAPE_MAX_LAYERS];   // [B][r][d_out] bf16
+  float* S[GRAPE_MAX_LAYERS];                  // [r][d_out] fp32
+  float* m[GRAPE_MAX_LAYERS];
+  float* v[GRAPE_MAX_LAYERS];
+  __nv_bfloat16* dR[GRAPE_MAX_LAYERS];
+  int64_t begin[GRAPE_MAX_LAYERS + 1];         // first unit of each layer; begin[L] = total
+};
+
+struct AggAdamUnit {
+  float m[8], v[8], xi[8];
+};
+
+__device__ __forceinline__ void agg_adam_load(const StepShape& sh, const AggAdamTable& t, uint32_t step, int l,
+                                              int64_t e, AggAdamUnit& a) {
+  const float4* m4 = reinterpret_cast<const float4*>(t.m[l]) + 2 * e;
+  const float4* v4 = reinterpret_cast<const float4*>(t.v[l]) + 2 * e;
+  const float4 ma = m4[0], mb = m4[1], va = v4[0], vb = v4[1];
+  a.m[0] = ma.x; a.m[1] = ma.y; a.m[2] = ma.z; a.m[3] = ma.w;
+  a.m[4] = mb.x; a.m[5] = mb.y; a.m[6] = mb.z; a.m[7] = mb.w;
+  a.v[0] = va.x; a.v[1] = va.y; a.v[2] = va.z; a.v[3] = va.w;
+  a.v[4] = vb.x; a.v[5] = vb.y; a.v[6] = vb.z; a.v[7] = vb.w;
+  if (sh.sigma_C != 0.0f) {
+    const float4 z0 = gaussian4(sh.seed, static_cast<uint32_t>(l), step, kStreamNoise, static_cast<uint32_t>(2 * e));
+    const float4 z1 =
+        gaussian4(sh.seed, static_cast<uint32_t>(l), step, kStreamNoise, static_cast<uint32_t>(2 * e + 1));
+    a.xi[0] = z0.x; a.xi[1] = z0.y; a.xi[2] = z0.z; a.xi[3] = z0.w;
+    a.xi[4] = z1.x; a.xi[5] = z1.y; a.xi[6] = z1.z; a.xi[7] = z1.w;
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a.xi[k] = 0.0f;
+  }
+}
+
+__global__ void __launch_bounds__(256) aggregate_adam_kernel(StepShape sh, AggAdamTable t, UpdateScalars u,
+                                                             const float* clip) {
+  ptx::griddep_launch_dependents();
+  const int64_t total = t.begin[sh.L];
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t unit = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  int l = 0;
+  AggAdamUnit a;
+  if (unit < total) {
+    while (unit >= t.begin[l + 1]) ++l;
+    agg_adam_load(sh, t, u.step, l, unit - t.begin[l], a);
+  }
+  ptx::griddep_wait();   // R_i from the norm kernel, c_i from the clip kernel
+  const int B = sh.B;
+  for (bool first = true; unit < total; unit += stride, first = false) {
+    while (unit >= t.begin[l + 1]) ++l;   // units only grow, so l only moves forward
+    const int64_t e = unit - t.begin[l];                     // unit within the layer
+    const int64_t n8 = t.begin[l + 1] - t.begin[l];         // units per sample
+    if (!first) agg_adam_load(sh, t, u.step, l, e, a);
+    const uint4* R = reinterpret_cast<const uint4*>(t.R[l]) + e;
+    float S[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    constexpr int kBatch = 8;   // loads in flight per thread
+    int i = 0;
+    for (; i + kBatch <= B; i += kBatch) {
+      uint4 x[kBatch];
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) x[k] = __ldcs(R + static_cast<int64_t>(i + k) * n8);
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) acc_bf16x8(S, x[k], __ldg(clip + i + k));
+    }
+    for (; i < B; ++i) acc_bf16x8(S, __ldcs(R + static_cast<int64_t>(i) * n8), __ldg(clip + i));
+    float4* S4 = reinterpret_cast<float4*>(t.S[l]) + 2 * e;
+    S4[0] = make_float4(S[0], S[1], S[2], S[3]);
+    S4[1] = make_float4(S[4], S[5], S[6], S[7]);
+    const float b1 = sh.beta1, b2 = sh.beta2;
+    const float ob1 = sh.one_minus_beta1, ob2 = sh.one_minus_beta2;
+    float d[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float g = fmaf(sh.sigma_C, a.xi[k], S[k]) * u.inv_batch;
+      a.m[k] = fmaf(b1, a.m[k], ob1 * g);
+      a.v[k] = fmaf(b2, a.v[k], ob2 * g * g);
+      d[k] = (a.m[k] * u.inv_bc1) / (sqrtf(a.v[k] * u.inv_bc2) + sh.eps);
+    }
+    float4* m4 = reinterpret_cast<float4*>(t.m[l]) + 2 * e;
+    float4* v4 = reinterpret_cast<float4*>(t.v[l]) + 2 * e;
+    m4[0] = make_float4(a.m[0], a.m[1], a.m[2], a.m[3]);
+    m4[1] = make_float4(a.m[4], a.m[5], a.m[6], a.m[7]);
+    v4[0] = make_float4(a.v[0], a.v[1], a.v[2], a.v[3]);
+    v4[1] = make_float4(a.v[4], a.v[5], a.v[6], a.v[7]);
+    reinterpret_cast<uint4*>(t.dR[l])[e] = make_uint4(pack_bf16(d[0], d[1]), pack_bf16(d[2], d[3]),
+                                                     pack_bf16(d[4], d[5]), pack_bf16(d[6], d[7]));
+  }
+}
+
 // ---------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------
@@ -2463,6 +2561,60 @@ cudaError_t tc_aggregate_stored(const StepShape& sh, const LayerWs* ws, const fl
   ++*launches;
   return launch_pdl(aggregate_stored_kernel, dim3(static_cast<unsigned>(blocks > 0 ? blocks : 1)), dim3(256), 0,
                     st, t, sh.L, sh.B, clip);
+}
+
+namespace {
+
+AggAdamTable make_agg_adam_table(const StepShape& sh, const LayerWs* ws) {
+  AggAdamTable t{};
+  int64_t at = 0;
+  for (int l = 0; l < sh.L; ++l) {
+    t.R[l] = ws[l].Rst;
+    t.S[l] = ws[l].S;
+    t.m[l] = ws[l].m;
+    t.v[l] = ws[l].v;
+    t.dR[l] = static_cast<__nv_bfloat16*>(ws[l].dR);
+    t.begin[l] = at;
+    at += static_cast<int64_t>(sh.r) * ws[l].d_out / 8;   // r % 128 == 0 on this path
+  }
+  t.begin[sh.L] = at;
+  return t;
+}
+
+// enough 256-thread blocks to fill every SM (8 per SM), never more than there are units
+unsigned agg_adam_blocks(const AggAdamTable& t, int L) {
+  int64_t blocks = (t.begin[L] + 255) / 256;
+  const int64_t fill = static_cast<int64_t>(sm_count()) * 8;
+  blocks = blocks < fill ? blocks : fill;
+  return static_cast<unsigned>(blocks > 0 ? blocks : 1);
+}
+
+}  // namespace
+
+cudaError_t tc_aggregate_adam(const StepShape& sh, const LayerWs* ws, const UpdateScalars& u, const float* clip,
+                              cudaStream_t st, int* launches) {
+  for (int l = 0; l < sh.L; ++l)
+    if (!ws[l].Rst) return cudaErrorInvalidValue;
+  const AggAdamTable t = make_agg_adam_table(sh, ws);
+  ++*launches;
+  return launch_pdl(aggregate_adam_kernel, dim3(agg_adam_blocks(t, sh.L)), dim3(256), 0, st, sh, t, u, clip);
+}
+
+const void* tc_aggregate_adam_func() { return reinterpret_cast<const void*>(aggregate_adam_kernel); }
+
+cudaError_t tc_aggregate_adam_set_node(cudaGraphExec_t exec, cudaGraphNode_t node, const StepShape& sh,
+                                       const LayerWs* ws, const UpdateScalars& u, const float* clip) {
+  cudaKernelNodeParams p{};
+  cudaError_t e = cudaGraphKernelNodeGetParams(node, &p);
+  if (e != cudaSuccess) return e;
+  StepShape a0 = sh;
+  AggAdamTable a1 = make_agg_adam_table(sh, ws);
+  UpdateScalars a2 = u;
+  const float* a3 = clip;
+  void* args[] = {&a0, &a1, &a2, &a3};
+  p.kernelParams = args;
+  p.extra = nullptr;
+  return cudaGraphExecKernelNodeSetParams(exec, node, &p);
 }
 
 namespace {

@@ -63,6 +63,15 @@ cudaError_t tc_clip_scale(const StepShape& sh, const LayerWs* ws, const TcWorksp
 cudaError_t tc_aggregate(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                          const TcWorkspace& tc, const float* clip, cudaStream_t st, int* launches);
 // S = sum_i c_i R_i over the R_i stored by tc_project_norm(store_R = true).
+// The stored aggregation fused with noise + Adam, for a one-process step: S = sum_i
+// c_i R_i (written to ws[l].S), then the update of m, v and dR (bf16) as noise_adam
+// computes it, with the same bits.  The _func / _set_node pair rewrites the captured
+// node's step-dependent arguments on a graph replay.
+cudaError_t tc_aggregate_adam(const StepShape& sh, const LayerWs* ws, const UpdateScalars& u, const float* clip,
+                              cudaStream_t st, int* launches);
+const void* tc_aggregate_adam_func();
+cudaError_t tc_aggregate_adam_set_node(cudaGraphExec_t exec, cudaGraphNode_t node, const StepShape& sh,
+                                       const LayerWs* ws, const UpdateScalars& u, const float* clip);
 cudaError_t tc_aggregate_stored(const StepShape& sh, const LayerWs* ws, const float* clip, cudaStream_t st,
                                 int* launches);
 cudaError_t tc_backproject(const StepShape& sh, const LayerWs* ws, const LayerIo* io,

@@ -38,7 +38,8 @@ EXPORTS = (
 )
 GRAPE_NORM_DIRECT, GRAPE_NORM_GHOST = 0, 1
 GRAPE_AGG_AUTO, GRAPE_AGG_RECOMPUTE, GRAPE_AGG_STORE = 0, 1, 2
-PHASES = ("gen_P", "project", "norm", "clip", "aggregate", "adam", "backproject", "compact")   # GRAPE_N_PHASES
+PHASES = ("gen_P", "project", "norm", "clip", "aggregate", "adam", "backproject", "compact",
+          "aggregate_adam")   # GRAPE_N_PHASES
 
 
 class grape_layer(ctypes.Structure):

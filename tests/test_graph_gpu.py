@@ -53,6 +53,9 @@ CASES = {
     "tc_mlp2_refresh3": (W.scaled(W.get("mlp4x1024"), n_layers=2, B=3, T=64, refresh=3), TC, None),
     "tc_ghost": (W.scaled(W.get("mlp4x1024"), n_layers=2, B=3, T=64), TC,
                  lambda g: g.set_norm_method(grape.GRAPE_NORM_GHOST)),
+    # the stored aggregation: the replayed node is the fused aggregation + noise + Adam
+    "tc_mlp2_stored": (W.scaled(W.get("mlp4x1024"), n_layers=2, B=3, T=64), TC,
+                       lambda g: g.set_aggregation(grape.GRAPE_AGG_STORE)),
     "simt_tiny": (W.get("tiny_f32"), SIMT, None),
 }
 

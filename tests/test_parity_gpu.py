@@ -251,11 +251,18 @@ def test_clipped_norm_bound(path):
     assert (c < 1).any() and (c == 1).any()
 
 
-@pytest.mark.parametrize("path", [SIMT, TC], ids=["simt", "tc"])
-def test_accumulate_apply_equals_step(path):
+@pytest.mark.parametrize("path,agg", [(SIMT, None), (TC, None), (TC, grape.GRAPE_AGG_STORE)],
+                         ids=["simt", "tc", "tc-stored"])
+def test_accumulate_apply_equals_step(path, agg):
+    """The data-parallel split gives the step's bits.  With the stored aggregation a step
+    sums the R_i inside its noise + Adam kernel, and the split keeps the two apart: the
+    same arithmetic in the same order."""
     w = W.scaled(W.get("mlp4x1024"), n_layers=2, B=3, T=32)
     W0 = W.make_weights(w)
     g1, g2 = GrapeStep.for_workload(w, path=path), GrapeStep.for_workload(w, path=path)
+    if agg is not None:
+        g1.set_aggregation(agg)
+        g2.set_aggregation(agg)
     W1 = [torch.from_numpy(x).cuda() for x in W0]
     W2 = [torch.from_numpy(x).cuda() for x in W0]
     for s in range(2):
@@ -266,6 +273,8 @@ def test_accumulate_apply_equals_step(path):
     torch.cuda.synchronize()
     for l in range(w.n_layers):
         assert torch.equal(W1[l], W2[l])
+        for f in ("S", "m", "v", "dR"):
+            assert np.array_equal(getattr(g1, f)(l), getattr(g2, f)(l)), (f, l)
 
 
 @pytest.mark.parametrize("path", [SIMT, TC], ids=["simt", "tc"])
