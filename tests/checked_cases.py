@@ -44,6 +44,19 @@ def main():
         worst = compare(w, lib, run_oracle(w, 2), 2e-2, 2)
         print("checked", name, {k: f"{v:.1e}" for k, v in worst.items()}, flush=True)
 
+    # the norm kernel with (A_i P)^T in TMEM and the fused aggregation + noise + Adam:
+    # stored R_i at T = 512 (the default there), and the ragged T = 130 forced onto it
+    w = W.Workload("r512_T512", ((512, 1024), (1024, 512)), r=512, B=2, T=512, dtype="bf16", C=1.0,
+                   sigma=1.0, steps=2)
+    worst = compare(w, run_library(w, 2, TC), run_oracle(w, 2), 2e-2, 2)
+    print("checked r512_T512", {k: f"{v:.1e}" for k, v in worst.items()}, flush=True)
+    os.environ["GRAPE_NORM_TMEM"] = "1"   # read when a context is created
+    w = CASES["r512_T130"]
+    lib = run_library(w, 2, TC, setup=lambda g: g.set_aggregation(grape.GRAPE_AGG_STORE))
+    del os.environ["GRAPE_NORM_TMEM"]
+    worst = compare(w, lib, run_oracle(w, 2), 2e-2, 2)
+    print("checked r512_T130 stored, TMEM norms", {k: f"{v:.1e}" for k, v in worst.items()}, flush=True)
+
     # ghost norms (T <= 128)
     w = W.scaled(W.get("mlp4x1024"), n_layers=2, B=3, T=100)
     g = GrapeStep.for_workload(w, path=TC)

@@ -1,8 +1,9 @@
 """The bounds-checked build (GRAPE_CHECKED) on the tensor-core path (needs a B200).
 
 tests/checked_cases.py runs in a fresh process with GRAPE_LIB=checked: ragged T and
-d_in, r = 512, two launch groups, the cluster aggregation, ghost norms, a masked step
-and the entry point with static scratch.  Every TMA box must pass its check: a failed
+d_in, r = 512, two launch groups, the cluster aggregation, the norm kernel with
+(A_i P)^T in TMEM and the fused aggregation + Adam, ghost norms, a masked step and the
+entry point with static scratch.  Every TMA box must pass its check: a failed
 check raises from the library (or gives NaN from the static entry point) and fails the
 run, and the results still match the oracle.
 """
