@@ -108,6 +108,9 @@ struct GroupParams {
   float* partials;   // NORM
   float lr;          // BACKPROJ
   int cluster;       // AGGREGATE on a cluster: CTAs per output tile (K split)
+  // tc_project_wide_kernel: the launch's tiles in the order CTAs take them (total_tiles
+  // ints), then each CTA's first position in that order (grid + 1 ints)
+  const int* sched;
   int* err;
 #ifdef GRAPE_CHECKED
   int extA[kMaxGroup][3];   // x, y, z extents of the tensors behind mapA, mapB, mapW
@@ -1544,6 +1547,209 @@ __global__ void __launch_bounds__(kNtThreads, 1) tc_norm_tmem_kernel(const __gri
   }
 }
 
+// ---- the projection in 256-row tiles ------------------------------------------------
+// AP = A P for r >= 256 in tiles of 256 stacked rows x 256 columns of r, K = d_in: two
+// M = 128 MMAs per 16-wide k step, one per 128-row half of the tile, share the P box of
+// the stage.  Against tc_gemm_kernel<PROJECT>'s 128-row tiles, each P block is read from
+// L2 by half as many CTAs: per 128 x 256 unit of output, 128 + 256 (here) instead of
+// 128 + 512 bytes per k.  The two 128 x 256 fp32 accumulators fill TMEM's 512 columns,
+// so the MMAs of a tile wait for the epilogue of the one before; with K = d_in that
+// hand-over is small next to a tile's K loop.
+//
+// Tiles are as long as their layer's d_in, and there are half as many as with 128-row
+// tiles, so a plain round robin over CTAs leaves some CTAs a long tile more than others
+// (on the 7B slice's launch groups, 31 % above the mean).  The host therefore gives each
+// CTA its own list: tiles in descending length, each to the CTA with the least work so
+// far (LPT), about 4 % above the mean; tiles of equal length keep their order, so the
+// column tiles of one row block run side by side and read its rows of A once from DRAM.
+//
+// Warps: 0 and 10 load the ring, alternating stages (A, a step input, before
+// griddepcontrol.wait; P after it); 1 owns TMEM and issues the MMAs; 2-9 are the
+// epilogue (warp w: lane quarter w % 4, 128-row half (w - 2) / 4 of the tile), which
+// writes AP as bf16.
+constexpr int kPwStages = 3;
+constexpr int kPwThreads = 32 * 11;
+constexpr int kPwProducer1 = 10;
+struct PwSmem {
+  static constexpr int kA = kBM * kBK * 2;                 // one 128-row half: 16 KB
+  static constexpr int kStage = 2 * kA + 256 * kBK * 2;    // two halves and P (64 x 256): 64 KB
+  static constexpr int kBarOff = kPwStages * kStage;
+  static constexpr int kBytes = kBarOff + 256 + 1024;      // barriers + alignment slack
+  static_assert(kBytes <= 232448, "exceeds the shared memory of a CTA");
+};
+
+__global__ void __launch_bounds__(kPwThreads, 1) tc_project_wide_kernel(const __grid_constant__ GroupParams p) {
+  using S = PwSmem;
+  constexpr int NS = kPwStages;
+  constexpr uint32_t kIdesc = ptx::idesc_bf16(kBM, 256, false, true);   // A K-major, P N-major
+  static_assert((2 * NS + 2) * 8 + 16 <= 256, "barrier area");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
+  uint64_t* empty = full + NS;
+  uint64_t* accfull = empty + NS;
+  uint64_t* accempty = accfull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto wait = [&](uint64_t* bar, uint32_t parity) {
+    return ptx::mbar_wait_or_abort(bar, parity, kWaitLimitNs, abort_flag);
+  };
+  ptx::griddep_launch_dependents();
+  if (warp == 0 && lane == 0) {
+    *abort_flag = 0;
+    for (int st = 0; st < NS; ++st) {
+      ptx::mbar_init(&full[st], 1);
+      ptx::mbar_init(&empty[st], 1);
+    }
+    ptx::mbar_init(accfull, 1);
+    ptx::mbar_init(accempty, kEpiWarps);
+    ptx::fence_mbar_init();
+    for (int g = 0; g < p.n_layers; ++g) {
+      ptx::prefetch_tmap(&p.mapA[g]);
+      ptx::prefetch_tmap(&p.mapB[g]);
+    }
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // this CTA's tiles: positions [k0, k1) of the launch's schedule
+  const int k0 = p.sched[p.total_tiles + blockIdx.x], k1 = p.sched[p.total_tiles + blockIdx.x + 1];
+
+  if (warp == 0 || warp == kPwProducer1) {
+    // ---------------- TMA producers: stage it is loaded by producer it % 2 ----------------
+    if (lane == 0) {
+      const int pi = warp == 0 ? 0 : 1;
+      const uint64_t polA = ptx::policy_evict_first();   // A is read by the r / 256 column tiles
+      const uint64_t polB = ptx::policy_evict_last();    // P is read by every row tile
+      bool waited = false, ok = true;
+      uint32_t it = 0, issued_end = 0;
+      for (int k = k0; ok && k < k1; ++k) {
+        const TileCoord c = decode_tile(p, p.sched[k], PROJECT);
+        const GroupLayer& L = p.lay[c.g];
+        const int m0 = c.m_t * 2 * kBM;
+        const bool two = m0 + kBM < L.M;   // the second half has rows of A
+        for (int kb = c.kb0; kb < c.kb1; ++kb, ++it) {
+          if (static_cast<int>(it & 1) != pi) continue;
+          const int st = it % NS;
+          const uint32_t use = it / NS;
+          if (use > 0 && !wait(&empty[st], (use - 1) & 1)) {
+            atomicOr(p.err, kErrTimeoutProducer);
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + st * S::kStage;
+          const int kk = kb * kBK;
+          ptx::mbar_arrive_expect_tx(&full[st], (two ? 2 : 1) * S::kA + 256 * kBK * 2);
+          GRAPE_BOX(p.err, p.extA[c.g], 2, kk, m0, 0)
+          ptx::tma_load_2d_hint(sa, &p.mapA[c.g], &full[st], kk, m0, polA);
+          if (two)
+            GRAPE_BOX(p.err, p.extA[c.g], 2, kk, m0 + kBM, 0)
+            ptx::tma_load_2d_hint(sa + S::kA, &p.mapA[c.g], &full[st], kk, m0 + kBM, polA);
+          if (!waited) {
+            ptx::griddep_wait();   // P is generated earlier in the step
+            waited = true;
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            GRAPE_BOX(p.err, p.extB[c.g], 2, c.n_t * 256 + 64 * q, kk, 0)
+            ptx::tma_load_2d_hint(sa + 2 * S::kA + q * 8192, &p.mapB[c.g], &full[st], c.n_t * 256 + 64 * q, kk,
+                                  polB);
+          issued_end = it + 1;
+        }
+      }
+      if (*abort_flag)   // leave none of this thread's loads in flight into shared memory
+        for (uint32_t k = issued_end > NS ? issued_end - NS : 0; k < issued_end; ++k)
+          if (static_cast<int>(k & 1) == pi) ptx::mbar_wait(&full[k % NS], (k / NS) & 1, kDrainLimitNs);
+    }
+  } else if (warp == 1) {
+    // ---------------- UMMA issuer ----------------
+    if (lane == 0) {
+      uint32_t it = 0, tc = 0;
+      bool ok = true;
+      for (int k = k0; ok && k < k1; ++k, ++tc) {
+        const TileCoord c = decode_tile(p, p.sched[k], PROJECT);
+        // the epilogue has the previous tile in registers
+        if (tc > 0 && !wait(accempty, (tc - 1) & 1)) {
+          atomicOr(p.err, kErrTimeoutMma);
+          break;
+        }
+        ptx::tc_fence_after();
+        for (int kb = c.kb0; kb < c.kb1; ++kb, ++it) {
+          const int st = it % NS;
+          if (!wait(&full[st], (it / NS) & 1)) {
+            atomicOr(p.err, kErrTimeoutMma);
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a_base = ptx::smem_u32(smem + st * S::kStage);
+          const uint32_t b_base = a_base + 2 * S::kA;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t bd = ptx::desc_sw128(b_base + k * 2048, 8192, 1024);
+            const uint32_t acc = (kb > c.kb0 || k > 0) ? 1u : 0u;
+            ptx::umma_bf16(tmem, ptx::desc_sw128(a_base + k * 32, 16, 1024), bd, kIdesc, acc);
+            ptx::umma_bf16(tmem + 256, ptx::desc_sw128(a_base + S::kA + k * 32, 16, 1024), bd, kIdesc, acc);
+          }
+          ptx::umma_commit(&empty[st]);
+        }
+        ptx::umma_commit(accfull);
+      }
+    }
+  } else {
+    // ---------------- epilogue: warps 2..9 ----------------
+    const int ew = warp - 2;
+    const int q = warp & 3;          // TMEM lanes (rows of a half) 32q .. 32q+31
+    const int h = ew >> 2;           // 128-row half of the tile: accumulator h
+    uint32_t tc = 0;
+    // The epilogue warps walk every tile even after a failed wait (their waits then
+    // return at once).
+    for (int k = k0; k < k1; ++k, ++tc) {
+      const TileCoord c = decode_tile(p, p.sched[k], PROJECT);
+      const GroupLayer& L = p.lay[c.g];
+      const bool got = wait(accfull, tc & 1);
+      if (!got) atomicOr(p.err, kErrTimeoutEpilogue);
+      ptx::tc_fence_after();
+      const int m = c.m_t * 2 * kBM + h * kBM + q * 32 + lane;
+      __nv_bfloat16* AP = static_cast<__nv_bfloat16*>(L.out);
+      const uint32_t tsrc = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 256;
+#pragma unroll 1
+      for (int cc = 0; cc < 256; cc += 64) {
+        float v[64];
+        ptx::tmem_ld64(tsrc + cc, v);
+        if (cc == 192) {   // the whole accumulator is in registers: the next tile may start
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(accempty);
+        }
+        if (got && m < L.M) {
+          uint4* dst = reinterpret_cast<uint4*>(AP + static_cast<size_t>(m) * L.ldo + c.n_t * 256 + cc);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            dst[u] = make_uint4(pack_bf16(v[8 * u + 0], v[8 * u + 1]), pack_bf16(v[8 * u + 2], v[8 * u + 3]),
+                                pack_bf16(v[8 * u + 4], v[8 * u + 5]), pack_bf16(v[8 * u + 6], v[8 * u + 7]));
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
 // ---- aggregation with the K split across a thread-block cluster --------------------
 // For few output tiles (r x d_out is small next to K = B*T): the CS CTAs of a cluster
 // share one 128 x BN output tile of S and each runs 1/CS of the stacked token rows.
@@ -2085,6 +2291,11 @@ struct HostState {
   // can (stored R_i, T <= 512); unset, tc_norm_a_in_tmem decides by T (a measurement
   // and test knob: both kernels compute the same partial slots and R_i)
   int norm_tmem = -1;
+  // GRAPE_PROJECT_WIDE=0 at context creation keeps the projection on 128-row tiles
+  // (tc_gemm_kernel<PROJECT>) at every r; by default r >= 256 runs tc_project_wide_kernel
+  bool project_wide = true;
+  std::vector<const int*> sched;   // per launch group: the wide projection's schedule
+  std::vector<int> sched_grid;     // and the grid it was built for
 };
 
 int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
@@ -2239,8 +2450,66 @@ bool tc_supported(int device, const grape_layer* layers, int n_layers, int r, in
 // One slot per 128 x 128 tile of R_i (row block of r, 128 columns of d_out).
 int tc_partials_per_sample(int r, int d_out) { return cdiv(r, kBM) * cdiv(d_out, 128); }
 
-size_t tc_workspace_bytes(const StepShape&, const LayerWs*) {
-  return 256;  // error word
+namespace {
+
+// The wide projection's schedules: one per launch group, sized on the host with no
+// device (grape_context_bytes) for at most kMaxSchedCtas CTAs.
+constexpr int kMaxSchedCtas = 1024;
+
+bool wide_projection(int r) { return r >= 256 && r % 256 == 0; }
+
+int wide_tiles_of_group(const StepShape& sh, int n_layers) {
+  const int64_t rows = static_cast<int64_t>(sh.B) * sh.T;
+  return n_layers * cdiv(rows, 2 * kBM) * (sh.r / 256);
+}
+
+size_t schedule_bytes(const StepShape& sh) {
+  if (!wide_projection(sh.r)) return 0;
+  size_t b = 0;
+  for (int l0 = 0; l0 < sh.L; l0 += kMaxGroup) {
+    const int n = (sh.L - l0) < kMaxGroup ? (sh.L - l0) : kMaxGroup;
+    b += static_cast<size_t>(wide_tiles_of_group(sh, n) + kMaxSchedCtas + 1) * 4;
+  }
+  return (b + 255) & ~size_t(255);
+}
+
+// LPT list scheduling of one launch group's tiles over `grid` CTAs: tiles in descending
+// k-blocks (stable), each to the CTA with the least k-blocks so far (the lowest index on
+// ties); each CTA runs its tiles in the order they were given.  out = the order, then
+// the CTAs' first positions (grid + 1 ints).
+std::vector<int> lpt_schedule(const std::vector<int>& work, int grid) {
+  const int n = static_cast<int>(work.size());
+  std::vector<int> idx(n);
+  for (int t = 0; t < n; ++t) idx[t] = t;
+  std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) { return work[a] > work[b]; });
+  std::vector<std::vector<int>> lists(grid);
+  std::vector<std::pair<int64_t, int>> heap;   // (load, cta), a min-heap
+  for (int b = 0; b < grid; ++b) heap.push_back({0, b});
+  auto cmp = [](const std::pair<int64_t, int>& x, const std::pair<int64_t, int>& y) { return x > y; };
+  std::make_heap(heap.begin(), heap.end(), cmp);
+  for (int t : idx) {
+    std::pop_heap(heap.begin(), heap.end(), cmp);
+    auto& top = heap.back();
+    lists[top.second].push_back(t);
+    top.first += work[t];
+    std::push_heap(heap.begin(), heap.end(), cmp);
+  }
+  std::vector<int> out;
+  out.reserve(n + grid + 1);
+  std::vector<int> begin(grid + 1, 0);
+  for (int b = 0; b < grid; ++b) {
+    begin[b] = static_cast<int>(out.size());
+    out.insert(out.end(), lists[b].begin(), lists[b].end());
+  }
+  begin[grid] = static_cast<int>(out.size());
+  out.insert(out.end(), begin.begin(), begin.end());
+  return out;
+}
+
+}  // namespace
+
+size_t tc_workspace_bytes(const StepShape& sh, const LayerWs*) {
+  return 256 + schedule_bytes(sh);  // error word, then the wide projection's schedules
 }
 
 cudaError_t tc_init(const StepShape& sh, const LayerWs* ws, void* scratch, size_t bytes,
@@ -2252,6 +2521,7 @@ cudaError_t tc_init(const StepShape& sh, const LayerWs* ws, void* scratch, size_
   hs->T = sh.T;
   hs->bn_project = sh.r == 128 ? 128 : 256;
   if (const char* v = std::getenv("GRAPE_NORM_TMEM")) hs->norm_tmem = std::strcmp(v, "0") == 0 ? 0 : 1;
+  if (const char* v = std::getenv("GRAPE_PROJECT_WIDE")) hs->project_wide = std::strcmp(v, "0") != 0;
   char* base = static_cast<char*>(scratch);
   size_t off = 0;
   hs->err = reinterpret_cast<int*>(base + off);
@@ -2282,6 +2552,38 @@ cudaError_t tc_init(const StepShape& sh, const LayerWs* ws, void* scratch, size_
       delete hs;
       return cudaErrorInvalidValue;
     }
+  }
+  if (wide_projection(sh.r)) {
+    // the wide projection's LPT schedules, one per launch group, for the grid it will
+    // launch (one CTA per SM, never more than there are tiles)
+    int per_sm = 0;
+    cudaError_t e = configure_kernel(reinterpret_cast<const void*>(tc_project_wide_kernel), PwSmem::kBytes,
+                                     kPwThreads, &per_sm);
+    if (e != cudaSuccess) {
+      delete hs;
+      return e;
+    }
+    const int ctas = std::min(sm_count() * per_sm, kMaxSchedCtas);
+    const int64_t rows = static_cast<int64_t>(sh.B) * sh.T;
+    char* sb = base + off;
+    for (int l0 = 0; l0 < sh.L; l0 += kMaxGroup) {
+      const int n = (sh.L - l0) < kMaxGroup ? (sh.L - l0) : kMaxGroup;
+      std::vector<int> work;   // k-blocks of each tile, numbered as tc_project numbers them
+      for (int g = 0; g < n; ++g)
+        work.insert(work.end(), static_cast<size_t>(cdiv(rows, 2 * kBM)) * (sh.r / 256),
+                    cdiv(ws[l0 + g].d_in, kBK));
+      const int grid = std::min(ctas, static_cast<int>(work.size()));
+      const std::vector<int> sched = lpt_schedule(work, grid);
+      e = cudaMemcpy(sb, sched.data(), sched.size() * sizeof(int), cudaMemcpyHostToDevice);
+      if (e != cudaSuccess) {
+        delete hs;
+        return e;
+      }
+      hs->sched.push_back(reinterpret_cast<const int*>(sb));
+      hs->sched_grid.push_back(grid);
+      sb += static_cast<size_t>(wide_tiles_of_group(sh, n) + kMaxSchedCtas + 1) * 4;
+    }
+    off += schedule_bytes(sh);
   }
   if (off > bytes) {
     delete hs;
@@ -2348,6 +2650,21 @@ cudaError_t tc_generate_P_set_node(cudaGraphExec_t exec, cudaGraphNode_t node, c
   return cudaGraphExecKernelNodeSetParams(exec, node, &p);
 }
 
+namespace {
+
+// Persistent, on the grid its schedule (gp.sched) was built for at tc_init.
+cudaError_t launch_project_wide(GroupParams& gp, int tiles, int grid, cudaStream_t st, bool pdl) {
+  int per_sm = 0;
+  cudaError_t e = configure_kernel(reinterpret_cast<const void*>(tc_project_wide_kernel), PwSmem::kBytes,
+                                   kPwThreads, &per_sm);
+  if (e != cudaSuccess) return e;
+  gp.total_tiles = tiles;
+  if (tiles <= 0) return cudaSuccess;
+  return launch_maybe_pdl(pdl, tc_project_wide_kernel, dim3(grid), dim3(kPwThreads), PwSmem::kBytes, st, gp);
+}
+
+}  // namespace
+
 cudaError_t tc_project(const StepShape& sh, const LayerWs* ws, const LayerIo* io,
                        const TcWorkspace& tc, cudaStream_t st, int* launches, bool first_in_step) {
   HostState& hs = *static_cast<HostState*>(tc.host_state);
@@ -2377,7 +2694,29 @@ cudaError_t tc_project(const StepShape& sh, const LayerWs* ws, const LayerIo* io
   };
   if (hs.bn_project == 128)
     return run_mode<PROJECT, 128, kStagesProject128>(hs, sh.L, st, launches, fill, gp, !first_in_step);
-  return run_mode<PROJECT, 256, kStagesProject256>(hs, sh.L, st, launches, fill, gp, !first_in_step);
+  if (!hs.project_wide)
+    return run_mode<PROJECT, 256, kStagesProject256>(hs, sh.L, st, launches, fill, gp, !first_in_step);
+  // 256-row tiles (tc_project_wide_kernel)
+  for (int l0 = 0; l0 < sh.L; l0 += kMaxGroup) {
+    const int n = (sh.L - l0) < kMaxGroup ? (sh.L - l0) : kMaxGroup;
+    gp.n_layers = n;
+    int tiles = 0;
+    for (int g = 0; g < n; ++g) {
+      int t = 0;
+      if (!fill(g, l0 + g, &t)) return cudaErrorInvalidValue;
+      GroupLayer& L = gp.lay[g];
+      L.mt = cdiv(rows, 2 * kBM);
+      L.tiles_begin = tiles;
+      tiles += L.mt * L.nt;
+    }
+    const size_t gi = static_cast<size_t>(l0 / kMaxGroup);
+    if (gi >= hs.sched.size()) return cudaErrorInvalidValue;
+    gp.sched = hs.sched[gi];
+    cudaError_t e = launch_project_wide(gp, tiles, hs.sched_grid[gi], st, l0 == 0 ? !first_in_step : true);
+    if (e != cudaSuccess) return e;
+    ++*launches;
+  }
+  return cudaSuccess;
 }
 
 namespace {

@@ -164,6 +164,26 @@ def test_both_norm_kernels_match_oracle_and_each_other(case, monkeypatch):
             assert rel_fro(a["S"][l], b["S"][l]) < 1e-3, (t, l)
 
 
+@pytest.mark.parametrize("case", ["r512_T130", "vit_qkv_down_B3", "r256_T500"])
+def test_projection_kernels_give_the_same_bits(case, monkeypatch):
+    """For r >= 256 the projection runs in 256-row tiles (two 128-row MMAs sharing each P
+    stage); GRAPE_PROJECT_WIDE=0 keeps the 128-row tiles.  Every AP element is the same
+    chain of 128 x 256 x 16 MMAs over the same k order either way, so the two give the
+    same bits, through to W.  The cases have a last tile whose second half is past the
+    stacked rows (r512_T130: 260 rows, vit_qkv_down_B3: 591)."""
+    w, steps = CASES[case]
+    monkeypatch.setenv("GRAPE_PROJECT_WIDE", "0")
+    narrow = run_library(w, steps, TC)
+    monkeypatch.delenv("GRAPE_PROJECT_WIDE")
+    wide = run_library(w, steps, TC)
+    for t in range(steps):
+        assert np.array_equal(narrow["trace"][t]["norms"], wide["trace"][t]["norms"]), t
+        for l in range(w.n_layers):
+            assert np.array_equal(narrow["trace"][t]["S"][l], wide["trace"][t]["S"][l]), (t, l)
+    for l in range(w.n_layers):
+        assert np.array_equal(narrow["W"][l], wide["W"][l]), l
+
+
 def test_auto_aggregation_follows_tokens_per_sample():
     """AUTO stores R_i from T = 256 tokens per sample on; the ghost norm forms no R_i and
     so recomputes; the CUDA-core path refuses STORE."""
