@@ -315,8 +315,9 @@ GRAPE_API int grape_device_bytes(const grape_ctx* ctx, uint64_t* bytes);
 /* The bytes grape_create would allocate for these arguments, computed on the host with no
  * device call: the Adam moments m and v (8 r d_out per layer), every S_l (4 r d_out), dR,
  * the projection scratch P (d_in r) and AP (B T r) per layer, the per-sample norm
- * buffers, and the stored R_i (2 B r d_out per layer) when GRAPE_AGG_AUTO chooses them,
- * each block rounded up to 256 bytes.  grape_enable_compaction and the staging of
+ * buffers, the tensor-core workspace (an error word and, for r >= 256, the projection's
+ * tile schedules, a few ints per 256-row tile), and the stored R_i (2 B r d_out per
+ * layer) when GRAPE_AGG_AUTO chooses them, each block rounded up to 256 bytes.  grape_enable_compaction and the staging of
  * grape_step_host allocate separately.  Errors: as grape_create's argument checks
  * (GRAPE_EINVAL; GRAPE_EUNSUPPORTED for the tensor-core path with fp32 inputs).  It does
  * not check that the device supports the tensor-core path. */

@@ -1,7 +1,9 @@
 // Tensor-core (tcgen05 / TMEM / TMA) path of the DP-GRAPE step for bf16 inputs.
 //
-// The step's dense contractions run as one warp-specialised UMMA kernel
-// template, instantiated four times:
+// The step's four dense contractions (the closing paragraph of "Metodologia: DP-GRAPE"
+// in the technical summary of "Memory-Efficient Differentially Private Training with
+// Gradient Random Projection": per-sample projection, norms for clipping, aggregation,
+// and the projected update of the parameters):
 //
 //   PROJECT    AP   = A P            M = B*T rows, N = r,     K = d_in
 //   NORM       ||R_i||^2, R_i = (A_i P)^T Gout_i
@@ -9,12 +11,21 @@
 //   AGGREGATE  S    = sum_i c_i R_i  M = r,        N = d_out, K = B*T (split-K)
 //   BACKPROJ   W   -= lr P dR        M = d_in,     N = d_out, K = r
 //
-// (the four contractions of the closing paragraph of "Metodologia: DP-GRAPE" in
-// the technical summary of "Memory-Efficient Differentially Private Training
-// with Gradient Random Projection": per-sample projection, norms for clipping,
-// aggregation, and the projected update of the parameters).
+// run on one warp-specialised UMMA kernel template, tc_gemm_kernel<MODE, BN, STAGES>,
+// described below, and on kernels built for the shapes where it is not the fastest:
 //
-// CTA layout (416 threads, one CTA per SM: the runtime places a single CTA of a kernel
+//   tc_project_wide_kernel    PROJECT for r >= 256 in 256-row tiles (two MMAs share
+//                             each P stage), on an LPT tile schedule made on the host
+//   tc_norm_tmem_kernel       NORM with the R_i store for 256 < T <= 512, the block
+//                             of (A_i P)^T resident in TMEM as the MMA's A operand
+//   tc_backproj_tmem_kernel   BACKPROJ for r = 512, the block of P resident in TMEM
+//   tc_agg_cluster_kernel     AGGREGATE with K split over a cluster (few output tiles)
+//
+// and CUDA-core kernels: P's generation (gen_P_bf16_kernel), the clip factors
+// (clip_scale_kernel), the sum of stored R_i alone (aggregate_stored_kernel) or fused
+// with noise + Adam (aggregate_adam_kernel), and the no-allocation entry point's helpers.
+//
+// tc_gemm_kernel's CTA layout (416 threads, one CTA per SM: the runtime places a single CTA of a kernel
 // that allocates TMEM on each SM): four producer warps (0, 10, 11, 12) issue the TMA
 // loads into a ring of shared-memory stages (128-byte swizzle), producer p filling the
 // stages of k-block iterations it = p (mod 4) -- the TMA stream of one issuing thread
