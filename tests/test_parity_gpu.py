@@ -393,12 +393,15 @@ def test_moment_memory_is_projected():
     g.close()
 
 
-@pytest.mark.parametrize("case", ["mlp_tc", "mlp_simt", "tiny_f32", "vit_tc"])
+@pytest.mark.parametrize("case", ["mlp_tc", "mlp_simt", "tiny_f32", "vit_tc", "r512_two_groups"])
 def test_device_bytes_equal_the_host_plan(case):
-    """grape_context_bytes, computed on the host, is what grape_create allocates."""
+    """grape_context_bytes, computed on the host, is what grape_create allocates, including
+    the projection's tile schedules (r >= 256; one per launch group of 16 layers)."""
     w, path = {"mlp_tc": (W.get("mlp4x1024"), TC), "mlp_simt": (W.get("mlp4x1024"), SIMT),
                "tiny_f32": (W.get("tiny_f32"), SIMT),
-               "vit_tc": (W.scaled(W.get("vit_b"), layers=((768, 2304), (3072, 768)), B=3), TC)}[case]
+               "vit_tc": (W.scaled(W.get("vit_b"), layers=((768, 2304), (3072, 768)), B=3), TC),
+               "r512_two_groups": (W.Workload("r512_18", tuple([(512, 256), (1024, 512)] * 9), r=512, B=2,
+                                              T=300, dtype="bf16", C=1.0, sigma=1.0, steps=1), TC)}[case]
     g = GrapeStep.for_workload(w, path=path)
     dt = grape.GRAPE_BF16 if w.dtype == "bf16" else grape.GRAPE_F32
     assert g.device_bytes() == grape.grape_context_bytes(w.layers, w.r, w.B, w.T, dt, path)
