@@ -59,12 +59,39 @@ __device__ __forceinline__ float2 box_muller(uint32_t xa, uint32_t xb) {
   return make_float2(rho * c, rho * s);
 }
 
+// Box-Muller with the special-function unit's log and sine/cosine (__logf,
+// __sincosf), for normals that are rounded to bf16 at once.  The angle is moved into
+// [-pi, pi), where __sincosf is most accurate: theta = 2 pi u2 - pi, and
+// (cos 2 pi u2, sin 2 pi u2) = -(cos theta, sin theta).  Against the exact transform
+// of the same words the error is at most about 1e-3 absolute, reached only where
+// rho is that small (the log's absolute error, about 4e-7 near u1 = 1, under the
+// square root), and a few 1e-6 elsewhere: below bf16's half ulp, 2^-9 of |z|, for
+// all but such tiny values.  That absolute error can make the log of a u1 just below
+// 1 positive, so -2 ln u1 is clamped at 0 before the square root.
+__device__ __forceinline__ float2 box_muller_fast(uint32_t xa, uint32_t xb) {
+  const float u1 = fmaf(static_cast<float>(xa), 0x1p-32f, 0x1p-32f);
+  const float theta = fmaf(static_cast<float>(xb), 0x1.921fb6p-30f, -0x1.921fb6p+1f);
+  const float rho = sqrtf(fmaxf(-2.0f * __logf(u1), 0.0f));
+  float s, c;
+  __sincosf(theta, &s, &c);
+  return make_float2(-rho * c, -rho * s);
+}
+
 // The four normals of block q: elements 4q .. 4q+3.
 __device__ __forceinline__ float4 gaussian4(uint64_t seed, uint32_t layer, uint32_t step,
                                             uint32_t stream, uint32_t q) {
   const uint4 w = philox_block(seed, layer, step, stream, q);
   const float2 a = box_muller(w.x, w.y);
   const float2 b = box_muller(w.z, w.w);
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
+// gaussian4 through box_muller_fast.
+__device__ __forceinline__ float4 gaussian4_fast(uint64_t seed, uint32_t layer, uint32_t step,
+                                                 uint32_t stream, uint32_t q) {
+  const uint4 w = philox_block(seed, layer, step, stream, q);
+  const float2 a = box_muller_fast(w.x, w.y);
+  const float2 b = box_muller_fast(w.z, w.w);
   return make_float4(a.x, a.y, b.x, b.y);
 }
 

@@ -1943,9 +1943,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_agg_cluster_kernel(const __gri
 }
 
 // ---- P_l in bf16, row-major d_in x r: element e = k*r + j ----------------------------
-// A thread unit is Philox block q of one layer (elements 4q .. 4q+3); the units of all
-// layers are numbered back to back (begin[l] .. begin[l+1]) and a grid of a few blocks
-// per SM strides over them, so layers of unequal size keep every SM busy.
+// A thread unit is Philox block q of one layer (elements 4q .. 4q+3), its normals from
+// the special-function unit's log and sine/cosine (gaussian4_fast): the values are
+// rounded to bf16 at once, and the precise functions made the kernel issue-bound on
+// them.  The units of all layers are numbered back to back (begin[l] .. begin[l+1]) and
+// a grid of a few blocks per SM strides over them, so layers of unequal size keep every
+// SM busy.
 struct PTable {
   __nv_bfloat16* P16[GRAPE_MAX_LAYERS];
   int64_t begin[GRAPE_MAX_LAYERS + 1];   // first unit of each layer; begin[L] = total
@@ -1961,8 +1964,8 @@ __global__ void __launch_bounds__(256) gen_P_bf16_kernel(PTable t, uint64_t seed
        u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     while (u >= t.begin[l + 1]) ++l;   // u only grows, so l only moves forward
     const int64_t q = u - t.begin[l];
-    const float4 z = gaussian4(seed, static_cast<uint32_t>(l), step, kStreamProjection,
-                               static_cast<uint32_t>(q));
+    const float4 z = gaussian4_fast(seed, static_cast<uint32_t>(l), step, kStreamProjection,
+                                    static_cast<uint32_t>(q));
     reinterpret_cast<uint2*>(t.P16[l])[q] =
         make_uint2(pack_bf16(z.x * scale, z.y * scale), pack_bf16(z.z * scale, z.w * scale));
   }
@@ -3225,7 +3228,7 @@ void* g_static_ptr[kMaxDevices] = {};
 
 size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
 
-// P of one layer with an explicit Philox layer index.
+// P of one layer with an explicit Philox layer index (the same normals as gen_P_bf16_kernel).
 __global__ void __launch_bounds__(256) gen_P_layer_static_kernel(__nv_bfloat16* P16, int d_in, int r,
                                                                  uint64_t seed, uint32_t layer,
                                                                  uint32_t step) {
@@ -3234,7 +3237,7 @@ __global__ void __launch_bounds__(256) gen_P_layer_static_kernel(__nv_bfloat16* 
   uint2* out = reinterpret_cast<uint2*>(P16);
   for (int64_t q = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; q < nq;
        q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const float4 z = gaussian4(seed, layer, step, kStreamProjection, static_cast<uint32_t>(q));
+    const float4 z = gaussian4_fast(seed, layer, step, kStreamProjection, static_cast<uint32_t>(q));
     out[q] = make_uint2(pack_bf16(z.x * scale, z.y * scale), pack_bf16(z.z * scale, z.w * scale));
   }
 }

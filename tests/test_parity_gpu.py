@@ -42,6 +42,36 @@ def test_gaussian_matches_oracle(n):
     assert rel_fro(got, ref) < 1e-6
 
 
+@pytest.mark.parametrize("layers,r,step", [(((256, 512), (520, 256)), 128, 0),
+                                           (((648, 512), (1024, 256)), 512, 3)],
+                         ids=["r128", "r512_step3"])
+def test_bf16_projection_matches_oracle_element_by_element(layers, r, step):
+    """The tensor-core path draws P_l in bf16 with the special-function unit's log and
+    sine/cosine.  Each element must be the oracle's fp64 N(0, 1/r) value of the same
+    Philox words, up to bf16 rounding (2^-8 of |P|, a bound on the half ulp) plus the
+    intrinsics' error: at most about 1e-3 in z (the log's absolute error near u1 = 1
+    under the square root), so 1e-3 / sqrt(r) in P.  A wrong stream, layer, step or
+    element index, a swapped cosine and sine or a flipped sign misses this by orders of
+    magnitude."""
+    w = W.Workload("p_bf16", layers, r=r, B=2, T=16, dtype="bf16", C=1.0, sigma=0.5,
+                   steps=step + 1)
+    g = GrapeStep.for_workload(w, path=TC)
+    Ws = [torch.from_numpy(x).cuda() for x in W.make_weights(w)]
+    x = W.make_step_inputs(w, step)
+    g.step([to_device(a, w.dtype) for a in x.A], [to_device(a, w.dtype) for a in x.Gout], Ws, step)
+    torch.cuda.synchronize()
+    h = O.Hyper.of(w)
+    for l, (d_in, _) in enumerate(layers):
+        got = g.P(l).astype(np.float64)
+        ref = O.projection_matrix(h.seed, l, h.projection_key(step), d_in, r)
+        bound = 2.0**-8 * np.abs(ref) + 1.01e-3 / np.sqrt(r)
+        err = np.abs(got - ref)
+        print(l, f"max err / bound {np.max(err / bound):.3f}, rel fro {rel_fro(got, ref):.2e}")
+        assert np.all(err <= bound), (l, np.unravel_index(np.argmax(err / bound), err.shape))
+        assert rel_fro(got, ref) < 2.0**-8
+    g.close()
+
+
 # ---------------------------------------------------------------------------------
 # full steps against the oracle
 # ---------------------------------------------------------------------------------
