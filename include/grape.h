@@ -23,7 +23,11 @@
  * Random Numbers: As Easy as 1, 2, 3", SC'11) with key (seed lo, seed hi) and
  * counter (e/4, layer, step, stream), and Box-Muller: words (x0, x1) give
  * elements 4q, 4q+1 (cosine, sine), words (x2, x3) give 4q+2, 4q+3, with
- * u1 = (x_a + 1)/2^32 and u2 = x_b/2^32.
+ * u1 = (x_a + 1)/2^32 and u2 = x_b/2^32.  The normals are fp32, from the precise
+ * logf, sqrtf and sincospif (grape_gaussian, the noise, the CUDA-core path's P),
+ * except the tensor-core path's P, which is rounded to bf16 as it is written
+ * and so takes the special-function unit's log and sine/cosine: at most about
+ * 1e-3 from the exact transform where rho is that small, a few 1e-6 elsewhere.
  *
  * Conventions
  *  - Every device pointer is a CUDA device address on the context's device;
