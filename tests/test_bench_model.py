@@ -40,6 +40,23 @@ def test_phase_work_of_the_tensor_core_path():
     assert bench.phase_work(w, "simt")["gen_P"]["bytes"] == 4 * 512 * 1024
 
 
+def test_phase_work_with_the_stored_aggregation():
+    w = W.get("mlp4x1024")
+    work = bench.phase_work(w, "tc", "store")
+    # each R_i in bf16: B * r * d_out * 2 B = 64 * 128 * 1024 * 2 = 16 MiB per layer
+    r_bytes = 4 * 16 * MIB
+    # the norm phase reads Gout (16 MiB) and AP (2 MiB) and writes the R_i
+    assert work["norm"]["bytes"] == 4 * 18 * MIB + r_bytes
+    assert work["norm"]["flops"] == 4 * 2 * 8192 * 128 * 1024
+    # the aggregation alone: R_i read once, S written (0.5 MiB per layer), no contraction
+    assert work["aggregate"] == {"bytes": r_bytes + 4 * MIB // 2, "flops": 0}
+    # fused with noise + Adam: R_i read, S written, m and v read and written (16 B per
+    # element), dR written in bf16: 128 * 1024 * (4 + 16 + 2) B per layer
+    assert work["aggregate_adam"] == {"bytes": r_bytes + 4 * 128 * 1024 * 22, "flops": 0}
+    # the recomputed aggregation has no fused phase
+    assert "aggregate_adam" not in bench.phase_work(w, "tc")
+
+
 def test_sqnorms_work_counts_both_contractions_and_the_outputs():
     w = W.get("mlp4x1024")
     flops, byts = bench.sqnorms_work(w)
